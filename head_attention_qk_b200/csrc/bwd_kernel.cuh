@@ -1,0 +1,522 @@
+// bwd_kernel.cuh -- deterministic attention backward for sm_100a (bf16).
+//
+// For dO = dL/dO, P = exp(scale * Q K^T - LSE) (LSE from the forward):
+//   dV = P^T dO,   dP = dO V^T,   Delta_i = sum_d dO_id O_id,
+//   dS = P * (dP - Delta),   dQ = scale * dS K,   dK = scale * dS^T Q.
+// RL-Kernel PR #319 ("feat(attention): add strict bitwise ROCm path", What the
+// strict contract costs) shows a deterministic mha_bwd whose workspace grows as
+// O(S^2); here every output tile is owned by one CTA that sums its terms in a
+// fixed order, with no atomics and no S x S buffer:
+//
+//   bwd_delta_kernel  Delta (fp32) from the forward's bf16 O and dO.
+//   bwd_dkdv_kernel   one CTA per (b, kv head, 128-key tile); loops over the
+//                     group's query heads (ascending) and their 128-row query
+//                     tiles (ascending).  Per step, four tcgen05 MMAs:
+//                       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q.
+//   bwd_dq_kernel     one CTA per (b, q head, 128-row query tile); loops over
+//                     KV tiles (ascending).  Per step, three MMAs:
+//                       S = Q K^T, dP = dO V^T, dQ += dS K.
+//
+// Roles: warps 0-3 compute (one TMEM lane / tile row per thread), warp 4 TMA
+// producer, warp 5 MMA issuer and tensor-memory owner.  P and dS are rounded to
+// bf16 before their MMAs; S, dP and the dQ/dK/dV accumulators are fp32.
+#pragma once
+
+#include "fwd_kernel.cuh"
+#include "sm100.cuh"
+
+namespace hattn {
+
+constexpr int kBwdThreads = 192;
+constexpr int kTile = 128;
+constexpr int kTileBytesBf16 = kTile * kHeadDim * 2;     // 32 KB, two 16 KB swizzle halves
+
+struct BwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  int B, Hq, Hkv, Sq, Sk;
+  int causal;
+  float scale;
+  float scale_log2;
+  const float* lse;       // [B,Hq,Sq] natural log
+  const float* delta;     // [B,Hq,Sq]
+  uint16_t* dq;           // [B,Hq,Sq,D] bf16
+  uint16_t* dk;           // [B,Hkv,Sk,D]
+  uint16_t* dv;
+};
+
+enum : int { kSiteBwdKV = 20, kSiteBwdStFull, kSiteBwdStEmpty, kSiteBwdS, kSiteBwdDP, kSiteBwdP, kSiteBwdDone };
+
+// ---------------------------------------------------------------------------- Delta
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                                        float* __restrict__ delta, long long rows) {
+  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + r * kHeadDim) + lane);
+  const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + r * kHeadDim) + lane);
+  auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+  auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
+  float s = lo(a.x) * lo(g.x) + hi(a.x) * hi(g.x) + lo(a.y) * lo(g.y) + hi(a.y) * hi(g.y);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) delta[r] = s;
+}
+
+// Shared helpers --------------------------------------------------------------
+
+// Load one 128 x 128 bf16 tile (two 64-column TMA boxes) of a 3-D tensor map.
+__device__ __forceinline__ void tma_tile_bf16(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int row, int head) {
+  tma_load_3d(dst, m, bar, 0, row, head);
+  tma_load_3d(dst + 16384, m, bar, 64, row, head);
+}
+
+// D (+)= A B^T with both operands K-major bf16 tiles in shared memory (M = N = 128, K = 128).
+__device__ __forceinline__ void mma_tile_ss_kmajor(uint32_t d, uint32_t sa, uint32_t sb, uint32_t acc) {
+  constexpr uint32_t idesc = make_idesc(1, 1, 0, 128, 128);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+    mma_f16_ss(d, make_sdesc(sa + off, 16, 1024), make_sdesc(sb + off, 16, 1024), idesc, (acc || k > 0) ? 1u : 0u);
+  }
+}
+
+// D (+)= A B where A (128 x 128, bf16 pairs) is in tensor memory and B is a
+// shared-memory tile read MN-major: the reduction runs over the tile's rows.
+__device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
+  constexpr uint32_t idesc = make_idesc(1, 1, 1, 128, 128);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    mma_f16_ts(d, a_tmem + k * 8, make_sdesc(sb + k * 2048, 16384, 1024), idesc, (acc || k > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&x)[128]) {
+  uint32_t u[32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    tmem_ld32(taddr + q * 32, u);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[q * 32 + e] = __uint_as_float(u[e]);
+  }
+}
+
+__device__ __forceinline__ void tmem_store_bf16_row128(uint32_t taddr, const float (&x)[128]) {
+  uint32_t u[32];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) u[e] = pack_bf16x2(x[q * 64 + 2 * e], x[q * 64 + 2 * e + 1]);
+    tmem_st32(taddr + q * 32, u);
+  }
+}
+
+// Read a 128-column fp32 TMEM row, scale it and store it as bf16 to global memory.
+__device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, uint16_t* dst, bool store) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t u[32];
+    __syncwarp();
+    tmem_ld32(taddr + q * 32, u);
+    tmem_wait_ld();
+    if (store) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + q * 32);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = pack_bf16x2(__uint_as_float(u[8 * e + 2 * t]) * mul, __uint_as_float(u[8 * e + 2 * t + 1]) * mul);
+        d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- dK / dV
+struct DkdvSmem {
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTileBytesBf16;
+  static constexpr int kQ = kV + kTileBytesBf16;               // 2 stages
+  static constexpr int kDO = kQ + 2 * kTileBytesBf16;          // 2 stages
+  static constexpr int kStats = kDO + 2 * kTileBytesBf16;      // 2 stages x (128 lse2 + 128 delta) fp32
+  static constexpr int kBars = kStats + 2 * 2 * kTile * 4;
+  static constexpr int kBytes = kBars + 16 * 8;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+__device__ __forceinline__ int bwd_first_q_tile(int j, int Sq, int Sk, int causal) {
+  if (!causal) return 0;
+  const int first_q = j * kTile - (Sk - Sq);          // smallest query that sees key j*128
+  return first_q <= 0 ? 0 : first_q / kTile;
+}
+
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+  using L = DkdvSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id(), lane = lane_id();
+
+  const int j = blockIdx.x;                      // key tile
+  const int bkv = blockIdx.y;                    // b * Hkv + kv head
+  const int b = bkv / a.Hkv, kvh = bkv - b * a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int nq = (a.Sq + kTile - 1) / kTile;
+  const int i0 = bwd_first_q_tile(j, a.Sq, a.Sk, a.causal);
+  const int steps = G * (nq - i0);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* st_full = bars + 1;      // [2]
+  uint64_t* st_empty = bars + 3;     // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* acc_done = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, kTile);
+    mbar_init(acc_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384), dP^T / dS^T [384,512)
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * kTileBytesBf16);
+      tma_tile_bf16(smem + L::kK, &a.tm_k, kv_full, j * kTile, bkv);
+      tma_tile_bf16(smem + L::kV, &a.tm_v, kv_full, j * kTile, bkv);
+    }
+    bool ok = true;
+    for (int n = 0; n < steps && ok; ++n) {
+      const int s = n & 1, u = n >> 1;
+      const int g = n / (nq - i0), i = i0 + n % (nq - i0);
+      const int h = kvh * G + g;
+      const int bh = b * a.Hq + h;
+      if (n >= 2) ok = warp_wait(&st_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(&st_full[s], 2 * kTileBytesBf16);
+        tma_tile_bf16(smem + L::kQ + s * kTileBytesBf16, &a.tm_q, &st_full[s], i * kTile, bh);
+        tma_tile_bf16(smem + L::kDO + s * kTileBytesBf16, &a.tm_do, &st_full[s], i * kTile, bh);
+      }
+      float* stats = reinterpret_cast<float*>(smem + L::kStats + s * 2 * kTile * 4);
+      for (int r = lane; r < kTile; r += 32) {
+        const int qi = i * kTile + r;
+        const bool valid = qi < a.Sq;
+        const size_t idx = (size_t)bh * a.Sq + (valid ? qi : 0);
+        stats[r] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
+        stats[kTile + r] = valid ? __ldg(&a.delta[idx]) : 0.f;
+      }
+      mbar_arrive(&st_full[s]);
+    }
+    // drain outstanding loads
+    if (lane == 0) {
+      mbar_wait(kv_full, 0, kSiteBwdKV);
+      for (int n = max(0, steps - 2); n < steps; ++n) mbar_wait(&st_full[n & 1], (n >> 1) & 1, kSiteBwdStFull);
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      bool ok = mbar_wait(kv_full, 0, kSiteBwdKV);
+      for (int n = 0; n < steps && ok; ++n) {
+        const int s = n & 1, u = n >> 1;
+        ok = mbar_wait(&st_full[s], u & 1, kSiteBwdStFull);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(smem + L::kQ + s * kTileBytesBf16);
+        const uint32_t sDO = smem_u32(smem + L::kDO + s * kTileBytesBf16);
+        mma_tile_ss_kmajor(tmem + 256, sK, sQ, 0);        // S^T  = K Q^T
+        mma_commit(s_full);
+        mma_tile_ss_kmajor(tmem + 384, sV, sDO, 0);       // dP^T = V dO^T
+        mma_commit(dp_full);
+        ok = mbar_wait(p_full, n & 1, kSiteBwdP);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO, n > 0);    // dV += P^T dO
+        mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ, n > 0);   // dK += dS^T Q
+        mma_commit(&st_empty[s]);
+      }
+      mma_commit(acc_done);
+      mbar_wait(acc_done, 0, kSiteBwdDone);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- compute (warps 0-3)
+    const int r = threadIdx.x;                       // key row within the tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int kj = j * kTile + r;
+    const float c = a.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < steps && ok; ++n) {
+      const int s = n & 1, u = n >> 1;
+      const int i = i0 + n % (nq - i0);
+      ok = warp_wait(&st_full[s], u & 1, kSiteBwdStFull);
+      if (ok) ok = warp_wait(s_full, n & 1, kSiteBwdS);
+      if (!ok) break;
+      tc_fence_after();
+      const float* stats = reinterpret_cast<const float*>(smem + L::kStats + s * 2 * kTile * 4);
+      float p[128];
+      tmem_load_row128(tmem + lane_base + 256, p);
+      // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
+      const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
+      const bool need_mask = a.causal && (i * kTile < lim);
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        float x = ex2_approx(fmaf(p[e], c, -stats[e]));
+        if (need_mask && i * kTile + e < lim) x = 0.f;
+        p[e] = x;
+      }
+      tmem_store_bf16_row128(tmem + lane_base + 256, p);     // P^T over S^T's first 64 columns
+      __syncwarp();
+      ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t uu[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          tmem_ld32(tmem + lane_base + 384 + q * 32, uu);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - stats[kTile + q * 32 + e];
+        }
+      }
+      tmem_store_bf16_row128(tmem + lane_base + 384, p);     // dS^T over dP^T's first 64 columns
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
+    if (ok) {
+      tc_fence_after();
+      const bool store = kj < a.Sk;
+      const size_t off = ((size_t)bkv * a.Sk + (store ? kj : 0)) * kHeadDim;
+      store_row_bf16(tmem + lane_base + 0, 1.f, a.dv + off, store);
+      store_row_bf16(tmem + lane_base + 128, a.scale, a.dk + off, store);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+// ---------------------------------------------------------------------------- dQ
+struct DqSmem {
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + kTileBytesBf16;
+  static constexpr int kK = kDO + kTileBytesBf16;              // 2 stages
+  static constexpr int kV = kK + 2 * kTileBytesBf16;           // 2 stages
+  static constexpr int kBars = kV + 2 * kTileBytesBf16;
+  static constexpr int kBytes = kBars + 16 * 8;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+  using L = DqSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id(), lane = lane_id();
+
+  const int nq = (a.Sq + kTile - 1) / kTile;
+  const int i = a.causal ? nq - 1 - (int)blockIdx.x : (int)blockIdx.x;   // heaviest first under a mask
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int G = a.Hq / a.Hkv;
+  const int bkv = b * a.Hkv + h / G;
+  int n_kv;
+  if (!a.causal) {
+    n_kv = (a.Sk + kTile - 1) / kTile;
+  } else {
+    const int last_row = min(i * kTile + kTile - 1, a.Sq - 1);
+    n_kv = min(last_row + (a.Sk - a.Sq), a.Sk - 1) / kTile + 1;
+  }
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;
+  uint64_t* dp_full = bars + 10;
+  uint64_t* ds_full = bars + 11;
+  uint64_t* dq_done = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, kTile);
+    mbar_init(dq_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S / dS [0,128), dP [128,256), dQ [256,384)
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * kTileBytesBf16);
+      tma_tile_bf16(smem + L::kQ, &a.tm_q, q_full, i * kTile, bh);
+      tma_tile_bf16(smem + L::kDO, &a.tm_do, q_full, i * kTile, bh);
+      bool ok = true;
+      for (int jj = 0; jj < n_kv && ok; ++jj) {
+        const int s = jj & 1, u = jj >> 1;
+        if (jj >= 2) ok = mbar_wait(&k_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&k_full[s], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kK + s * kTileBytesBf16, &a.tm_k, &k_full[s], jj * kTile, bkv);
+        if (jj >= 2) ok = mbar_wait(&v_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&v_full[s], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kV + s * kTileBytesBf16, &a.tm_v, &v_full[s], jj * kTile, bkv);
+      }
+      mbar_wait(q_full, 0, kSiteBwdKV);
+      for (int jj = max(0, n_kv - 2); jj < n_kv; ++jj) {
+        mbar_wait(&k_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull);
+        mbar_wait(&v_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
+      bool ok = mbar_wait(q_full, 0, kSiteBwdKV);
+      for (int jj = 0; jj < n_kv && ok; ++jj) {
+        const int s = jj & 1, u = jj >> 1;
+        const uint32_t sK = smem_u32(smem + L::kK + s * kTileBytesBf16);
+        const uint32_t sV = smem_u32(smem + L::kV + s * kTileBytesBf16);
+        ok = mbar_wait(&k_full[s], u & 1, kSiteBwdStFull);
+        if (ok) ok = mbar_wait(&v_full[s], u & 1, kSiteBwdStFull);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tile_ss_kmajor(tmem + 0, sQ, sK, 0);          // S  = Q K^T
+        mma_commit(s_full);
+        mma_tile_ss_kmajor(tmem + 128, sDO, sV, 0);       // dP = dO V^T
+        mma_commit(dp_full);
+        mma_commit(&v_empty[s]);
+        ok = mbar_wait(ds_full, jj & 1, kSiteBwdP);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tile_ts_mnmajor(tmem + 256, tmem + 0, sK, jj > 0);   // dQ += dS K
+        mma_commit(&k_empty[s]);
+      }
+      mma_commit(dq_done);
+      mbar_wait(dq_done, 0, kSiteBwdDone);
+    }
+    __syncwarp();
+  } else {
+    const int r = threadIdx.x;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int qi = i * kTile + r;
+    const bool valid = qi < a.Sq;
+    const size_t ridx = (size_t)bh * a.Sq + (valid ? qi : 0);
+    const float lse2 = valid ? __ldg(&a.lse[ridx]) * 1.4426950408889634f : INFINITY;
+    const float dlt = valid ? __ldg(&a.delta[ridx]) : 0.f;
+    const int kv_limit = a.causal ? min(a.Sk - 1, qi + (a.Sk - a.Sq)) : a.Sk - 1;
+    const float c = a.scale_log2;
+    bool ok = true;
+    for (int jj = 0; jj < n_kv && ok; ++jj) {
+      ok = warp_wait(s_full, jj & 1, kSiteBwdS);
+      if (!ok) break;
+      tc_fence_after();
+      float p[128];
+      tmem_load_row128(tmem + lane_base + 0, p);
+      const int kbase = jj * kTile;
+      const bool need_mask = kbase + kTile - 1 > kv_limit;
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        float x = ex2_approx(fmaf(p[e], c, -lse2));
+        if (need_mask && kbase + e > kv_limit) x = 0.f;
+        p[e] = x;
+      }
+      __syncwarp();
+      ok = warp_wait(dp_full, jj & 1, kSiteBwdDP);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t uu[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          tmem_ld32(tmem + lane_base + 128 + q * 32, uu);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
+        }
+      }
+      tmem_store_bf16_row128(tmem + lane_base + 0, p);     // dS over S's first 64 columns
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok) ok = warp_wait(dq_done, 0, kSiteBwdDone);
+    if (ok) {
+      tc_fence_after();
+      store_row_bf16(tmem + lane_base + 256, a.scale, a.dq + ridx * kHeadDim, valid);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+}
+
+// ---------------------------------------------------------------------------- host launch
+bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uint64_t heads);
+
+inline int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                      const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
+                      float scale, bool causal, float* delta, cudaStream_t st) {
+  static bool attr_ok = [] {
+    return cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvSmem::kAlloc) ==
+               cudaSuccess &&
+           cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem::kAlloc) ==
+               cudaSuccess;
+  }();
+  if (!attr_ok) return -5;
+  static thread_local BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return -5;
+  if (!encode_rows(&a.tm_do, dout, false, Sq, (uint64_t)B * Hq)) return -5;
+  if (!encode_rows(&a.tm_k, k, false, Sk, (uint64_t)B * Hkv)) return -5;
+  if (!encode_rows(&a.tm_v, v, false, Sk, (uint64_t)B * Hkv)) return -5;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq; a.Sk = Sk;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.delta = delta;
+  a.dq = reinterpret_cast<uint16_t*>(dq);
+  a.dk = reinterpret_cast<uint16_t*>(dk);
+  a.dv = reinterpret_cast<uint16_t*>(dv);
+  const long long rows = (long long)B * Hq * Sq;
+  bwd_delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(reinterpret_cast<const uint16_t*>(out),
+                                                                reinterpret_cast<const uint16_t*>(dout), delta, rows);
+  bwd_dkdv_kernel<<<dim3((Sk + kTile - 1) / kTile, B * Hkv), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
+  bwd_dq_kernel<<<dim3((Sq + kTile - 1) / kTile, B * Hq), kBwdThreads, DqSmem::kAlloc, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+}  // namespace hattn

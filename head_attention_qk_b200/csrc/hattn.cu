@@ -1,0 +1,238 @@
+// hattn.cu -- host side of libhattn.so: argument checks, TMA descriptor
+// encoding, launch configuration and the extern "C" entry points of hattn.h.
+//
+// The library holds no device memory of its own and never synchronises the
+// host except in attn_get_device_error().  cuTensorMapEncodeTiled is resolved
+// through cudaGetDriverEntryPoint so the library links only the static CUDA
+// runtime and loads on machines without a GPU driver (calls then fail with
+// HATTN_ELAUNCH).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/hattn.h"
+#include "bwd_kernel.cuh"
+#include "fwd_kernel.cuh"
+
+namespace hattn {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename K>
+bool set_smem_attr(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+template <bool kFp8, bool kPartial>
+int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, cudaStream_t st) {
+  using L = FwdSmemLayout<kFp8>;
+  static std::once_flag once;
+  static bool attr_ok = false;
+  std::call_once(once, [] { attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial>, L::kAlloc); });
+  if (!attr_ok) return HATTN_ELAUNCH;
+  dim3 grid(a.n_qpairs, a.B * a.Hq, n_blocks_in_launch);
+  attn_fwd_kernel<kFp8, kPartial><<<grid, kFwdThreads, L::kAlloc, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
+}
+
+int check_common(int B, int Hq, int Hkv, int Sq, int D, float scale) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || D <= 0) return HATTN_EINVAL;
+  if (Hq % Hkv != 0) return HATTN_EINVAL;
+  if (!(scale > 0.f) || scale != scale) return HATTN_EINVAL;
+  if (D != kHeadDim) return HATTN_EUNSUPPORTED;
+  return HATTN_OK;
+}
+
+int check_descales(int dtype, const float* qd, const float* kd, const float* vd) {
+  if (dtype == HATTN_BF16) return (qd || kd || vd) ? HATTN_EINVAL : HATTN_OK;
+  if (dtype == HATTN_E4M3) {
+    return (qd && kd && vd) ? HATTN_OK : HATTN_EINVAL;   // read as 4-byte scalars
+  }
+  return HATTN_EINVAL;
+}
+
+// Guard against 32-bit overflow of grid dimensions and row counts.
+bool sizes_fit(long long B, long long H, long long S) {
+  return B * H <= 65535LL * 1024 && B * H * S < (1LL << 40) && S < (1LL << 30);
+}
+
+}  // namespace
+
+// 3-D view (D, S, heads) of a [.., heads, S, D] tensor, box (box_x, 128 rows, 1 head),
+// 128-byte swizzle.  box_x * elt_bytes == 128.
+bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uint64_t heads) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const uint64_t eb = e4m3 ? 1 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)(kHeadDim * eb), (cuuint64_t)(rows * kHeadDim * eb)};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)kBlockM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace hattn
+
+using namespace hattn;
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+             int Sk, int D, float scale, int causal, int dtype, const float* q_descale, const float* k_descale,
+             const float* v_descale, void* stream) {
+  if (!q || !k || !v || !out || !lse) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if (Sk <= 0) return HATTN_EINVAL;
+  if ((rc = check_descales(dtype, q_descale, k_descale, v_descale))) return rc;
+  if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return HATTN_EALIGN;
+
+  const bool fp8 = dtype == HATTN_E4M3;
+  static thread_local FwdArgs a;   // ~8 KB: kept off the stack
+  memset(&a, 0, sizeof(a));
+  if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+  if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+  if (!encode_rows(&a.tm_v[0], v, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+  a.sk[0] = Sk;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
+  a.causal = causal ? 1 : 0;
+  a.n_qpairs = (Sq + kQTilesPerCta * kBlockM - 1) / (kQTilesPerCta * kBlockM);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
+  a.block_offset = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return fp8 ? launch_fwd<true, false>(a, 1, st) : launch_fwd<false, false>(a, 1, st);
+}
+
+size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0 || D <= 0 || n_blocks <= 0) return 0;
+  return (size_t)n_blocks * (size_t)B * Hq * Sq * ((size_t)D + 1) * sizeof(float);
+}
+
+int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* const* v_blocks, const int* blk_len,
+                      int n_blocks, void* out, float* lse, int B, int Hq, int Hkv, int Sq, int D, float scale,
+                      int dtype, const float* q_descale, const float* k_descale, const float* v_descale,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k_blocks || !v_blocks || !blk_len || !out || !lse || !workspace) return HATTN_EINVAL;
+  if (n_blocks <= 0) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if ((rc = check_descales(dtype, q_descale, k_descale, v_descale))) return rc;
+  if (dtype != HATTN_BF16) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  for (int i = 0; i < n_blocks; ++i) {
+    if (!k_blocks[i] || !v_blocks[i]) return HATTN_EINVAL;
+    if (blk_len[i] <= 0) return HATTN_EUNSUPPORTED;
+    if (!sizes_fit(B, Hkv, blk_len[i])) return HATTN_EUNSUPPORTED;
+    if (!aligned16(k_blocks[i]) || !aligned16(v_blocks[i])) return HATTN_EALIGN;
+  }
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(workspace)) return HATTN_EALIGN;
+  if (workspace_bytes < attn_fwd_kvblocks_workspace_size(B, Hq, Sq, D, n_blocks)) return HATTN_EWORKSPACE;
+
+  const long long rows = (long long)B * Hq * Sq;
+  float* o_parts = reinterpret_cast<float*>(workspace);
+  float* lse_parts = o_parts + (size_t)n_blocks * rows * kHeadDim;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  static thread_local FwdArgs a;
+  for (int first = 0; first < n_blocks; first += kMaxKvBlocks) {
+    const int cnt = n_blocks - first < kMaxKvBlocks ? n_blocks - first : kMaxKvBlocks;
+    memset(&a, 0, sizeof(a));
+    if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    for (int i = 0; i < cnt; ++i) {
+      if (!encode_rows(&a.tm_k[i], k_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
+        return HATTN_ELAUNCH;
+      if (!encode_rows(&a.tm_v[i], v_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
+        return HATTN_ELAUNCH;
+      a.sk[i] = blk_len[first + i];
+    }
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
+    a.causal = 0;
+    a.n_qpairs = (Sq + kQTilesPerCta * kBlockM - 1) / (kQTilesPerCta * kBlockM);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.out = o_parts;
+    a.lse = lse_parts;
+    a.block_offset = first;
+    if ((rc = launch_fwd<false, true>(a, cnt, st))) return rc;
+  }
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  lse_merge_kernel<<<grid, 256, 0, st>>>(o_parts, lse_parts, n_blocks, rows, reinterpret_cast<uint16_t*>(out), lse);
+  return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  return (size_t)B * Hq * Sq * sizeof(float);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if (Sk <= 0) return HATTN_EINVAL;
+  if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return HATTN_EALIGN;
+  if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq)) return HATTN_EWORKSPACE;
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
+                    reinterpret_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_get_device_error(void* stream, int* code_out) {
+  if (!code_out) return HATTN_EINVAL;
+  *code_out = 0;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HATTN_ELAUNCH;
+  int code = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&code, g_device_error, sizeof(int)) != cudaSuccess) return HATTN_ELAUNCH;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return HATTN_ELAUNCH;
+  *code_out = code;
+  return HATTN_OK;
+}
+
+const char* attn_error_string(int code) {
+  switch (code) {
+    case HATTN_OK: return "ok";
+    case HATTN_EINVAL: return "invalid argument";
+    case HATTN_EUNSUPPORTED: return "unsupported request (refused, not approximated)";
+    case HATTN_EALIGN: return "device pointer not 16-byte aligned";
+    case HATTN_EWORKSPACE: return "workspace too small";
+    case HATTN_ELAUNCH: return "CUDA error while encoding or launching";
+    case HATTN_EDEVICE: return "a kernel gave up on a bounded wait";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

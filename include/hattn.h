@@ -1,0 +1,143 @@
+/*
+ * hattn.h -- C ABI of the B200 (sm_100a) fused attention library libhattn.so.
+ *
+ * The library computes scaled-dot-product multi-head attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * together with the per-row log-sum-exp LSE_i = ln sum_j exp(scale * q_i . k_j),
+ * the operation AITER's fmha_v3_fwd performs with return_softmax_lse and
+ * q/k/v descales (AITER PR #2911 "F8 fmha ASM gfx950", Test Result), the
+ * "(out, lse)" attention core with an attention-domain LSE, a fixed block
+ * merge order and a deterministic backward (RL-Kernel PR #319 "feat(attention):
+ * add strict bitwise ROCm path", Summary table), and the block-KV-cache
+ * streaming self-attention of FlashDreams PR #486 "flashdreams.accelerated
+ * API v0", section 1.2 Optimized MHA.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are dense, contiguous, row-major [B, H, S, D] in device memory;
+ *    D (head dim) must be 128.  LSE arrays are fp32 [B, Hq, Sq] in natural log.
+ *  - Grouped KV heads: Hq % Hkv == 0, and query head h reads KV head
+ *    h / (Hq / Hkv).
+ *  - causal != 0 masks key j for query i unless j <= i + (Sk - Sq)
+ *    (bottom-right aligned); it requires Sq <= Sk so every row sees a key.
+ *  - All device pointers must be 16-byte aligned.
+ *  - The caller owns every buffer.  Calls allocate nothing, never synchronise
+ *    the host, and enqueue their kernels on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream), so they may be captured into a CUDA graph.
+ *  - Results are bitwise reproducible: every output element is written by one
+ *    thread block, reductions run in a fixed order, and tile sizes do not depend
+ *    on B, H or the number of SMs, so a row's result does not change with the
+ *    batch it is submitted in or with how many heads are launched.
+ *  - Return value: 0 on success or a negative HATTN_E* code; arguments are
+ *    checked before anything is launched, and unsupported requests are refused,
+ *    never approximated.
+ */
+#ifndef HATTN_H_
+#define HATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define HATTN_API __attribute__((visibility("default")))
+#else
+#define HATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { HATTN_BF16 = 0, HATTN_E4M3 = 1 } hattn_dtype;
+
+enum {
+  HATTN_OK = 0,
+  HATTN_EINVAL = -1,        /* null pointer, size <= 0, Hq % Hkv != 0, scale <= 0,
+                               descales given for bf16 or missing for e4m3 */
+  HATTN_EUNSUPPORTED = -2,  /* D != 128, causal with Sq > Sk, fp8 backward, a zero-length block */
+  HATTN_EALIGN = -3,        /* a device pointer is not 16-byte aligned */
+  HATTN_EWORKSPACE = -4,    /* workspace smaller than the matching *_workspace_size() */
+  HATTN_ELAUNCH = -5,       /* CUDA reported an error when encoding or launching */
+  HATTN_EDEVICE = -6        /* a kernel gave up on a bounded wait (see attn_get_device_error) */
+};
+
+/*
+ * Forward attention (fmha_v3_fwd semantics, AITER PR #2911 Test Result).
+ *   q    [B, Hq,  Sq, D]  bf16, or e4m3fn codes when dtype == HATTN_E4M3
+ *   k, v [B, Hkv, Sk, D]  same element type as q
+ *   out  [B, Hq,  Sq, D]  bf16, written
+ *   lse  [B, Hq,  Sq]     fp32, written
+ *   scale: softmax scale (> 0), e.g. 1/sqrt(D).
+ *   q_descale [B*Hq], k_descale [B*Hkv], v_descale [B*Hkv]: fp32 device arrays
+ *     for e4m3 (the real value of a code x of head (b, h) is x * descale[b*H + h];
+ *     one value per tensor is the case where all entries are equal); all three
+ *     must be NULL for bf16.  Descales must be positive.
+ * Softmax statistics and both matrix products accumulate in fp32.  For e4m3
+ * inputs the probabilities are rounded to fp16 before the P V product.
+ */
+HATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int dtype,
+             const float* q_descale, const float* k_descale, const float* v_descale,
+             void* stream);
+
+/*
+ * Streaming forward over a block KV cache (FlashDreams PR #486 section 1.2;
+ * merge rule from RL-Kernel PR #319 Summary table).  Queries attend, without a
+ * mask, to the concatenation of n_blocks caller-managed KV blocks.  Each block
+ * is computed separately into the workspace as (O_b, LSE_b), then the blocks
+ * are folded in ascending order:
+ *     M = max(L, L_b); w = e^(L - M); w_b = e^(L_b - M);
+ *     L = M + ln(w + w_b); O = (w O + w_b O_b) / (w + w_b),  from (O, L) = (0, -inf).
+ *   q          [B, Hq, Sq, D] bf16 (dtype must be HATTN_BF16 in this version)
+ *   k_blocks, v_blocks: HOST arrays of n_blocks device pointers; block i is
+ *              [B, Hkv, blk_len[i], D] bf16
+ *   blk_len    HOST array of n_blocks lengths, each > 0
+ *   out, lse   as for attn_fwd
+ *   workspace  device buffer of at least attn_fwd_kvblocks_workspace_size() bytes;
+ *              its contents on entry do not matter.
+ */
+HATTN_API int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* const* v_blocks,
+                      const int* blk_len, int n_blocks, void* out, float* lse,
+                      int B, int Hq, int Hkv, int Sq, int D, float scale, int dtype,
+                      const float* q_descale, const float* k_descale, const float* v_descale,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_fwd_kvblocks needs: n_blocks * B*Hq*Sq * (D + 1) * 4. */
+HATTN_API size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks);
+
+/*
+ * Deterministic backward (RL-Kernel PR #319: mha_bwd with deterministic
+ * reduction, dQ/dK/dV bitwise stable across repeats and batch composition).
+ * For dO = dL/dO and P = exp(scale Q K^T - LSE):
+ *     dV = P^T dO;  dP = dO V^T;  Delta_i = sum_d dO_id O_id;
+ *     dS = P * (dP - Delta);  dQ = scale dS K;  dK = scale dS^T Q,
+ * with dK, dV of a KV head summed over its Hq/Hkv query heads in ascending
+ * order.  bf16 only.
+ *   q, out, dout [B, Hq, Sq, D] bf16;  k, v [B, Hkv, Sk, D] bf16;
+ *   lse [B, Hq, Sq] fp32 from attn_fwd on the same inputs;
+ *   dq [B, Hq, Sq, D], dk, dv [B, Hkv, Sk, D] bf16, written;
+ *   workspace: at least attn_bwd_workspace_size() bytes.
+ * Memory is O(S): no Sq x Sk buffer and no atomics.
+ */
+HATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_bwd needs: B*Hq*Sq * 4 (the Delta vector). */
+HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word that
+ * kernels set when a bounded wait gives up (0 = none; 0x100 | site otherwise).
+ * Returns 0, or HATTN_ELAUNCH if CUDA reports an error.  For tests and
+ * diagnostics; it is the one call that blocks the host.
+ */
+HATTN_API int attn_get_device_error(void* stream, int* code_out);
+
+/* Static text for a return code. */
+HATTN_API const char* attn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HATTN_H_ */

@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: the library loads, exports every symbol hattn.h
+declares, sizes its workspaces, and refuses bad requests on the host (fail
+closed) before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def h():
+    from head_attention_qk_b200 import build
+
+    build.build()
+    import head_attention_qk_b200 as pkg
+
+    return pkg
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "hattn.h")).read()
+    return sorted(set(re.findall(r"HATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ("attn_fwd", "attn_fwd_kvblocks", "attn_bwd", "attn_fwd_kvblocks_workspace_size",
+              "attn_bwd_workspace_size", "attn_get_device_error", "attn_error_string"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(h):
+    for s in declared_symbols():
+        assert hasattr(h.lib, s), s
+        assert s in h.EXPORTED
+
+
+def test_workspace_sizes(h):
+    assert h.kvblocks_workspace_size(1, 40, 1560, 128, 21) == 21 * 40 * 1560 * 129 * 4
+    assert h.bwd_workspace_size(2, 32, 2048) == 2 * 32 * 2048 * 4
+    assert h.kvblocks_workspace_size(0, 1, 1, 128, 1) == 0
+
+
+# Fake, never-dereferenced device addresses: every case below is refused by the
+# host checks before any CUDA call.
+A = ctypes.c_void_p(0x10000)
+B_ = ctypes.c_void_p(0x20000)
+MIS = ctypes.c_void_p(0x20008)
+
+
+def fwd(h, q=A, k=A, v=A, out=A, lse=A, B=1, Hq=2, Hkv=2, Sq=128, Sk=128, D=128, scale=0.088, causal=0, dtype=0,
+        qd=None, kd=None, vd=None):
+    return h.lib.attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, dtype, qd, kd, vd, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(lse=None), -1), (dict(B=0), -1), (dict(Sq=0), -1), (dict(Sk=-1), -1),
+    (dict(Hq=3, Hkv=2), -1), (dict(scale=0.0), -1), (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1),
+    (dict(qd=A, kd=A, vd=A), -1),               # descales with bf16
+    (dict(dtype=1), -1),                        # e4m3 without descales
+    (dict(dtype=1, qd=A, kd=A, vd=None), -1),
+    (dict(dtype=7), -1),
+    (dict(D=64), -2), (dict(D=256), -2),        # only head dim 128
+    (dict(causal=1, Sq=300, Sk=200), -2),       # causal rows without any key
+    (dict(q=MIS), -3), (dict(out=MIS), -3), (dict(lse=MIS), -3),
+])
+def test_fwd_fails_closed(h, kw, code):
+    assert fwd(h, **kw) == code
+
+
+def test_kvblocks_fails_closed(h):
+    lib = h.lib
+    kp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    lens = (ctypes.c_int * 2)(100, 0)
+    need = h.kvblocks_workspace_size(1, 2, 64, 128, 2)
+
+    def call(lens=lens, n=2, ws=A, wsb=need, dtype=0, D=128, qd=None):
+        return lib.attn_fwd_kvblocks(A, ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(kp, ctypes.c_void_p),
+                                     ctypes.cast(lens, ctypes.c_void_p), n, A, A, 1, 2, 2, 64, D, 0.088, dtype,
+                                     qd, qd, qd, ws, wsb, None)
+
+    assert call() == -2                                   # a zero-length block
+    ok_lens = (ctypes.c_int * 2)(100, 50)
+    assert call(lens=ok_lens, n=0) == -1
+    assert call(lens=ok_lens, wsb=need - 1) == -4          # workspace too small
+    assert call(lens=ok_lens, ws=MIS) == -3
+    assert call(lens=ok_lens, D=64) == -2
+    assert call(lens=ok_lens, dtype=1, qd=A) == -2         # fp8 block-KV not offered
+
+
+def test_bwd_fails_closed(h):
+    lib = h.lib
+    need = h.bwd_workspace_size(1, 2, 128)
+
+    def call(ws=A, wsb=need, causal=0, Sq=128, Sk=128, D=128, dq=A):
+        return lib.attn_bwd(A, A, A, A, A, A, dq, A, A, 1, 2, 2, Sq, Sk, D, 0.088, causal, ws, wsb, None)
+
+    assert call(wsb=need - 4) == -4
+    assert call(dq=None) == -1
+    assert call(dq=MIS) == -3
+    assert call(D=96) == -2
+    assert call(causal=1, Sq=256, Sk=128) == -2
+
+
+def test_error_strings(h):
+    for c in (0, -1, -2, -3, -4, -5, -6, -99):
+        assert isinstance(h.lib.attn_error_string(c), bytes)
+
+
+def test_binding_refuses_fp32_inputs(h):
+    import torch
+
+    with pytest.raises((TypeError, ValueError)):
+        h.attn_fwd(torch.zeros(1, 1, 8, 128), torch.zeros(1, 1, 8, 128), torch.zeros(1, 1, 8, 128))

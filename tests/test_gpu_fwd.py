@@ -1,0 +1,185 @@
+"""GPU parity of the forward (bf16 and e4m3) against the CPU fp64 oracle, plus
+the bitwise properties: repeat runs, batch composition, head slicing, and
+canary bytes around the outputs.
+
+Bars: bf16 max |dO| <= 2e-2, max |dLSE| <= 1e-3; e4m3 normalised RMS of O
+<= 1e-2 against the oracle on the dequantized inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
+from workloads import Workload, make_fwd_inputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import head_attention_qk_b200 as pkg
+
+    return pkg
+
+
+def cuda(d):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def run_fwd(h, x, causal):
+    ds = {}
+    if x["q"].dtype == torch.float8_e4m3fn:
+        ds = dict(q_descale=x["q_descale"], k_descale=x["k_descale"], v_descale=x["v_descale"])
+    out, lse = h.attn_fwd(x["q"], x["k"], x["v"], causal=causal, **ds)
+    assert h.get_device_error() == 0
+    return out, lse
+
+
+def check_bf16(h, w, rows=None):
+    x_cpu = make_fwd_inputs(w)
+    x = cuda(x_cpu)
+    out, lse = run_fwd(h, x, w.causal)
+    o_ref, lse_ref = oracle_fwd(x_cpu["q"], x_cpu["k"], x_cpu["v"], w.scale, w.causal, rows=rows)
+    e = fwd_errors(out, lse, o_ref, lse_ref, rows)
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+    return e
+
+
+# ------------------------------------------------------------------ small / ragged, full compare
+
+def test_tiny_config(h):
+    check_bf16(h, workloads.get("tiny"))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
+    (1, 1, 1, 1, 1, False),
+    (1, 2, 1, 1, 300, False),
+    (2, 4, 2, 77, 300, False),
+    (1, 2, 2, 300, 77, False),          # Sq > Sk without a mask
+    (2, 4, 1, 257, 513, False),
+    (1, 4, 2, 1000, 1000, True),
+    (2, 2, 2, 129, 1100, True),         # causal, Sq < Sk (bottom-right)
+    (1, 2, 2, 640, 640, True),
+    (1, 40, 40, 600, 512, False),       # cross-attention shape, even head count
+])
+def test_ragged_shapes(h, B, Hq, Hkv, Sq, Sk, causal):
+    w = Workload("ragged", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, seed=100 + Sq + Sk)
+    check_bf16(h, w)
+
+
+def test_llm_config_sampled_rows(h):
+    w = workloads.get("llm_gqa")
+    check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
+
+
+def test_video_config_sampled_rows(h):
+    w = workloads.get("video")
+    check_bf16(h, w, rows=sample_rows(w.Sq, 48, seed=w.seed))
+
+
+def test_cross_attention_long_q_sampled_rows(h):
+    # Sq >> Sk with an even head count (AITER PR #2911, Wan 2.2 cross-attention report)
+    w = Workload("cross", B=1, Hq=40, Hkv=40, Sq=90000, Sk=512, seed=7)
+    check_bf16(h, w, rows=sample_rows(w.Sq, 64, seed=7))
+
+
+# ------------------------------------------------------------------ e4m3
+
+def check_fp8(h, w, rows=None):
+    x_cpu = make_fwd_inputs(w)
+    x = cuda(x_cpu)
+    out, lse = run_fwd(h, x, w.causal)
+    o_ref, lse_ref = oracle_fwd(x_cpu["q"], x_cpu["k"], x_cpu["v"], w.scale, w.causal, rows=rows,
+                                descales=(x_cpu["q_descale"], x_cpu["k_descale"], x_cpu["v_descale"]))
+    e = fwd_errors(out, lse, o_ref, lse_ref, rows)
+    assert e["o_nrms"] <= FP8_NRMS, e
+    assert np.isfinite(e["lse_max_abs"]) and e["lse_max_abs"] < 5e-2, e
+    return e
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
+    (1, 2, 2, 256, 256, False),
+    (2, 4, 2, 333, 517, False),
+    (1, 2, 1, 700, 700, True),
+])
+def test_fp8_small(h, B, Hq, Hkv, Sq, Sk, causal):
+    check_fp8(h, Workload("f8", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, dtype="e4m3", seed=Sq))
+
+
+def test_fp8_config_sampled_rows(h):
+    w = workloads.get("fp8")
+    check_fp8(h, w, rows=sample_rows(w.Sq, 64, seed=w.seed))
+
+
+# ------------------------------------------------------------------ bitwise properties
+
+def test_repeat_runs_are_bitwise_equal(h):
+    w = workloads.get("llm_gqa")
+    x = cuda(make_fwd_inputs(w))
+    o1, l1 = run_fwd(h, x, True)
+    o2, l2 = run_fwd(h, x, True)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
+
+
+def test_batch_composition_is_bitwise_invariant(h):
+    w = workloads.get("llm_gqa")
+    x2 = cuda(make_fwd_inputs(w, B=2))
+    x4 = cuda(make_fwd_inputs(w, B=4))
+    assert torch.equal(x4["q"][:2], x2["q"])                  # same rows by construction
+    o2, l2 = run_fwd(h, x2, True)
+    o4, l4 = run_fwd(h, x4, True)
+    assert torch.equal(o4[:2].view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l4[:2], l2)
+    x1 = {k: v[1:2].contiguous() for k, v in x2.items()}      # one row at a time
+    o1, l1 = run_fwd(h, x1, True)
+    assert torch.equal(o1.view(torch.int16), o2[1:2].view(torch.int16))
+
+
+def test_head_slice_is_bitwise_invariant(h):
+    # a tensor-parallel rank holding query heads 8..15 and their KV heads 2..3
+    w = workloads.get("llm_gqa", B=1)
+    x = cuda(make_fwd_inputs(w, B=1))
+    o, l = run_fwd(h, x, True)
+    xs = {"q": x["q"][:, 8:16].contiguous(), "k": x["k"][:, 2:4].contiguous(), "v": x["v"][:, 2:4].contiguous()}
+    os_, ls = run_fwd(h, xs, True)
+    assert torch.equal(os_.view(torch.int16), o[:, 8:16].view(torch.int16))
+    assert torch.equal(ls, l[:, 8:16])
+
+
+def test_outputs_leave_neighbouring_bytes_untouched(h):
+    w = Workload("canary", B=1, Hq=2, Hkv=2, Sq=200, Sk=333, seed=9)
+    x = cuda(make_fwd_inputs(w))
+    pad = 4096
+    o_buf = torch.full((pad + 2 * 200 * 128 + pad,), -12345, dtype=torch.int16, device="cuda")
+    l_buf = torch.full((pad + 2 * 200 + pad,), float("nan"), dtype=torch.float32, device="cuda")
+    out = o_buf[pad:pad + 2 * 200 * 128].view(torch.bfloat16).view(1, 2, 200, 128)
+    lse = l_buf[pad:pad + 400].view(1, 2, 200)
+    h.attn_fwd(x["q"], x["k"], x["v"], out=out, lse=lse)
+    assert h.get_device_error() == 0
+    assert torch.all(o_buf[:pad] == -12345) and torch.all(o_buf[-pad:] == -12345)
+    assert torch.all(torch.isnan(l_buf[:pad])) and torch.all(torch.isnan(l_buf[-pad:]))
+    assert torch.all(torch.isfinite(lse))
+
+
+def test_closed_forms_on_gpu(h):
+    # identical keys: O = mean(V), LSE = ln Sk + scale q.k; zero queries: LSE = ln Sk
+    Sk = 777
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(1, 2, 130, 128, generator=g).to(torch.bfloat16)
+    k1 = torch.randn(1, 2, 1, 128, generator=g).to(torch.bfloat16)
+    k = k1.expand(1, 2, Sk, 128).contiguous()
+    v = torch.randn(1, 2, Sk, 128, generator=g).to(torch.bfloat16)
+    out, lse = h.attn_fwd(q.cuda(), k.cuda(), v.cuda())
+    scale = 1 / math.sqrt(128)
+    mean_v = v.double().mean(dim=2, keepdim=True)
+    assert (out.double().cpu() - mean_v).abs().max() <= O_MAX_ABS
+    expect = math.log(Sk) + scale * torch.einsum("bhid,bhd->bhi", q.double(), k1[:, :, 0].double())
+    assert (lse.double().cpu() - expect).abs().max() <= LSE_MAX_ABS
+    out0, lse0 = h.attn_fwd(torch.zeros_like(q).cuda(), k.cuda(), v.cuda())
+    assert (lse0.double().cpu() - math.log(Sk)).abs().max() <= LSE_MAX_ABS
