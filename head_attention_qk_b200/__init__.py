@@ -2,17 +2,22 @@
 descales, with LSE), block-KV streaming forward with a fixed-order LSE merge,
 and a deterministic backward.  The kernels live in libhattn.so (built from
 csrc/ by build.py); this package is its ctypes binding.
+
+The binding is loaded on first use of any of its names, so ``build`` can be
+imported before the library exists; using the API without the library raises
+ImportError (there is no fallback).
 """
-from .hattn import (  # noqa: F401
-    BF16,
-    E4M3,
-    EXPORTED,
-    HattnError,
-    attn_bwd,
-    attn_fwd,
-    attn_fwd_kvblocks,
-    bwd_workspace_size,
-    get_device_error,
-    kvblocks_workspace_size,
-    lib,
-)
+_API = ("BF16", "E4M3", "EXPORTED", "NOALLOC_MAX_ROWS", "HattnError", "attn_bwd", "attn_bwd_noalloc", "attn_fwd",
+        "attn_fwd_kvblocks", "bwd_workspace_size", "get_device_error", "kvblocks_workspace_size", "lib")
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import hattn
+
+        return getattr(hattn, name)
+    raise AttributeError(name)
+
+
+def __dir__():
+    return sorted(list(globals()) + list(_API))

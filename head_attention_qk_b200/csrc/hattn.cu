@@ -211,6 +211,54 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
                     reinterpret_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------- allocation-free backward
+// Scratch for attn_bwd_noalloc: the Delta vector (one fp32 per query row) lives
+// in this file-scope device array instead of a caller-provided workspace.
+// Every GPU that loads the library holds it until the process exits.  In host
+// code the name g_noalloc_delta is only a host-side stand-in; the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) float g_noalloc_delta[HATTN_NOALLOC_MAX_ROWS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_delta on the current device, or nullptr.
+float* noalloc_scratch() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_delta) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                     float scale, int causal, void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if (Sk <= 0) return HATTN_EINVAL;
+  if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if ((long long)B * Hq * Sq > (long long)HATTN_NOALLOC_MAX_ROWS) return HATTN_EWORKSPACE;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return HATTN_EALIGN;
+  float* delta = noalloc_scratch();
+  if (!delta) return HATTN_ELAUNCH;
+  // Delta is fully rewritten for every row this call reads, so the array needs
+  // no clearing between calls.
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
 int attn_get_device_error(void* stream, int* code_out) {
   if (!code_out) return HATTN_EINVAL;
   *code_out = 0;

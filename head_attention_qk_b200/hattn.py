@@ -32,6 +32,8 @@ lib.attn_fwd_kvblocks_workspace_size.argtypes = [_i, _i, _i, _i, _i]
 lib.attn_fwd_kvblocks_workspace_size.restype = _sz
 lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]
 lib.attn_bwd.restype = _i
+lib.attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
+lib.attn_bwd_noalloc.restype = _i
 lib.attn_bwd_workspace_size.argtypes = [_i, _i, _i]
 lib.attn_bwd_workspace_size.restype = _sz
 lib.attn_get_device_error.argtypes = [_vp, ctypes.POINTER(_i)]
@@ -41,7 +43,8 @@ lib.attn_error_string.restype = ctypes.c_char_p
 
 BF16, E4M3 = 0, 1
 EXPORTED = ("attn_fwd", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
-            "attn_bwd_workspace_size", "attn_get_device_error", "attn_error_string")
+            "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_error", "attn_error_string")
+NOALLOC_MAX_ROWS = 1 << 22
 
 
 class HattnError(RuntimeError):
@@ -153,6 +156,23 @@ def attn_bwd(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, 
                       B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
                       workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, stream=None):
+    """attn_bwd without a workspace, for callers that may not allocate device
+    scratch; the library's static 16 MiB array holds Delta (B*Hq*Sq <= 2^22)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (lse, "lse"), (dout, "dout")):
+        _require(t, n)
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    rc = lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                              _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _stream(stream))
+    _check(rc, "attn_bwd_noalloc")
     return dq, dk, dv
 
 

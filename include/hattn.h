@@ -126,6 +126,33 @@ HATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* 
 HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
 
 /*
+ * Backward without a workspace argument, for callers that cannot allocate
+ * device memory at call time -- for example a plug-in running inside a host
+ * framework that owns the GPU allocator and its memory budget, or an engine
+ * whose device memory is planned once up front.  (The pages have no
+ * counterpart; this is an interface convenience of this library.)
+ * Same arguments, results and bitwise reproducibility as attn_bwd, minus the
+ * workspace.  The Delta scratch lives in a static device array of
+ * HATTN_NOALLOC_MAX_ROWS floats (16 MiB) that every GPU loading the library
+ * holds until the process exits; this call allocates nothing.
+ *  - B*Hq*Sq must be <= HATTN_NOALLOC_MAX_ROWS, else HATTN_EWORKSPACE and
+ *    nothing is launched.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.  The graph-capture remark at the top of this
+ *    file does not cover this entry point.
+ *  - All calls share the one array: calls that overlap on the GPU (different
+ *    streams, or several host threads) race on it and must be serialised by
+ *    the caller.  Every call rewrites all the rows it reads, so no clearing is
+ *    needed between calls.
+ */
+#define HATTN_NOALLOC_MAX_ROWS (1 << 22)
+HATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word that
  * kernels set when a bounded wait gives up (0 = none; 0x100 | site otherwise).
  * Returns 0, or HATTN_ELAUNCH if CUDA reports an error.  For tests and
