@@ -73,10 +73,12 @@ __device__ __forceinline__ void tma_tile_bf16(uint8_t* dst, const CUtensorMap* m
 // D (+)= A B^T with both operands K-major bf16 tiles in shared memory (M = N = 128, K = 128).
 __device__ __forceinline__ void mma_tile_ss_kmajor(uint32_t d, uint32_t sa, uint32_t sb, uint32_t acc) {
   constexpr uint32_t idesc = make_idesc(1, 1, 0, 128, 128);
+  constexpr uint32_t hi = sdesc_hi(1024);
+  const uint32_t a_lo = sdesc_lo(sa, 16), b_lo = sdesc_lo(sb, 16);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-    mma_f16_ss(d, make_sdesc(sa + off, 16, 1024), make_sdesc(sb + off, 16, 1024), idesc, (acc || k > 0) ? 1u : 0u);
+    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+    mma_f16_ss2(d, a_lo + off, hi, b_lo + off, hi, idesc, (acc || k > 0) ? 1u : 0u);
   }
 }
 
@@ -84,9 +86,11 @@ __device__ __forceinline__ void mma_tile_ss_kmajor(uint32_t d, uint32_t sa, uint
 // shared-memory tile read MN-major: the reduction runs over the tile's rows.
 __device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
   constexpr uint32_t idesc = make_idesc(1, 1, 1, 128, 128);
+  constexpr uint32_t hi = sdesc_hi(1024);
+  const uint32_t b_lo = sdesc_lo(sb, 16384);
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    mma_f16_ts(d, a_tmem + k * 8, make_sdesc(sb + k * 2048, 16384, 1024), idesc, (acc || k > 0) ? 1u : 0u);
+    mma_f16_ts2(d, a_tmem + k * 8, b_lo + k * (2048 >> 4), hi, idesc, (acc || k > 0) ? 1u : 0u);
 }
 
 __device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&x)[128]) {

@@ -23,7 +23,8 @@
 // S0_{j+1} overwrites the columns PV0_j reads its A operand (P0) from; the MMAs
 // of one thread execute in issue order, so PV0_j has consumed P0 first.  A
 // commit after S_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j) it
-// may rescale O_i and overwrite P_i.
+// may rescale O_i and overwrite P_i.  P is written and released in two halves of
+// 64 keys so the P V of the first half can start while the second is computed.
 //
 // Online softmax in base 2: x = s * c with c = scale * log2(e) (fp8: times the
 // q and k descales), p = 2^(x - m), l = sum p.  The running max m is raised
@@ -42,6 +43,25 @@ constexpr int kQTilesPerCta = 2;
 constexpr int kFwdThreads = 384;
 constexpr int kMaxKvBlocks = 32;  // KV-cache blocks per launch of the block-KV forward
 constexpr float kRescaleThreshold = 8.0f;
+// setmaxnreg split: 2 softmax warpgroups at kRegsSoftmax, 1 warpgroup at
+// kRegsOther.  The sum must not exceed the registers the launch holds
+// (registers per thread x 384); the host checks this before every launch, since
+// an increase that cannot be satisfied would wait forever.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsOther = 88;
+constexpr int kRegsNeeded = (2 * kRegsSoftmax + kRegsOther) * 128;
+static_assert(kRegsNeeded <= (65536 / 384) / 8 * 8 * 384, "setmaxnreg split exceeds a 384-thread launch");
+// Of every 8 pairs of softmax elements, this many take the software exp2
+// (FMA pipe) and the rest the MUFU ex2; bf16 MMAs and MUFU are balanced at
+// D = 128, the fp8 QK^T runs at twice the rate, so fp8 moves more to the FMA pipe.
+#ifndef HATTN_POLY_PAIRS_BF16
+#define HATTN_POLY_PAIRS_BF16 2
+#endif
+#ifndef HATTN_POLY_PAIRS_FP8
+#define HATTN_POLY_PAIRS_FP8 4
+#endif
+template <bool kFp8>
+struct PolyShare { static constexpr int kPairs = kFp8 ? HATTN_POLY_PAIRS_FP8 : HATTN_POLY_PAIRS_BF16; };
 
 struct FwdArgs {
   CUtensorMap tm_q;
@@ -63,32 +83,33 @@ struct FwdArgs {
 template <bool kFp8>
 struct FwdSmemLayout {
   static constexpr int kElt = kFp8 ? 1 : 2;
-  static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;      // Q or K tile
-  static constexpr int kStagesK = kFp8 ? 3 : 2;
-  static constexpr int kStagesV = 2;                                 // V as loaded (bf16 / e4m3)
+  static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;      // Q, K or V tile as loaded
+  // One ring holds the K and V tiles in load order K_0, V_0, K_1, V_1, ...; they
+  // are also released in that order (K_j when S1_j completes, V_j when PV1_j
+  // completes), so the producer can run kRing tiles ahead of the MMAs.
+  static constexpr int kRing = kFp8 ? 8 : 5;
+  static_assert(!kFp8 || kRing % 2 == 0, "fp8 ring slots must keep one role (K or V)");
   static constexpr int kStagesV16 = kFp8 ? 2 : 0;                    // fp8: V widened to fp16
   static constexpr int kV16Bytes = kBlockN * kHeadDim * 2;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQTilesPerCta * kTileBytes;
-  static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
-  static constexpr int kV16Off = kVOff + kStagesV * kTileBytes;
+  static constexpr int kRingOff = kQOff + kQTilesPerCta * kTileBytes;
+  static constexpr int kV16Off = kRingOff + kRing * kTileBytes;
   static constexpr int kBarOff = kV16Off + kStagesV16 * kV16Bytes;
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 * kStagesV16 + 6;
+  static constexpr int kNumBars = 1 + 2 * kRing + 2 * kStagesV16 + 8;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
 struct FwdBars {
   uint64_t* q_full;
-  uint64_t* k_full;
-  uint64_t* k_empty;
-  uint64_t* v_full;
-  uint64_t* v_empty;
+  uint64_t* ring_full;   // [kRing]
+  uint64_t* ring_empty;  // [kRing]
   uint64_t* v16_full;
   uint64_t* v16_empty;
-  uint64_t* s_full;   // [2]
-  uint64_t* p_full;   // [2]
-  uint64_t* o_done;   // [2]
+  uint64_t* s_full;   // [2]: S_t ready
+  uint64_t* p_full;   // [2 tiles][2 halves of 64 keys]: P_t,h written (128 arrivals)
+  uint64_t* o_done;   // [2]: last P V of the tile completed
   uint32_t* tmem_slot;
 };
 
@@ -131,29 +152,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   {
     uint64_t* p = bars;
     bb.q_full = p; p += 1;
-    bb.k_full = p; p += L::kStagesK;
-    bb.k_empty = p; p += L::kStagesK;
-    bb.v_full = p; p += L::kStagesV;
-    bb.v_empty = p; p += L::kStagesV;
+    bb.ring_full = p; p += L::kRing;
+    bb.ring_empty = p; p += L::kRing;
     bb.v16_full = p; p += L::kStagesV16;
     bb.v16_empty = p; p += L::kStagesV16;
     bb.s_full = p; p += 2;
-    bb.p_full = p; p += 2;
+    bb.p_full = p; p += 4;
     bb.o_done = p; p += 2;
     bb.tmem_slot = reinterpret_cast<uint32_t*>(p);
   }
 
   if (threadIdx.x == 0) {
     mbar_init(bb.q_full, 1);
-    for (int s = 0; s < L::kStagesK; ++s) { mbar_init(&bb.k_full[s], 1); mbar_init(&bb.k_empty[s], 1); }
-    for (int s = 0; s < L::kStagesV; ++s) {
-      mbar_init(&bb.v_full[s], 1);
-      mbar_init(&bb.v_empty[s], kFp8 ? 64 : 1);    // fp8: released by the 64 widening threads
+    for (int s = 0; s < L::kRing; ++s) {
+      mbar_init(&bb.ring_full[s], 1);
+      // fp8: odd slots always hold V (even ring), released by the 64 widening threads;
+      // every other slot is released by one MMA commit.
+      mbar_init(&bb.ring_empty[s], (kFp8 && (s & 1)) ? 64 : 1);
     }
     for (int s = 0; s < L::kStagesV16; ++s) { mbar_init(&bb.v16_full[s], 64); mbar_init(&bb.v16_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bb.s_full[i], 1);
-      mbar_init(&bb.p_full[i], kBlockM);
+      mbar_init(&bb.p_full[2 * i], kBlockM);
+      mbar_init(&bb.p_full[2 * i + 1], kBlockM);
       mbar_init(&bb.o_done[i], 1);
     }
     fence_barrier_init();
@@ -173,10 +194,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   const uint32_t tmem = *bb.tmem_slot;
 
   uint8_t* sQ = smem + L::kQOff;
-  uint8_t* sK = smem + L::kKOff;
-  uint8_t* sV = smem + L::kVOff;
+  uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sV16 = smem + L::kV16Off;
 
+  // Register split: the launch gives 168 x 384 = 64512 registers.  The
+  // producer / MMA / widening warpgroup (warps 8-11) drops to 64 per thread and
+  // the two softmax warpgroups rise to 216: 2*128*216 + 128*64 = 63488 <= 64512.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsOther) : "memory");
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -191,28 +216,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         for (int x = 0; x < kBoxes; ++x)
           tma_load_3d(sQ + t * L::kTileBytes + x * kBoxBytes, tq, bb.q_full, x * kBoxCols, q_row0 + t * kBlockM, bh);
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int sk_ = j % L::kStagesK, uk = j / L::kStagesK;
-        if (j >= L::kStagesK) ok = mbar_wait(&bb.k_empty[sk_], (uk - 1) & 1, kSiteKEmpty);
+      // sequence n: K_{n/2} for even n, V_{n/2} for odd n
+      for (int n = 0; n < 2 * n_kv && ok; ++n) {
+        const int slot = n % L::kRing, u = n / L::kRing;
+        if (n >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], (u - 1) & 1, kSiteKEmpty);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bb.k_full[sk_], L::kTileBytes);
+        mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
+        const CUtensorMap* tm = (n & 1) ? tv : tk;
         for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(sK + sk_ * L::kTileBytes + x * kBoxBytes, tk, &bb.k_full[sk_], x * kBoxCols, j * kBlockN, kvh);
-        const int sv = j % L::kStagesV, uv = j / L::kStagesV;
-        if (j >= L::kStagesV) ok = mbar_wait(&bb.v_empty[sv], (uv - 1) & 1, kSiteVEmpty);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bb.v_full[sv], L::kTileBytes);
-        for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(sV + sv * L::kTileBytes + x * kBoxBytes, tv, &bb.v_full[sv], x * kBoxCols, j * kBlockN, kvh);
+          tma_load_3d(sRing + slot * L::kTileBytes + x * kBoxBytes, tm, &bb.ring_full[slot], x * kBoxCols,
+                      (n >> 1) * kBlockN, kvh);
       }
       // Drain: every load issued must land before the CTA may exit.
-      const int last = n_kv - 1;
-      if (n_kv > 0) {
-        for (int j = max(0, last - L::kStagesK + 1); j <= last; ++j)
-          mbar_wait(&bb.k_full[j % L::kStagesK], (j / L::kStagesK) & 1, kSiteKFull);
-        for (int j = max(0, last - L::kStagesV + 1); j <= last; ++j)
-          mbar_wait(&bb.v_full[j % L::kStagesV], (j / L::kStagesV) & 1, kSiteVFull);
-      }
+      for (int n = max(0, 2 * n_kv - L::kRing); n < 2 * n_kv; ++n)
+        mbar_wait(&bb.ring_full[n % L::kRing], (n / L::kRing) & 1, kSiteKFull);
       mbar_wait(bb.q_full, 0, kSiteQFull);
     }
     __syncwarp();
@@ -225,72 +242,90 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       constexpr uint32_t kIdescPV = kFp8 ? make_idesc(0, 0, 1, 128, 128) : make_idesc(1, 1, 1, 128, 128);
       constexpr int kQKSteps = kFp8 ? 4 : 8;               // K = 32 (e4m3) or 16 (bf16) per MMA
       constexpr int kQKStepBytes = 32;
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-      const uint32_t sVa = kFp8 ? smem_u32(sV16) : smem_u32(sV);
-      constexpr int kVStageBytes = kFp8 ? L::kV16Bytes : L::kTileBytes;
-      constexpr int kVStages = kFp8 ? L::kStagesV16 : L::kStagesV;
+      const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
+      const uint32_t sV16a = smem_u32(sV16);
 
-      auto issue_qk = [&](int t, int kstage) {
+      // K_j sits in ring slot (2j) % kRing, V_j in (2j+1) % kRing.
+      // Descriptor halves: Q / K tiles K-major (SBO 1024 B), V MN-major (LBO 16 KB
+      // between the two 64-column halves of the head dim, SBO 1024 B).
+      constexpr uint32_t kHi = sdesc_hi(1024);
+      const uint32_t q_lo0 = sdesc_lo(sQa, 16);
+      const uint32_t ring_lo0 = sdesc_lo(sRa, 16);
+      auto issue_qk = [&](int t, int kslot) {
         const uint32_t d = tmem + t * 128;
+        const uint32_t a_lo = q_lo0 + t * (L::kTileBytes >> 4);
+        const uint32_t b_lo = ring_lo0 + kslot * (L::kTileBytes >> 4);
+#pragma unroll
         for (int k = 0; k < kQKSteps; ++k) {
           // bf16: two 64-column swizzle atoms of 16 KB; step k in atom k/4 at byte (k%4)*32.
-          const uint32_t off = kFp8 ? k * kQKStepBytes : (k >> 2) * 16384 + (k & 3) * kQKStepBytes;
-          const uint64_t da = make_sdesc(sQa + t * L::kTileBytes + off, 16, 1024);
-          const uint64_t db = make_sdesc(sKa + kstage * L::kTileBytes + off, 16, 1024);
-          if (kFp8) mma_f8_ss(d, da, db, kIdescQK, k > 0);
-          else mma_f16_ss(d, da, db, kIdescQK, k > 0);
+          const uint32_t off = (kFp8 ? k * kQKStepBytes : (k >> 2) * 16384 + (k & 3) * kQKStepBytes) >> 4;
+          if (kFp8) mma_f8_ss2(d, a_lo + off, kHi, b_lo + off, kHi, kIdescQK, k > 0);
+          else mma_f16_ss2(d, a_lo + off, kHi, b_lo + off, kHi, kIdescQK, k > 0);
         }
       };
-      auto issue_pv = [&](int t, int vstage, uint32_t acc) {
+      // O_t (+)= P_t V for keys [64 half, 64 half + 64): 4 MMAs of 16 keys.
+      auto issue_pv_half = [&](int t, uint32_t vbase, int half, uint32_t acc) {
         const uint32_t d = tmem + 256 + t * 128;
         const uint32_t a = tmem + t * 128;                 // P_t: 64 columns of packed 16-bit pairs
-        for (int k = 0; k < kBlockN / 16; ++k) {
-          // 16 keys per MMA: rows 16k..16k+15 of the V tile = 2048 bytes; the two
-          // 64-column halves of the head dim are 16 KB apart (LBO).
-          const uint64_t db = make_sdesc(sVa + vstage * kVStageBytes + k * 2048, 16384, 1024);
-          mma_f16_ts(d, a + k * 8, db, kIdescPV, (acc || k > 0) ? 1u : 0u);
+        const uint32_t b_lo = sdesc_lo(vbase, 16384);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int k = half * 4 + kk;
+          // 16 keys per MMA: rows 16k..16k+15 of the V tile = 2048 bytes.
+          mma_f16_ts2(d, a + k * 8, b_lo + k * (2048 >> 4), kHi, kIdescPV, (acc || k > 0) ? 1u : 0u);
         }
+      };
+      // Wait for each half of P_t and issue its MMAs.
+      auto pv = [&](int t, uint32_t vbase, int j) -> bool {
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(&bb.p_full[t * 2 + half], j & 1, kSitePFull)) return false;
+          tc_fence_after();
+          issue_pv_half(t, vbase, half, j > 0);
+        }
+        return true;
       };
 
       bool ok = mbar_wait(bb.q_full, 0, kSiteQFull);
-      if (ok && n_kv > 0) ok = mbar_wait(&bb.k_full[0], 0, kSiteKFull);
+      if (ok && n_kv > 0) ok = mbar_wait(&bb.ring_full[0], 0, kSiteKFull);
       if (ok && n_kv > 0) {
         tc_fence_after();
         issue_qk(0, 0);
         mma_commit(&bb.s_full[0]);
         issue_qk(1, 0);
         mma_commit(&bb.s_full[1]);
-        mma_commit(&bb.k_empty[0]);
+        mma_commit(&bb.ring_empty[0]);
       }
       for (int j = 0; j < n_kv && ok; ++j) {
-        const int vs = j % kVStages, uv = j / kVStages;
-        if (kFp8) ok = mbar_wait(&bb.v16_full[vs], uv & 1, kSiteV16Full);
-        else ok = mbar_wait(&bb.v_full[vs], uv & 1, kSiteVFull);
-        if (ok) ok = mbar_wait(&bb.p_full[0], j & 1, kSitePFull);
+        const int nv = 2 * j + 1, vslot = nv % L::kRing;
+        const int vs = j % max(L::kStagesV16, 1), u16 = j / max(L::kStagesV16, 1);
+        uint32_t vbase;
+        if (kFp8) {
+          ok = mbar_wait(&bb.v16_full[vs], u16 & 1, kSiteV16Full);
+          vbase = sV16a + vs * L::kV16Bytes;
+        } else {
+          ok = mbar_wait(&bb.ring_full[vslot], (nv / L::kRing) & 1, kSiteVFull);
+          vbase = sRa + vslot * L::kTileBytes;
+        }
+        if (ok) ok = pv(0, vbase, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, vs, j > 0);
         if (j == n_kv - 1) mma_commit(&bb.o_done[0]);
-        const int jn = j + 1;
-        const int ks = jn % L::kStagesK;
+        const int jn = j + 1, nk = 2 * jn, kslot = nk % L::kRing;
         if (jn < n_kv) {
-          ok = mbar_wait(&bb.k_full[ks], (jn / L::kStagesK) & 1, kSiteKFull);
+          ok = mbar_wait(&bb.ring_full[kslot], (nk / L::kRing) & 1, kSiteKFull);
           if (!ok) break;
           tc_fence_after();
-          issue_qk(0, ks);
+          issue_qk(0, kslot);
           mma_commit(&bb.s_full[0]);
         }
-        ok = mbar_wait(&bb.p_full[1], j & 1, kSitePFull);
+        ok = pv(1, vbase, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, vs, j > 0);
         if (kFp8) mma_commit(&bb.v16_empty[vs]);
-        else mma_commit(&bb.v_empty[vs]);
+        else mma_commit(&bb.ring_empty[vslot]);
         if (j == n_kv - 1) mma_commit(&bb.o_done[1]);
         if (jn < n_kv) {
-          issue_qk(1, ks);
+          issue_qk(1, kslot);
           mma_commit(&bb.s_full[1]);
-          mma_commit(&bb.k_empty[ks]);
+          mma_commit(&bb.ring_empty[kslot]);
         }
       }
       if (!ok) {
@@ -309,12 +344,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       const int t = threadIdx.x - 320;                       // 0..63
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
-        const int sv = j % L::kStagesV, uv = j / L::kStagesV;
+        const int nv = 2 * j + 1, vslot = nv % L::kRing;
         const int s16 = j % max(L::kStagesV16, 1), u16 = j / max(L::kStagesV16, 1);
-        ok = warp_wait(&bb.v_full[sv], uv & 1, kSiteVFull);
+        ok = warp_wait(&bb.ring_full[vslot], (nv / L::kRing) & 1, kSiteVFull);
         if (ok && j >= L::kStagesV16) ok = warp_wait(&bb.v16_empty[s16], (u16 - 1) & 1, kSiteV16Empty);
         if (!ok) break;
-        const uint8_t* src = sV + sv * L::kTileBytes;
+        const uint8_t* src = sRing + vslot * L::kTileBytes;
         uint8_t* dst = sV16 + s16 * L::kV16Bytes;
         // e4m3 tile: row r (key) = 128 bytes, 16-byte chunk c holds head dims [16c, 16c+16),
         // stored at chunk c ^ (r & 7).  fp16 tile: two 64-dim halves of 16 KB; row r of a
@@ -339,10 +374,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(&bb.v16_full[s16]);
-        mbar_arrive(&bb.v_empty[sv]);
+        mbar_arrive(&bb.ring_empty[vslot]);     // this thread is done reading the e4m3 slot
       }
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax) : "memory");
     // ------------------------------------------------------------ softmax groups 0 and 1
     const int tile = warp >> 2;                       // 0 or 1
     const int r = threadIdx.x & 127;                  // row within the tile == TMEM lane
@@ -352,6 +389,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     const int row = q_row0 + tile * kBlockM + r;
     const int kv_limit = args.causal ? min(sk - 1, row + (sk - args.Sq)) : sk - 1;
 
+    constexpr int kPolyPairs = PolyShare<kFp8>::kPairs;
     float c = args.scale_log2;
     float v_scale = 1.f;
     if (kFp8) {
@@ -368,26 +406,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       tc_fence_after();
       float s[128];
       {
-        uint32_t u[32];
+        uint32_t u[128];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32(tS + q * 32, u);
-          tmem_wait_ld();
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[q * 32]));
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[q * 32 + e] = __uint_as_float(u[e]);
-        }
+        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(u[e]);
       }
       const int kbase = j * kBlockN;
-      if (kbase + kBlockN - 1 > kv_limit) {
+      const bool masked = kbase + kBlockN - 1 > kv_limit;
+      if (masked) {
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (kbase + e > kv_limit) s[e] = -INFINITY;
       }
-      __syncwarp();
-      float mx = s[0];
+      // row max: eight independent three-input chains
+      float mx[8];
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
-      const float m_tile = mx * c;                     // -inf if every key of the tile is masked
+      for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+#pragma unroll
+      for (int e = 24; e < 120; e += 16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[e + i], s[e + 8 + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+      const float m_tile = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
       const bool need = m_tile > m + kRescaleThreshold || (m == -INFINITY && m_tile > -INFINITY);
       float f = 1.f;
       if (need) {
@@ -410,29 +454,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         tmem_wait_st();
       }
       const float mneg = (m == -INFINITY) ? 0.f : -m;
-      float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[64];
+      const float2 c2 = make_float2(c, c), mneg2 = make_float2(mneg, mneg);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // Two halves of 64 keys: each half is written to TMEM and released to the
+      // MMA warp as soon as it is ready, so P V can start on keys 0..63.
 #pragma unroll
-      for (int e = 0; e < 128; e += 2) {
-        const float p0 = ex2_approx(fmaf(s[e], c, mneg));
-        const float p1 = ex2_approx(fmaf(s[e + 1], c, mneg));
-        sum0 += p0;
-        sum1 += p1;
-        pk[e >> 1] = kFp8 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
-      }
-      l += sum0 + sum1;
-      {
-        uint32_t u[32];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = pk[q * 32 + e];
-          tmem_st32(tS + q * 32, u);
+        for (int e2 = 0; e2 < 32; ++e2) {
+          const int e = half * 64 + 2 * e2;
+          const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, mneg2);
+          float2 p;
+          if ((e2 & 7) < kPolyPairs) {
+            p = exp2_poly2(x);
+            if (masked) {                               // the polynomial is never exactly 0
+              p.x = kbase + e > kv_limit ? 0.f : p.x;
+              p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
+            }
+          } else {
+            p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          }
+          acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
+          pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
         }
+        __syncwarp();
+        tmem_st32(tS + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bb.p_full[tile * 2 + half]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bb.p_full[tile]);
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a = __fadd2_rn(a01, a23);
+      l += a.x + a.y;
     }
     if (ok) ok = warp_wait(&bb.o_done[tile], 0, kSiteODone);
     if (ok) {

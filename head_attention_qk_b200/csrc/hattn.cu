@@ -50,7 +50,12 @@ int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, cudaStream_t st) {
   using L = FwdSmemLayout<kFp8>;
   static std::once_flag once;
   static bool attr_ok = false;
-  std::call_once(once, [] { attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial>, L::kAlloc); });
+  std::call_once(once, [] {
+    cudaFuncAttributes fa;
+    attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial>, L::kAlloc) &&
+              cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8, kPartial>) == cudaSuccess &&
+              fa.numRegs * kFwdThreads >= kRegsNeeded;   // the setmaxnreg split must fit the launch
+  });
   if (!attr_ok) return HATTN_ELAUNCH;
   dim3 grid(a.n_qpairs, a.B * a.Hq, n_blocks_in_launch);
   attn_fwd_kernel<kFp8, kPartial><<<grid, kFwdThreads, L::kAlloc, st>>>(a);
