@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], 1); }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, kTile);
+    mbar_init(p_full, kTile / 32);   // one arrival per compute warp
     mbar_init(acc_done, 1);
     fence_barrier_init();
   }
@@ -301,7 +301,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       tmem_store_bf16_row128(tmem + lane_base + 384, p);     // dS^T over dP^T's first 64 columns
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
     }
     if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
     if (ok) {
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, kTile);
+    mbar_init(ds_full, kTile / 32);  // one arrival per compute warp
     mbar_init(dq_done, 1);
     fence_barrier_init();
   }
@@ -473,7 +474,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       tmem_store_bf16_row128(tmem + lane_base + 0, p);     // dS over S's first 64 columns
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
     }
     if (ok) ok = warp_wait(dq_done, 0, kSiteBwdDone);
     if (ok) {

@@ -9,7 +9,7 @@
 // CTA layout (384 threads, one CTA per SM):
 //   warps 0-3  softmax group 0: query tile 0 (rows q0 .. q0+127), one row per thread
 //   warps 4-7  softmax group 1: query tile 1 (rows q0+128 .. q0+255)
-//   warp 8     TMA producer: Q once, then K_j / V_j into stage rings
+//   warp 8     TMA producer: Q once, then K_j / V_j into one ring
 //   warp 9     MMA issuer (one thread) and tensor-memory owner
 //   warps 10-11  fp8 only: widen each e4m3 V tile to fp16 in shared memory
 //
@@ -166,15 +166,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     mbar_init(bb.q_full, 1);
     for (int s = 0; s < L::kRing; ++s) {
       mbar_init(&bb.ring_full[s], 1);
-      // fp8: odd slots always hold V (even ring), released by the 64 widening threads;
+      // fp8: odd slots always hold V (even ring), released by the 2 widening warps;
       // every other slot is released by one MMA commit.
-      mbar_init(&bb.ring_empty[s], (kFp8 && (s & 1)) ? 64 : 1);
+      mbar_init(&bb.ring_empty[s], (kFp8 && (s & 1)) ? 2 : 1);
     }
-    for (int s = 0; s < L::kStagesV16; ++s) { mbar_init(&bb.v16_full[s], 64); mbar_init(&bb.v16_empty[s], 1); }
+    for (int s = 0; s < L::kStagesV16; ++s) { mbar_init(&bb.v16_full[s], 2); mbar_init(&bb.v16_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bb.s_full[i], 1);
-      mbar_init(&bb.p_full[2 * i], kBlockM);
-      mbar_init(&bb.p_full[2 * i + 1], kBlockM);
+      // one arrival per softmax warp (elected after __syncwarp), not per thread:
+      // 128 atomic updates of one shared-memory word per half tile would contend
+      // with the MMA thread polling it
+      mbar_init(&bb.p_full[2 * i], kBlockM / 32);
+      mbar_init(&bb.p_full[2 * i + 1], kBlockM / 32);
       mbar_init(&bb.o_done[i], 1);
     }
     fence_barrier_init();
@@ -217,15 +220,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           tma_load_3d(sQ + t * L::kTileBytes + x * kBoxBytes, tq, bb.q_full, x * kBoxCols, q_row0 + t * kBlockM, bh);
       bool ok = true;
       // sequence n: K_{n/2} for even n, V_{n/2} for odd n
+      int slot = 0;
+      uint32_t ph = 0;
       for (int n = 0; n < 2 * n_kv && ok; ++n) {
-        const int slot = n % L::kRing, u = n / L::kRing;
-        if (n >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], (u - 1) & 1, kSiteKEmpty);
+        if (n >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], ph ^ 1u, kSiteKEmpty);
         if (!ok) break;
         mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
         const CUtensorMap* tm = (n & 1) ? tv : tk;
         for (int x = 0; x < kBoxes; ++x)
           tma_load_3d(sRing + slot * L::kTileBytes + x * kBoxBytes, tm, &bb.ring_full[slot], x * kBoxCols,
                       (n >> 1) * kBlockN, kvh);
+        if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
       }
       // Drain: every load issued must land before the CTA may exit.
       for (int n = max(0, 2 * n_kv - L::kRing); n < 2 * n_kv; ++n)
@@ -373,8 +378,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           *reinterpret_cast<uint4*>(rowp + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&bb.v16_full[s16]);
-        mbar_arrive(&bb.ring_empty[vslot]);     // this thread is done reading the e4m3 slot
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bb.v16_full[s16]);
+          mbar_arrive(&bb.ring_empty[vslot]);   // this warp is done reading the e4m3 slot
+        }
       }
     }
   }
@@ -482,7 +490,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         tmem_st32(tS + half * 32, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bb.p_full[tile * 2 + half]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bb.p_full[tile * 2 + half]);
       }
       const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
       const float2 a = __fadd2_rn(a01, a23);
