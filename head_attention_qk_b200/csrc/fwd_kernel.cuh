@@ -52,13 +52,17 @@ constexpr int kRegsOther = 88;
 constexpr int kRegsNeeded = (2 * kRegsSoftmax + kRegsOther) * 128;
 static_assert(kRegsNeeded <= (65536 / 384) / 8 * 8 * 384, "setmaxnreg split exceeds a 384-thread launch");
 // Of every 8 pairs of softmax elements, this many take the software exp2
-// (FMA pipe) and the rest the MUFU ex2; bf16 MMAs and MUFU are balanced at
-// D = 128, the fp8 QK^T runs at twice the rate, so fp8 moves more to the FMA pipe.
+// (FMA pipe) and the rest the MUFU ex2.  MUFU ex2 runs at 16 per clock per SM,
+// exactly the bf16 MMA rate at D = 128, and the fp8 path takes its exponentials
+// as fp16 pairs (two per MUFU operation).  Measured on B200, moving a share to
+// the polynomial (about 9 issue slots per element) did not pay on this kernel,
+// whose softmax is bound by its dependency chain rather than by MUFU, so the
+// default share is 0; the knob stays for other tile shapes.
 #ifndef HATTN_POLY_PAIRS_BF16
-#define HATTN_POLY_PAIRS_BF16 2
+#define HATTN_POLY_PAIRS_BF16 0
 #endif
 #ifndef HATTN_POLY_PAIRS_FP8
-#define HATTN_POLY_PAIRS_FP8 4
+#define HATTN_POLY_PAIRS_FP8 0
 #endif
 template <bool kFp8>
 struct PolyShare { static constexpr int kPairs = kFp8 ? HATTN_POLY_PAIRS_FP8 : HATTN_POLY_PAIRS_BF16; };
@@ -480,11 +484,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
               p.x = kbase + e > kv_limit ? 0.f : p.x;
               p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
             }
+            pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
+          } else if (kFp8) {
+            // fp8 path: P is fp16, so the exponent is taken as fp16 pairs by one
+            // MUFU operation; the row sum adds exactly the fp16 values P V uses.
+            pk[e2] = ex2_f16x2(pack_f16x2(x.x, x.y));
+            p = unpack_f16x2(pk[e2]);
           } else {
             p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            pk[e2] = pack_bf16x2(p.x, p.y);
           }
           acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
-          pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
         }
         __syncwarp();
         tmem_st32(tS + half * 32, pk);
