@@ -94,9 +94,19 @@ __device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem,
 }
 
 __device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&x)[128]) {
-  uint32_t u[32];
+  uint32_t u[128];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[q * 32]));
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
+}
+
+// Same, one 32-column chunk at a time (fewer live registers).
+__device__ __forceinline__ void tmem_load_row128_chunked(uint32_t taddr, float (&x)[128]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
+    uint32_t u[32];
     tmem_ld32(taddr + q * 32, u);
     tmem_wait_ld();
 #pragma unroll
@@ -160,8 +170,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
 
-  const int j = blockIdx.x;                      // key tile
-  const int bkv = blockIdx.y;                    // b * Hkv + kv head
+  // Key tiles are the slow grid index so that, under a causal mask, the tiles
+  // with the most query tiles (small j) are launched first.
+  const int j = blockIdx.y;                      // key tile
+  const int bkv = blockIdx.x;                    // b * Hkv + kv head
   const int b = bkv / a.Hkv, kvh = bkv - b * a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int nq = (a.Sq + kTile - 1) / kTile;
@@ -174,9 +186,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   uint64_t* st_empty = bars + 3;     // [2]
   uint64_t* s_full = bars + 5;
   uint64_t* dp_full = bars + 6;
-  uint64_t* p_full = bars + 7;
+  uint64_t* p_full = bars + 7;       // P^T written
   uint64_t* acc_done = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* ds_full = bars + 9;      // dS^T written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -184,6 +197,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, kTile / 32);   // one arrival per compute warp
+    mbar_init(ds_full, kTile / 32);
     mbar_init(acc_done, 1);
     fence_barrier_init();
   }
@@ -246,10 +260,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         mma_commit(s_full);
         mma_tile_ss_kmajor(tmem + 384, sV, sDO, 0);       // dP^T = V dO^T
         mma_commit(dp_full);
+        // dV needs only P^T, so it runs while the compute warps form dS^T
         ok = mbar_wait(p_full, n & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
         mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO, n > 0);    // dV += P^T dO
+        ok = mbar_wait(ds_full, n & 1, kSiteBwdP);
+        if (!ok) break;
+        tc_fence_after();
         mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ, n > 0);   // dK += dS^T Q
         mma_commit(&st_empty[s]);
       }
@@ -271,38 +289,75 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       if (ok) ok = warp_wait(s_full, n & 1, kSiteBwdS);
       if (!ok) break;
       tc_fence_after();
-      const float* stats = reinterpret_cast<const float*>(smem + L::kStats + s * 2 * kTile * 4);
-      float p[128];
-      tmem_load_row128(tmem + lane_base + 256, p);
+      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + s * 2 * kTile * 4);
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
       const bool need_mask = a.causal && (i * kTile < lim);
+      const float2 c2 = make_float2(c, c);
+      // P^T row as 64 bf16 pairs: the values dV's MMA consumes, reused for dS^T
+      uint32_t pk[64];
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        float x = ex2_approx(fmaf(p[e], c, -stats[e]));
-        if (need_mask && i * kTile + e < lim) x = 0.f;
-        p[e] = x;
-      }
-      tmem_store_bf16_row128(tmem + lane_base + 256, p);     // P^T over S^T's first 64 columns
-      __syncwarp();
-      ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        uint32_t uu[32];
+      for (int q = 0; q < 4; ++q) {
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_base + 256 + q * 32, u);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32(tmem + lane_base + 384 + q * 32, uu);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - stats[kTile + q * 32 + e];
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const int e = q * 32 + 4 * k4;
+          const float4 l4 = lds128(&stats4[e / 4]); // log2-domain LSE of queries e .. e+3 (broadcast)
+          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(u[4 * k4]), __uint_as_float(u[4 * k4 + 1])), c2,
+                                       make_float2(-l4.x, -l4.y));
+          const float2 x1 = __ffma2_rn(make_float2(__uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3])),
+                                       c2, make_float2(-l4.z, -l4.w));
+          float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x), p3 = ex2_approx(x1.y);
+          if (need_mask) {
+            const int q0 = i * kTile + e;
+            p0 = q0 < lim ? 0.f : p0;
+            p1 = q0 + 1 < lim ? 0.f : p1;
+            p2 = q0 + 2 < lim ? 0.f : p2;
+            p3 = q0 + 3 < lim ? 0.f : p3;
+          }
+          pk[e / 2] = pack_bf16x2(p0, p1);
+          pk[e / 2 + 1] = pack_bf16x2(p2, p3);
         }
       }
-      tmem_store_bf16_row128(tmem + lane_base + 384, p);     // dS^T over dP^T's first 64 columns
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) tmem_st32(tmem + lane_base + 256 + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[q * 32]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full);                // P^T over S^T's first 64 columns
+      ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t uu[32];
+        tmem_ld32(tmem + lane_base + 384 + q * 32, uu);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const int e = q * 32 + 4 * k4;
+          const float4 d4 = lds128(&stats4[kTile / 4 + e / 4]);  // Delta of queries e .. e+3
+          const uint32_t w0 = pk[e / 2], w1 = pk[e / 2 + 1];
+          const float2 pa = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
+          const float2 pb = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
+          const float2 a0 = __fmul2_rn(pa, __fadd2_rn(make_float2(__uint_as_float(uu[4 * k4]), __uint_as_float(uu[4 * k4 + 1])),
+                                                      make_float2(-d4.x, -d4.y)));
+          const float2 a1 = __fmul2_rn(pb, __fadd2_rn(make_float2(__uint_as_float(uu[4 * k4 + 2]), __uint_as_float(uu[4 * k4 + 3])),
+                                                      make_float2(-d4.z, -d4.w)));
+          pk[e / 2] = pack_bf16x2(a0.x, a0.y);
+          pk[e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) tmem_st32(tmem + lane_base + 384 + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[q * 32]));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
     }
     if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
     if (ok) {
@@ -520,7 +575,7 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   const long long rows = (long long)B * Hq * Sq;
   bwd_delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(reinterpret_cast<const uint16_t*>(out),
                                                                 reinterpret_cast<const uint16_t*>(dout), delta, rows);
-  bwd_dkdv_kernel<<<dim3((Sk + kTile - 1) / kTile, B * Hkv), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
+  bwd_dkdv_kernel<<<dim3(B * Hkv, (Sk + kTile - 1) / kTile), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
   bwd_dq_kernel<<<dim3((Sq + kTile - 1) / kTile, B * Hq), kBwdThreads, DqSmem::kAlloc, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }

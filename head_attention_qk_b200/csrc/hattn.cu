@@ -208,6 +208,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (Sk <= 0) return HATTN_EINVAL;
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
   if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if ((Sk + kTile - 1) / kTile > 65535) return HATTN_EUNSUPPORTED;   // key tiles index the grid's y dimension
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return HATTN_EALIGN;
@@ -252,6 +253,7 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   if (Sk <= 0) return HATTN_EINVAL;
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
   if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if ((Sk + kTile - 1) / kTile > 65535) return HATTN_EUNSUPPORTED;   // key tiles index the grid's y dimension
   if ((long long)B * Hq * Sq > (long long)HATTN_NOALLOC_MAX_ROWS) return HATTN_EWORKSPACE;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* p : ptrs)
