@@ -46,7 +46,8 @@ from workloads import make_bwd_inputs, make_fwd_inputs, make_kvblock_inputs, sam
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-WORKLOAD_NAMES = {"video": "video-DiT self-attention fwd (B1 H40 S32760 D128 bf16, Q/K RMS-norm)",
+WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
+                  "video": "video-DiT self-attention fwd (B1 H40 S32760 D128 bf16, Q/K RMS-norm)",
                   "fp8": "fp8 e4m3 attention fwd (B1 H5 S75600 D128, per-head descales)",
                   "llm_gqa": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16)",
                   "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)"}
@@ -161,11 +162,20 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Maximum of a host scalar over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, steps, seconds_this_rank, world):
+    """Weak scaling: every rank runs `steps` steps of its own units; the job's
+    throughput is all ranks' FLOPs over the slowest rank's time."""
+    slowest = max_over_ranks(seconds_this_rank, world)
+    return world * flops_per_step * steps / slowest / 1e12, slowest
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -173,22 +183,25 @@ def max_over_ranks(x, world):
 class Step:
     """One workload: device inputs, a step function and its FLOP count."""
 
-    def __init__(self, name, h, heads=None):
+    def __init__(self, name, h, heads=None, rank=0):
         self.name = name
         self.h = h
         self.w = workloads.get(name)
         if heads:
             self.w = workloads.get(name, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
+        if rank:
+            # weak scaling: each rank attends over its own units (its own seeded draws)
+            self.w = workloads.get(name, seed=self.w.seed + 7919 * rank, Hq=self.w.Hq, Hkv=self.w.Hkv)
         w = self.w
         self.launches = 1
-        if name in ("video", "fp8"):
+        if name in ("video", "fp8", "tiny"):
             x = make_fwd_inputs(w)
             self.host = x
             self.x = {k: v.cuda() for k, v in x.items()}
             self.out = torch.empty((w.B, w.Hq, w.Sq, w.D), dtype=torch.bfloat16, device="cuda")
             self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
             self.flops = w.fwd_flops()
-            self.dtype = "bf16" if name == "video" else "e4m3"
+            self.dtype = "e4m3" if name == "fp8" else "bf16"
         elif name == "llm_gqa":
             x = make_bwd_inputs(w)
             self.host = x
@@ -223,7 +236,7 @@ class Step:
 
     def __call__(self):
         h, w = self.h, self.w
-        if self.name in ("video", "fp8"):
+        if self.name in ("video", "fp8", "tiny"):
             x = self.x
             ds = {}
             if self.name == "fp8":
@@ -344,7 +357,7 @@ def run_reference(args, world, rank):
         return 0
     name = args.workload
     w = workloads.get(name)
-    rows = {"video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64}[name]
+    rows = {"tiny": 256, "video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64}[name]
     vals = []
     for _ in range(args.warmup):
         oracle_sample_tflops(name, rows)
@@ -391,13 +404,12 @@ def main(argv=None):
     torch.cuda.set_device(local)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     name = args.workload
-    step = Step(name, h, heads=args.heads or None)
+    step = Step(name, h, heads=args.heads or None, rank=rank)
     ms, clocks = time_steps(step, args.steps, args.warmup, world, flush,
                             sampler_index=local if rank == 0 else None)
     if h.get_device_error() != 0:
         raise RuntimeError("a kernel reported a bounded-wait timeout")
-    total_s = max_over_ranks(sum(ms) * 1e-3, world)
-    value = world * step.flops * args.steps / total_s / 1e12
+    value, total_s = whole_job_tflops(step.flops, args.steps, sum(ms) * 1e-3, world)
     ms_per_step = total_s * 1e3 / args.steps
 
     fp8 = step.dtype == "e4m3"
@@ -423,7 +435,7 @@ def main(argv=None):
                        "l2": "256 MB write before each timed step, outside its CUDA events"},
             "gpu_launches": step.launches * args.steps,
             "clocks": clocks, "roofline": roofline}
-    if not args.no_e2e and name in ("video", "fp8"):
+    if not args.no_e2e and name in ("video", "fp8", "tiny"):
         e2e = e2e_video_like(step, max(2, args.steps // 2), 1)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world)
         e2e["value"] = world * step.flops / (e2e["ms_per_step"] * 1e-3) / 1e12
@@ -434,7 +446,7 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_sub:
         sub = {}
         for other in WORKLOAD_NAMES:
-            if other == name:
+            if other == name or other == "tiny":
                 continue
             st = Step(other, h)
             oms, _ = time_steps(st, max(3, args.steps // 2), args.warmup, 1, flush)
@@ -451,8 +463,7 @@ def main(argv=None):
         line["sub"] = sub
 
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, dt, desc, cores = oracle_sample_tflops(name, {"video": 256, "fp8": 256, "llm_gqa": 256,
-                                                         "streaming": 256}[name])
+        v, dt, desc, cores = oracle_sample_tflops(name, 256)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
                                 "seconds": dt}
 

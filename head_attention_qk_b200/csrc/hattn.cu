@@ -19,6 +19,21 @@
 
 namespace hattn {
 
+// Failure-detection self-test: one warp waits on a barrier that nothing ever
+// arrives on; the bounded wait must give up after limit_ns, record the site in
+// the error word and let the kernel return normally.
+constexpr int kSiteSelfTest = 0x7F;
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_for(&bar, 0, kSiteSelfTest, limit_ns);
+  __syncwarp();
+}
+
 namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -264,6 +279,12 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   // no clearing between calls.
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_selftest_bounded_wait(void* stream, unsigned int timeout_us) {
+  if (timeout_us == 0 || timeout_us > 10000000u) return HATTN_EINVAL;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(1000ull * timeout_us);
+  return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
 int attn_get_device_error(void* stream, int* code_out) {

@@ -84,9 +84,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;   // 2 s
 
 // Wait until the barrier's phase with the given parity has completed.  Gives
-// up (returns false, error word set) after kWaitLimitNs or as soon as another
-// CTA has raised an error.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+// up (returns false, error word set to 0x100 | site) after limit_ns, or as soon
+// as another CTA has raised an error.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int site, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -94,12 +94,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 255u) == 0) {
       if (error_raised()) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         raise_error(0x100 | site);
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+  return mbar_wait_for(bar, parity, site, kWaitLimitNs);
 }
 
 // Whole-warp wait: every lane waits, and the warp leaves converged with one

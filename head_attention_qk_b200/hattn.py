@@ -38,12 +38,15 @@ lib.attn_bwd_workspace_size.argtypes = [_i, _i, _i]
 lib.attn_bwd_workspace_size.restype = _sz
 lib.attn_get_device_error.argtypes = [_vp, ctypes.POINTER(_i)]
 lib.attn_get_device_error.restype = _i
+lib.attn_selftest_bounded_wait.argtypes = [_vp, ctypes.c_uint]
+lib.attn_selftest_bounded_wait.restype = _i
 lib.attn_error_string.argtypes = [_i]
 lib.attn_error_string.restype = ctypes.c_char_p
 
 BF16, E4M3 = 0, 1
 EXPORTED = ("attn_fwd", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
-            "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_error", "attn_error_string")
+            "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_error", "attn_selftest_bounded_wait",
+            "attn_error_string")
 NOALLOC_MAX_ROWS = 1 << 22
 
 

@@ -160,6 +160,16 @@ HATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, cons
  */
 HATTN_API int attn_get_device_error(void* stream, int* code_out);
 
+/*
+ * Failure-detection self-test (no counterpart on the pages): enqueues one small
+ * kernel whose only wait can never be satisfied, with a limit of timeout_us
+ * microseconds (1 .. 10^7).  The wait gives up, sets the device error word to
+ * 0x17F (0x100 | site 0x7F) and the kernel returns normally; the context stays
+ * usable.  Read the word with attn_get_device_error.  Returns 0, HATTN_EINVAL
+ * or HATTN_ELAUNCH.
+ */
+HATTN_API int attn_selftest_bounded_wait(void* stream, unsigned int timeout_us);
+
 /* Static text for a return code. */
 HATTN_API const char* attn_error_string(int code);
 

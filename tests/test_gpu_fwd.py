@@ -106,6 +106,9 @@ def check_fp8(h, w, rows=None):
     (1, 2, 2, 256, 256, False),
     (2, 4, 2, 333, 517, False),
     (1, 2, 1, 700, 700, True),
+    (1, 4, 2, 130, 700, True),          # causal, Sq < Sk, grouped heads
+    (1, 2, 2, 1, 1, False),             # a single key
+    (2, 2, 1, 5, 300, False),
 ])
 def test_fp8_small(h, B, Hq, Hkv, Sq, Sk, causal):
     check_fp8(h, Workload("f8", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, dtype="e4m3", seed=Sq))

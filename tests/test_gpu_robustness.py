@@ -1,0 +1,87 @@
+"""Failure detection, CUDA-graph capture and fail-closed behaviour on the GPU.
+
+- A kernel whose wait can never be satisfied gives up after a short limit,
+  reports the site in the device error word, and the context stays usable.
+- The forward and backward calls allocate nothing and never synchronise, so
+  they can be captured into a CUDA graph; replay equals the eager results bit
+  for bit.
+- Unsupported requests raise instead of being approximated.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from parity import LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
+from workloads import Workload, make_bwd_inputs, make_fwd_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import head_attention_qk_b200 as pkg
+
+    return pkg
+
+
+def test_bounded_wait_gives_up_and_context_survives(h):
+    assert h.get_device_error() == 0
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert h.lib.attn_selftest_bounded_wait(stream, 100_000) == 0        # 100 ms limit
+    assert h.get_device_error() == 0x17F                                  # 0x100 | self-test site
+    assert h.get_device_error() == 0                                      # read clears the word
+    # the context is still usable: a normal forward is correct afterwards
+    w = Workload("after", B=1, Hq=2, Hkv=2, Sq=200, Sk=300, seed=77)
+    x = make_fwd_inputs(w)
+    out, lse = h.attn_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda())
+    assert h.get_device_error() == 0
+    o_ref, lse_ref = oracle_fwd(x["q"], x["k"], x["v"], w.scale)
+    e = fwd_errors(out, lse, o_ref, lse_ref)
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS
+
+
+def test_selftest_rejects_bad_limits(h):
+    assert h.lib.attn_selftest_bounded_wait(None, 0) == -1
+    assert h.lib.attn_selftest_bounded_wait(None, 20_000_000) == -1
+
+
+def test_cuda_graph_capture_matches_eager(h):
+    w = Workload("graph", B=2, Hq=4, Hkv=2, Sq=333, Sk=333, causal=True, seed=78)
+    x = {k: v.cuda() for k, v in make_bwd_inputs(w).items()}
+    out_e, lse_e = h.attn_fwd(x["q"], x["k"], x["v"], causal=True)
+    dq_e, dk_e, dv_e = h.attn_bwd(x["q"], x["k"], x["v"], out_e, lse_e, x["dout"], causal=True)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            out_g, lse_g = h.attn_fwd(x["q"], x["k"], x["v"], causal=True, stream=s)
+            dq_g, dk_g, dv_g = h.attn_bwd(x["q"], x["k"], x["v"], out_g, lse_g, x["dout"], causal=True, stream=s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    for a, b in ((out_g, out_e), (dq_g, dq_e), (dk_g, dk_e), (dv_g, dv_e)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(lse_g, lse_e)
+
+
+def test_fail_closed_on_device(h):
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")     # head dim 64 is not offered
+    with pytest.raises(h.HattnError) as ei:
+        h.attn_fwd(q, q, q)
+    assert ei.value.code == -2
+    q = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 2, 32, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(h.HattnError) as ei:
+        h.attn_fwd(q, k, k, causal=True)                                    # causal with Sq > Sk
+    assert ei.value.code == -2
+    q8 = torch.zeros(1, 2, 64, 128, dtype=torch.float8_e4m3fn, device="cuda")
+    with pytest.raises(h.HattnError) as ei:
+        h.attn_fwd(q8, q8, q8)                                              # e4m3 without descales
+    assert ei.value.code == -1
+    assert h.get_device_error() == 0
