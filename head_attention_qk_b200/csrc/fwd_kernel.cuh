@@ -52,12 +52,10 @@ constexpr int kRegsOther = 88;
 constexpr int kRegsNeeded = (2 * kRegsSoftmax + kRegsOther) * 128;
 static_assert(kRegsNeeded <= (65536 / 384) / 8 * 8 * 384, "setmaxnreg split exceeds a 384-thread launch");
 // Of every 8 pairs of softmax elements, this many take the software exp2
-// (FMA pipe) and the rest the MUFU ex2.  MUFU ex2 runs at 16 per clock per SM,
-// exactly the bf16 MMA rate at D = 128, and the fp8 path takes its exponentials
-// as fp16 pairs (two per MUFU operation).  Measured on B200, moving a share to
-// the polynomial (about 9 issue slots per element) did not pay on this kernel,
-// whose softmax is bound by its dependency chain rather than by MUFU, so the
-// default share is 0; the knob stays for other tile shapes.
+// (FMA pipe) and the rest the MUFU ex2.  MUFU ex2 runs at 16 per clock per SM
+// in every format (measured: fp32, fp16 pairs and bf16 pairs alike), exactly
+// the bf16 MMA rate at D = 128 and three quarters of the fp8 QK^T + fp16 PV
+// rate, so the fp8 path moves a share of its exponentials to the FMA pipe.
 #ifndef HATTN_POLY_PAIRS_BF16
 #define HATTN_POLY_PAIRS_BF16 0
 #endif
@@ -479,21 +477,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, mneg2);
           float2 p;
           if ((e2 & 7) < kPolyPairs) {
-            p = exp2_poly2(x);
+            // fp16 P (fp8 path) tolerates the quadratic, bf16 P takes the cubic
+            p = exp2_poly2<kFp8 ? 2 : 3>(x);
             if (masked) {                               // the polynomial is never exactly 0
               p.x = kbase + e > kv_limit ? 0.f : p.x;
               p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
             }
-            pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
-          } else if (kFp8) {
-            // fp8 path: P is fp16, so the exponent is taken as fp16 pairs by one
-            // MUFU operation; the row sum adds exactly the fp16 values P V uses.
-            pk[e2] = ex2_f16x2(pack_f16x2(x.x, x.y));
-            p = unpack_f16x2(pk[e2]);
           } else {
             p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            pk[e2] = pack_bf16x2(p.x, p.y);
           }
+          pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
           acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
         }
         __syncwarp();
