@@ -1,10 +1,15 @@
 // fwd_kernel.cuh -- fused attention forward for sm_100a (bf16 and e4m3 inputs).
 //
-// Computes, for one (batch, query head) and 256 query rows per CTA,
+// Computes, for one (batch, query head) and 256 query rows per work unit,
 //   O = softmax(scale * Q K^T [+ causal mask]) V   and   LSE = ln sum_j exp(s_j),
 // the operation of fmha_v3_fwd with return_softmax_lse and q/k/v descales
 // (AITER PR #2911 "F8 fmha ASM gfx950", Test Result), at head dim 128 with
 // grouped KV heads (RL-Kernel PR #319, ROCm Validation table: Hq=32, Hkv=8).
+//
+// Persistent: one CTA per SM loops over work units (256 query rows of one
+// (b, h) against one KV block); barrier phases and ring positions carry over
+// from unit to unit, tensor memory is allocated once, and the next unit's Q is
+// loaded as soon as the current unit's last S = Q K^T has been issued.
 //
 // CTA layout (384 threads, one CTA per SM):
 //   warps 0-3  softmax group 0: query tile 0 (rows q0 .. q0+127), one row per thread
@@ -80,6 +85,7 @@ struct FwdArgs {
   const float* k_descale;
   const float* v_descale;
   int block_offset;              // index of this launch's first block among all blocks
+  int total_units;               // n_qpairs * B * Hq * (blocks in this launch); CTAs loop over them
 };
 
 template <bool kFp8>
@@ -97,7 +103,7 @@ struct FwdSmemLayout {
   static constexpr int kRingOff = kQOff + kQTilesPerCta * kTileBytes;
   static constexpr int kV16Off = kRingOff + kRing * kTileBytes;
   static constexpr int kBarOff = kV16Off + kStagesV16 * kV16Bytes;
-  static constexpr int kNumBars = 1 + 2 * kRing + 2 * kStagesV16 + 8;
+  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -105,6 +111,8 @@ struct FwdSmemLayout {
 
 struct FwdBars {
   uint64_t* q_full;
+  uint64_t* q_empty;  // the unit's last S MMA has been issued (Q may be reloaded)
+  uint64_t* mma_drain;  // every MMA of the CTA has completed (committed once, at exit)
   uint64_t* ring_full;   // [kRing]
   uint64_t* ring_empty;  // [kRing]
   uint64_t* v16_full;
@@ -118,7 +126,7 @@ struct FwdBars {
 // Barrier sites recorded in the error word when a wait times out.
 enum : int {
   kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteV16Full, kSiteV16Empty,
-  kSiteSFull, kSitePFull, kSiteODone
+  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain
 };
 
 __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int q_row0) {
@@ -128,7 +136,47 @@ __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int 
   return max_key / kBlockN + 1;
 }
 
-template <bool kFp8, bool kPartial>
+// One work unit: 256 query rows of one (b, h) against one KV block.
+struct FwdUnit {
+  int bh, kvh, q_row0, blk, sk, n_kv;
+};
+
+// Units are numbered block-major.  Without a mask, consecutive units share a
+// head (its K/V stays hot in L2); under a causal mask the order is rank-major
+// over heads, heaviest query tiles first, so the persistent CTAs pick up the
+// long units before the short ones.
+__device__ __forceinline__ FwdUnit fwd_unit(const FwdArgs& a, int u) {
+  FwdUnit w;
+  const int nbh = a.B * a.Hq;
+  const int per_blk = a.n_qpairs * nbh;
+  w.blk = u / per_blk;
+  const int r = u - w.blk * per_blk;
+  int qpair;
+  if (a.causal) {
+    const int rank = r / nbh;
+    w.bh = r - rank * nbh;
+    qpair = a.n_qpairs - 1 - rank;
+  } else {
+    w.bh = r / a.n_qpairs;
+    qpair = r - w.bh * a.n_qpairs;
+  }
+  const int b = w.bh / a.Hq, h = w.bh - b * a.Hq;
+  w.kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
+  w.q_row0 = qpair * (kQTilesPerCta * kBlockM);
+  w.sk = a.sk[w.blk];
+  w.n_kv = fwd_num_kv_tiles(w.sk, a.Sq, a.causal, w.q_row0);
+  return w;
+}
+
+// Unit loop condition.  Persistent launches loop while units remain; a
+// one-unit-per-CTA launch runs the body exactly once (the compiler sees a single
+// iteration, so the per-tile code is the same as a kernel without the loop).
+template <bool kPersist>
+__device__ __forceinline__ bool fwd_more_units(int u, int u_first, int u_end, bool ok) {
+  return kPersist ? (u < u_end && ok) : (u == u_first);
+}
+
+template <bool kFp8, bool kPartial, bool kPersist>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
   using L = FwdSmemLayout<kFp8>;
   extern __shared__ uint8_t smem_raw[];
@@ -136,24 +184,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
   const int warp = warp_id();
   const int lane = lane_id();
-
-  const int blk_local = blockIdx.z;
-  const int bh = blockIdx.y;
-  const int b = bh / args.Hq;
-  const int h = bh - b * args.Hq;
-  const int G = args.Hq / args.Hkv;
-  const int kvh = b * args.Hkv + h / G;
-  // heaviest tiles first under a causal mask
-  const int qpair = args.causal ? (args.n_qpairs - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int q_row0 = qpair * (kQTilesPerCta * kBlockM);
-  const int sk = args.sk[blk_local];
-  const int n_kv = fwd_num_kv_tiles(sk, args.Sq, args.causal, q_row0);
+  // Persistent: this CTA takes units blockIdx.x, blockIdx.x + gridDim.x, ...
+  // otherwise the grid holds one CTA per unit.
+  const int u_first = blockIdx.x, u_step = kPersist ? (int)gridDim.x : 1, u_end = args.total_units;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   FwdBars bb;
   {
     uint64_t* p = bars;
     bb.q_full = p; p += 1;
+    bb.q_empty = p; p += 1;
+    bb.mma_drain = p; p += 1;
     bb.ring_full = p; p += L::kRing;
     bb.ring_empty = p; p += L::kRing;
     bb.v16_full = p; p += L::kStagesV16;
@@ -166,6 +207,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     mbar_init(bb.q_full, 1);
+    mbar_init(bb.q_empty, 1);
+    mbar_init(bb.mma_drain, 1);
     for (int s = 0; s < L::kRing; ++s) {
       mbar_init(&bb.ring_full[s], 1);
       // fp8: odd slots always hold V (even ring), released by the 2 widening warps;
@@ -188,11 +231,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     tmem_alloc(bb.tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
-    prefetch_tmap(&args.tm_q);
-    prefetch_tmap(&args.tm_k[blk_local]);
-    prefetch_tmap(&args.tm_v[blk_local]);
-  }
+  if (warp == 8 && lane == 0) prefetch_tmap(&args.tm_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -202,42 +241,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   uint8_t* sRing = smem + L::kRingOff;
   uint8_t* sV16 = smem + L::kV16Off;
 
-  // Register split: the launch gives 168 x 384 = 64512 registers.  The
-  // producer / MMA / widening warpgroup (warps 8-11) drops to 64 per thread and
-  // the two softmax warpgroups rise to 216: 2*128*216 + 128*64 = 63488 <= 64512.
+  // Register split (see kRegsSoftmax): the producer / MMA / widening warpgroup
+  // gives registers up, the two softmax warpgroups take them.
   if (warp >= 8) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsOther) : "memory");
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const CUtensorMap* tq = &args.tm_q;
-      const CUtensorMap* tk = &args.tm_k[blk_local];
-      const CUtensorMap* tv = &args.tm_v[blk_local];
       constexpr int kBoxes = kFp8 ? 1 : 2;                 // 128-byte-wide boxes per 128-column row
       constexpr int kBoxBytes = L::kTileBytes / kBoxes;
       constexpr int kBoxCols = 128 / L::kElt;
-      mbar_arrive_expect_tx(bb.q_full, kQTilesPerCta * L::kTileBytes);
-      for (int t = 0; t < kQTilesPerCta; ++t)
-        for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(sQ + t * L::kTileBytes + x * kBoxBytes, tq, bb.q_full, x * kBoxCols, q_row0 + t * kBlockM, bh);
       bool ok = true;
-      // sequence n: K_{n/2} for even n, V_{n/2} for odd n
-      int slot = 0;
+      int slot = 0, units = 0;
       uint32_t ph = 0;
-      for (int n = 0; n < 2 * n_kv && ok; ++n) {
-        if (n >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], ph ^ 1u, kSiteKEmpty);
+      long long nseq = 0;                                  // K/V tiles loaded by this CTA
+      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+        const FwdUnit w = fwd_unit(args, u);
+        const CUtensorMap* tk = &args.tm_k[w.blk];
+        const CUtensorMap* tv = &args.tm_v[w.blk];
+        // the previous unit's last S has been issued before Q is overwritten
+        if (units > 0) ok = mbar_wait(bb.q_empty, (units - 1) & 1, kSiteQFull);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
-        const CUtensorMap* tm = (n & 1) ? tv : tk;
-        for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(sRing + slot * L::kTileBytes + x * kBoxBytes, tm, &bb.ring_full[slot], x * kBoxCols,
-                      (n >> 1) * kBlockN, kvh);
-        if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
+        mbar_arrive_expect_tx(bb.q_full, kQTilesPerCta * L::kTileBytes);
+        for (int t = 0; t < kQTilesPerCta; ++t)
+          for (int x = 0; x < kBoxes; ++x)
+            tma_load_3d(sQ + t * L::kTileBytes + x * kBoxBytes, &args.tm_q, bb.q_full, x * kBoxCols,
+                        w.q_row0 + t * kBlockM, w.bh);
+        // sequence n: K_{n/2} for even n, V_{n/2} for odd n
+        for (int n = 0; n < 2 * w.n_kv && ok; ++n, ++nseq) {
+          if (nseq >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], ph ^ 1u, kSiteKEmpty);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
+          const CUtensorMap* tm = (n & 1) ? tv : tk;
+          for (int x = 0; x < kBoxes; ++x)
+            tma_load_3d(sRing + slot * L::kTileBytes + x * kBoxBytes, tm, &bb.ring_full[slot], x * kBoxCols,
+                        (n >> 1) * kBlockN, w.kvh);
+          if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
+        }
       }
       // Drain: every load issued must land before the CTA may exit.
-      for (int n = max(0, 2 * n_kv - L::kRing); n < 2 * n_kv; ++n)
-        mbar_wait(&bb.ring_full[n % L::kRing], (n / L::kRing) & 1, kSiteKFull);
-      mbar_wait(bb.q_full, 0, kSiteQFull);
+      for (long long pos = nseq - L::kRing < 0 ? 0 : nseq - L::kRing; pos < nseq; ++pos)
+        mbar_wait_drain(&bb.ring_full[pos % L::kRing], (uint32_t)((pos / L::kRing) & 1), kSiteDrain);
+      if (units > 0) mbar_wait_drain(bb.q_full, (units - 1) & 1, kSiteDrain);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -251,8 +296,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       constexpr int kQKStepBytes = 32;
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
       const uint32_t sV16a = smem_u32(sV16);
-
-      // K_j sits in ring slot (2j) % kRing, V_j in (2j+1) % kRing.
       // Descriptor halves: Q / K tiles K-major (SBO 1024 B), V MN-major (LBO 16 KB
       // between the two 64-column halves of the head dim, SBO 1024 B).
       constexpr uint32_t kHi = sdesc_hi(1024);
@@ -282,108 +325,130 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           mma_f16_ts2(d, a + k * 8, b_lo + k * (2048 >> 4), kHi, kIdescPV, (acc || k > 0) ? 1u : 0u);
         }
       };
-      // Wait for each half of P_t and issue its MMAs.
-      auto pv = [&](int t, uint32_t vbase, int j) -> bool {
+      // Wait for each half of P_t and issue its MMAs (jg: this CTA's tile count).
+      auto pv = [&](int t, uint32_t vbase, uint32_t jg, int j) -> bool {
         for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(&bb.p_full[t * 2 + half], j & 1, kSitePFull)) return false;
+          if (!mbar_wait(&bb.p_full[t * 2 + half], jg & 1, kSitePFull)) return false;
           tc_fence_after();
           issue_pv_half(t, vbase, half, j > 0);
         }
         return true;
       };
+      auto next_pos = [](int& slot, uint32_t& ph) {
+        if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
+      };
 
-      bool ok = mbar_wait(bb.q_full, 0, kSiteQFull);
-      if (ok && n_kv > 0) ok = mbar_wait(&bb.ring_full[0], 0, kSiteKFull);
-      if (ok && n_kv > 0) {
+      bool ok = true;
+      int kslot = 0, vs16 = 0, units = 0;
+      uint32_t kph = 0, vph16 = 0, jg = 0;
+      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+        const FwdUnit w = fwd_unit(args, u);
+        const int n_kv = w.n_kv;
+        ok = mbar_wait(bb.q_full, units & 1, kSiteQFull);
+        if (ok) ok = mbar_wait(&bb.ring_full[kslot], kph, kSiteKFull);
+        if (!ok) break;
         tc_fence_after();
-        issue_qk(0, 0);
+        issue_qk(0, kslot);
         mma_commit(&bb.s_full[0]);
-        issue_qk(1, 0);
+        issue_qk(1, kslot);
         mma_commit(&bb.s_full[1]);
-        mma_commit(&bb.ring_empty[0]);
-      }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int nv = 2 * j + 1, vslot = nv % L::kRing;
-        const int vs = j % max(L::kStagesV16, 1), u16 = j / max(L::kStagesV16, 1);
-        uint32_t vbase;
-        if (kFp8) {
-          ok = mbar_wait(&bb.v16_full[vs], u16 & 1, kSiteV16Full);
-          vbase = sV16a + vs * L::kV16Bytes;
-        } else {
-          ok = mbar_wait(&bb.ring_full[vslot], (nv / L::kRing) & 1, kSiteVFull);
-          vbase = sRa + vslot * L::kTileBytes;
-        }
-        if (ok) ok = pv(0, vbase, j);
-        if (!ok) break;
-        if (j == n_kv - 1) mma_commit(&bb.o_done[0]);
-        const int jn = j + 1, nk = 2 * jn, kslot = nk % L::kRing;
-        if (jn < n_kv) {
-          ok = mbar_wait(&bb.ring_full[kslot], (nk / L::kRing) & 1, kSiteKFull);
+        mma_commit(&bb.ring_empty[kslot]);
+        if (n_kv == 1) mma_commit(bb.q_empty);             // last S of the unit issued
+        for (int j = 0; j < n_kv && ok; ++j, ++jg) {
+          int vslot = kslot;
+          uint32_t vph = kph;
+          next_pos(vslot, vph);                            // V_j follows K_j
+          uint32_t vbase;
+          if (kFp8) {
+            ok = mbar_wait(&bb.v16_full[vs16], vph16, kSiteV16Full);
+            vbase = sV16a + vs16 * L::kV16Bytes;
+          } else {
+            ok = mbar_wait(&bb.ring_full[vslot], vph, kSiteVFull);
+            vbase = sRa + vslot * L::kTileBytes;
+          }
+          if (ok) ok = pv(0, vbase, jg, j);
           if (!ok) break;
-          tc_fence_after();
-          issue_qk(0, kslot);
-          mma_commit(&bb.s_full[0]);
-        }
-        ok = pv(1, vbase, j);
-        if (!ok) break;
-        if (kFp8) mma_commit(&bb.v16_empty[vs]);
-        else mma_commit(&bb.ring_empty[vslot]);
-        if (j == n_kv - 1) mma_commit(&bb.o_done[1]);
-        if (jn < n_kv) {
-          issue_qk(1, kslot);
-          mma_commit(&bb.s_full[1]);
-          mma_commit(&bb.ring_empty[kslot]);
+          if (j == n_kv - 1) mma_commit(&bb.o_done[0]);
+          kslot = vslot;
+          kph = vph;
+          next_pos(kslot, kph);                            // K_{j+1} (or the next unit's K_0)
+          const bool more = j + 1 < n_kv;
+          if (more) {
+            ok = mbar_wait(&bb.ring_full[kslot], kph, kSiteKFull);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(0, kslot);
+            mma_commit(&bb.s_full[0]);
+          }
+          ok = pv(1, vbase, jg, j);
+          if (!ok) break;
+          if (kFp8) {
+            mma_commit(&bb.v16_empty[vs16]);
+            if (++vs16 == L::kStagesV16) { vs16 = 0; vph16 ^= 1u; }
+          } else {
+            mma_commit(&bb.ring_empty[vslot]);
+          }
+          if (j == n_kv - 1) mma_commit(&bb.o_done[1]);
+          if (more) {
+            issue_qk(1, kslot);
+            mma_commit(&bb.s_full[1]);
+            mma_commit(&bb.ring_empty[kslot]);
+            if (j + 1 == n_kv - 1) mma_commit(bb.q_empty);  // last S of the unit issued
+          }
         }
       }
-      if (!ok) {
-        // Error path: make sure no MMA is still in flight before TMEM is freed.
-        mma_commit(&bb.o_done[0]);
-        mma_commit(&bb.o_done[1]);
-      }
-      // Drain: wait for the final commits so no tcgen05 op outlives the CTA.
-      mbar_wait(&bb.o_done[0], 0, kSiteODone);
-      mbar_wait(&bb.o_done[1], 0, kSiteODone);
+      // Drain (normal and error paths): the commit tracks every MMA this thread
+      // issued, so none is in flight when tensor memory is freed.
+      mma_commit(bb.mma_drain);
+      mbar_wait_drain(bb.mma_drain, 0, kSiteDrain);
     }
     __syncwarp();
   } else if (warp >= 10) {
     // ------------------------------------------------------------ fp8: widen V to fp16
-    if (kFp8) {
+    if constexpr (kFp8) {
       const int t = threadIdx.x - 320;                       // 0..63
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int nv = 2 * j + 1, vslot = nv % L::kRing;
-        const int s16 = j % max(L::kStagesV16, 1), u16 = j / max(L::kStagesV16, 1);
-        ok = warp_wait(&bb.ring_full[vslot], (nv / L::kRing) & 1, kSiteVFull);
-        if (ok && j >= L::kStagesV16) ok = warp_wait(&bb.v16_empty[s16], (u16 - 1) & 1, kSiteV16Empty);
-        if (!ok) break;
-        const uint8_t* src = sRing + vslot * L::kTileBytes;
-        uint8_t* dst = sV16 + s16 * L::kV16Bytes;
-        // e4m3 tile: row r (key) = 128 bytes, 16-byte chunk c holds head dims [16c, 16c+16),
-        // stored at chunk c ^ (r & 7).  fp16 tile: two 64-dim halves of 16 KB; row r of a
-        // half = 128 bytes, chunk c8 holds dims [8 c8, 8 c8 + 8) of the half at c8 ^ (r & 7).
+      uint32_t jg = 0;                                       // this CTA's tile count
+      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step) {
+        const int n_kv = fwd_unit(args, u).n_kv;
+        for (int j = 0; j < n_kv && ok; ++j, ++jg) {
+          // V of tile jg sits at ring position 2 jg + 1
+          const int vslot = (int)((2u * jg + 1u) % L::kRing);
+          const uint32_t vph = ((2u * jg + 1u) / L::kRing) & 1u;
+          const int s16 = jg % L::kStagesV16;
+          const uint32_t u16 = jg / L::kStagesV16;
+          ok = warp_wait(&bb.ring_full[vslot], vph, kSiteVFull);
+          if (ok && jg >= (uint32_t)L::kStagesV16) ok = warp_wait(&bb.v16_empty[s16], (u16 - 1) & 1, kSiteV16Empty);
+          if (!ok) break;
+          const uint8_t* src = sRing + vslot * L::kTileBytes;
+          uint8_t* dst = sV16 + s16 * L::kV16Bytes;
+          // e4m3 tile: row r (key) = 128 bytes, 16-byte chunk c holds head dims [16c, 16c+16),
+          // stored at chunk c ^ (r & 7).  fp16 tile: two 64-dim halves of 16 KB; row r of a
+          // half = 128 bytes, chunk c8 holds dims [8 c8, 8 c8 + 8) of the half at c8 ^ (r & 7).
 #pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-          const int idx = t + 64 * it;
-          const int r = idx >> 3, c = idx & 7;
-          const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + ((c ^ (r & 7)) << 4));
-          const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-          uint32_t o[8];
+          for (int it = 0; it < 16; ++it) {
+            const int idx = t + 64 * it;
+            const int r = idx >> 3, c = idx & 7;
+            const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint32_t wv[4] = {in.x, in.y, in.z, in.w};
+            uint32_t o[8];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            o[2 * q] = e4m3x2_to_f16x2((uint16_t)(w[q] & 0xFFFFu));
-            o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(w[q] >> 16));
+            for (int q = 0; q < 4; ++q) {
+              o[2 * q] = e4m3x2_to_f16x2((uint16_t)(wv[q] & 0xFFFFu));
+              o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(wv[q] >> 16));
+            }
+            const int half = c >> 2;
+            const int c8 = (c & 3) * 2;
+            uint8_t* rowp = dst + half * 16384 + r * 128;
+            *reinterpret_cast<uint4*>(rowp + ((c8 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(rowp + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
           }
-          const int half = c >> 2;
-          const int c8 = (c & 3) * 2;
-          uint8_t* rowp = dst + half * 16384 + r * 128;
-          *reinterpret_cast<uint4*>(rowp + ((c8 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(rowp + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bb.v16_full[s16]);
-          mbar_arrive(&bb.ring_empty[vslot]);   // this warp is done reading the e4m3 slot
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bb.v16_full[s16]);
+            mbar_arrive(&bb.ring_empty[vslot]);   // this warp is done reading the e4m3 slot
+          }
         }
       }
     }
@@ -396,122 +461,129 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + tile * 128;
     const uint32_t tO = tmem + lane_base + 256 + tile * 128;
-    const int row = q_row0 + tile * kBlockM + r;
-    const int kv_limit = args.causal ? min(sk - 1, row + (sk - args.Sq)) : sk - 1;
-
     constexpr int kPolyPairs = PolyShare<kFp8>::kPairs;
-    float c = args.scale_log2;
-    float v_scale = 1.f;
-    if (kFp8) {
-      c *= __ldg(&args.q_descale[bh]) * __ldg(&args.k_descale[kvh]);
-      v_scale = __ldg(&args.v_descale[kvh]);
-    }
 
-    float m = -INFINITY;     // running max of x = s * c (base-2 units)
-    float l = 0.f;           // running sum of 2^(x - m)
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = warp_wait(&bb.s_full[tile], j & 1, kSiteSFull);
-      if (!ok) break;
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t u[128];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[q * 32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(u[e]);
+    uint32_t jg = 0;                                  // this CTA's tile count
+    int units = 0;
+    for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+      const FwdUnit w = fwd_unit(args, u);
+      const int n_kv = w.n_kv, sk = w.sk, bh = w.bh;
+      const int row = w.q_row0 + tile * kBlockM + r;
+      const int kv_limit = args.causal ? min(sk - 1, row + (sk - args.Sq)) : sk - 1;
+      float c = args.scale_log2;
+      float v_scale = 1.f;
+      if (kFp8) {
+        c *= __ldg(&args.q_descale[bh]) * __ldg(&args.k_descale[w.kvh]);
+        v_scale = __ldg(&args.v_descale[w.kvh]);
       }
-      const int kbase = j * kBlockN;
-      const bool masked = kbase + kBlockN - 1 > kv_limit;
-      if (masked) {
+
+      float m = -INFINITY;     // running max of x = s * c (base-2 units)
+      float l = 0.f;           // running sum of 2^(x - m)
+      for (int j = 0; j < n_kv; ++j, ++jg) {
+        ok = warp_wait(&bb.s_full[tile], jg & 1, kSiteSFull);
+        if (!ok) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t uu[128];
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (kbase + e > kv_limit) s[e] = -INFINITY;
-      }
-      // row max: eight independent three-input chains
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[8 + i], s[16 + i]);
-#pragma unroll
-      for (int e = 24; e < 120; e += 16) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[e + i], s[e + 8 + i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
-      const float m_tile = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
-      const bool need = m_tile > m + kRescaleThreshold || (m == -INFINITY && m_tile > -INFINITY);
-      float f = 1.f;
-      if (need) {
-        f = ex2_approx(m - m_tile);                    // 0 when m = -inf
-        m = m_tile;
-        l *= f;
-      }
-      __syncwarp();
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // Rescale this warp's 32 rows of O (PV_{j-1} completed before S_j).
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t u[32];
-          tmem_ld32(tO + q * 32, u);
+          for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&uu[q * 32]));
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
-          tmem_st32(tO + q * 32, u);
+          for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(uu[e]);
         }
-        tmem_wait_st();
-      }
-      const float mneg = (m == -INFINITY) ? 0.f : -m;
-      const float2 c2 = make_float2(c, c), mneg2 = make_float2(mneg, mneg);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // Two halves of 64 keys: each half is written to TMEM and released to the
-      // MMA warp as soon as it is ready, so P V can start on keys 0..63.
+        const int kbase = j * kBlockN;
+        const bool masked = kbase + kBlockN - 1 > kv_limit;
+        if (masked) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+          for (int e = 0; e < 128; ++e)
+            if (kbase + e > kv_limit) s[e] = -INFINITY;
+        }
+        // row max: eight independent three-input chains
+        float mx[8];
 #pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) {
-          const int e = half * 64 + 2 * e2;
-          const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, mneg2);
-          float2 p;
-          if ((e2 & 7) < kPolyPairs) {
-            // fp16 P (fp8 path) tolerates the quadratic, bf16 P takes the cubic
-            p = exp2_poly2<kFp8 ? 2 : 3>(x);
-            if (masked) {                               // the polynomial is never exactly 0
-              p.x = kbase + e > kv_limit ? 0.f : p.x;
-              p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
-            }
-          } else {
-            p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+#pragma unroll
+        for (int e = 24; e < 120; e += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[e + i], s[e + 8 + i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+        const float m_tile = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
+        const bool need = m_tile > m + kRescaleThreshold || (m == -INFINITY && m_tile > -INFINITY);
+        float f = 1.f;
+        if (need) {
+          f = ex2_approx(m - m_tile);                    // 0 when m = -inf
+          m = m_tile;
+          l *= f;
+        }
+        __syncwarp();
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // Rescale this warp's 32 rows of O (PV_{j-1} completed before S_j).
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t uq[32];
+            tmem_ld32(tO + q * 32, uq);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) uq[e] = __float_as_uint(__uint_as_float(uq[e]) * f);
+            tmem_st32(tO + q * 32, uq);
           }
-          pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
-          acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
+          tmem_wait_st();
         }
-        __syncwarp();
-        tmem_st32(tS + half * 32, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bb.p_full[tile * 2 + half]);
+        const float mneg = (m == -INFINITY) ? 0.f : -m;
+        const float2 c2 = make_float2(c, c), mneg2 = make_float2(mneg, mneg);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // Two halves of 64 keys: each half is written to TMEM and released to the
+        // MMA warp as soon as it is ready, so P V can start on keys 0..63.
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) {
+            const int e = half * 64 + 2 * e2;
+            const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, mneg2);
+            float2 p;
+            if ((e2 & 7) < kPolyPairs) {
+              // fp16 P (fp8 path) tolerates the quadratic, bf16 P takes the cubic
+              p = exp2_poly2<kFp8 ? 2 : 3>(x);
+              if (masked) {                               // the polynomial is never exactly 0
+                p.x = kbase + e > kv_limit ? 0.f : p.x;
+                p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
+              }
+            } else {
+              p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            }
+            pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
+            acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
+          }
+          __syncwarp();
+          tmem_st32(tS + half * 32, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bb.p_full[tile * 2 + half]);
+        }
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+        const float2 a2 = __fadd2_rn(a01, a23);
+        l += a2.x + a2.y;
       }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 a = __fadd2_rn(a01, a23);
-      l += a.x + a.y;
-    }
-    if (ok) ok = warp_wait(&bb.o_done[tile], 0, kSiteODone);
-    if (ok) {
+      if (ok) ok = warp_wait(&bb.o_done[tile], units & 1, kSiteODone);
+      if (!ok) break;
+      // Epilogue.  The next unit's first P V (which overwrites O) waits for this
+      // group's first P of that unit, so these O reads complete first.
       tc_fence_after();
       const float inv_l = (l > 0.f) ? (v_scale / l) : 0.f;
       const bool store = row < args.Sq;
-      const size_t orow = ((size_t)bh * args.Sq + (size_t)max(row, 0)) * kHeadDim;
-      const size_t part = (size_t)(args.block_offset + blk_local);
+      const size_t orow = ((size_t)bh * args.Sq + (size_t)row) * kHeadDim;
+      const size_t part = (size_t)(args.block_offset + w.blk);
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
-        uint32_t u[32];
+        uint32_t uq[32];
         __syncwarp();
-        tmem_ld32(tO + q * 32, u);
+        tmem_ld32(tO + q * 32, uq);
         tmem_wait_ld();
         if (store) {
           if (kPartial) {
@@ -520,13 +592,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4*>(dst + e) =
-                  make_float4(__uint_as_float(u[e]) * inv_l, __uint_as_float(u[e + 1]) * inv_l,
-                              __uint_as_float(u[e + 2]) * inv_l, __uint_as_float(u[e + 3]) * inv_l);
+                  make_float4(__uint_as_float(uq[e]) * inv_l, __uint_as_float(uq[e + 1]) * inv_l,
+                              __uint_as_float(uq[e + 2]) * inv_l, __uint_as_float(uq[e + 3]) * inv_l);
           } else {
             uint32_t pkd[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-              pkd[e] = pack_bf16x2(__uint_as_float(u[2 * e]) * inv_l, __uint_as_float(u[2 * e + 1]) * inv_l);
+              pkd[e] = pack_bf16x2(__uint_as_float(uq[2 * e]) * inv_l, __uint_as_float(uq[2 * e + 1]) * inv_l);
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.out) + orow + q * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);

@@ -11,6 +11,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+#include <climits>
 #include <mutex>
 
 #include "../../include/hattn.h"
@@ -60,21 +62,56 @@ bool set_smem_attr(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
-template <bool kFp8, bool kPartial>
-int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, cudaStream_t st) {
+// Number of SMs of the current device, looked up once per device.
+int device_sm_count() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return -1;
+  if (dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+template <bool kFp8, bool kPartial, bool kPersist>
+int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
   using L = FwdSmemLayout<kFp8>;
   static std::once_flag once;
   static bool attr_ok = false;
   std::call_once(once, [] {
     cudaFuncAttributes fa;
-    attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial>, L::kAlloc) &&
-              cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8, kPartial>) == cudaSuccess &&
+    attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial, kPersist>, L::kAlloc) &&
+              cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8, kPartial, kPersist>) == cudaSuccess &&
               fa.numRegs * kFwdThreads >= kRegsNeeded;   // the setmaxnreg split must fit the launch
   });
   if (!attr_ok) return HATTN_ELAUNCH;
-  dim3 grid(a.n_qpairs, a.B * a.Hq, n_blocks_in_launch);
-  attn_fwd_kernel<kFp8, kPartial><<<grid, kFwdThreads, L::kAlloc, st>>>(a);
+  attn_fwd_kernel<kFp8, kPartial, kPersist><<<grid, kFwdThreads, L::kAlloc, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
+}
+
+// Units of 256 query rows x one KV block.  Short units (few KV tiles, no mask)
+// go to the persistent kernel, one CTA per SM, which overlaps each unit's
+// epilogue and the next unit's Q load with the running MMAs; long or causal
+// units go one CTA per unit, ordered heaviest first, and the hardware
+// scheduler balances them.
+constexpr int kPersistMaxKvTiles = 8;
+
+template <bool kFp8, bool kPartial>
+int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, int max_sk, cudaStream_t st) {
+  const long long units = (long long)a.n_qpairs * a.B * a.Hq * n_blocks_in_launch;
+  if (units <= 0 || units > INT_MAX) return HATTN_EUNSUPPORTED;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HATTN_EDEVICE;
+  FwdArgs args = a;
+  args.total_units = (int)units;
+  const bool persist = !a.causal && (max_sk + kBlockN - 1) / kBlockN <= kPersistMaxKvTiles && units > sms;
+  if (persist) return launch_fwd_grid<kFp8, kPartial, true>(args, sms, st);
+  return launch_fwd_grid<kFp8, kPartial, false>(args, (int)units, st);
 }
 
 int check_common(int B, int Hq, int Hkv, int Sq, int D, float scale) {
@@ -131,7 +168,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if (Sk <= 0) return HATTN_EINVAL;
   if ((rc = check_descales(dtype, q_descale, k_descale, v_descale))) return rc;
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
-  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk)) return HATTN_EUNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return HATTN_EALIGN;
 
   const bool fp8 = dtype == HATTN_E4M3;
@@ -150,7 +187,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
   a.block_offset = 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return fp8 ? launch_fwd<true, false>(a, 1, st) : launch_fwd<false, false>(a, 1, st);
+  return fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
 }
 
 size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks) {
@@ -168,7 +205,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
   if (rc) return rc;
   if ((rc = check_descales(dtype, q_descale, k_descale, v_descale))) return rc;
   if (dtype != HATTN_BF16) return HATTN_EUNSUPPORTED;
-  if (!sizes_fit(B, Hq, Sq) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, Hq, Sq)) return HATTN_EUNSUPPORTED;
   for (int i = 0; i < n_blocks; ++i) {
     if (!k_blocks[i] || !v_blocks[i]) return HATTN_EINVAL;
     if (blk_len[i] <= 0) return HATTN_EUNSUPPORTED;
@@ -188,7 +225,9 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     const int cnt = n_blocks - first < kMaxKvBlocks ? n_blocks - first : kMaxKvBlocks;
     memset(&a, 0, sizeof(a));
     if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    int max_len = 0;
     for (int i = 0; i < cnt; ++i) {
+      max_len = blk_len[first + i] > max_len ? blk_len[first + i] : max_len;
       if (!encode_rows(&a.tm_k[i], k_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
         return HATTN_ELAUNCH;
       if (!encode_rows(&a.tm_v[i], v_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
@@ -202,7 +241,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     a.out = o_parts;
     a.lse = lse_parts;
     a.block_offset = first;
-    if ((rc = launch_fwd<false, true>(a, cnt, st))) return rc;
+    if ((rc = launch_fwd<false, true>(a, cnt, max_len, st))) return rc;
   }
   const unsigned grid = (unsigned)((rows + 7) / 8);
   lse_merge_kernel<<<grid, 256, 0, st>>>(o_parts, lse_parts, n_blocks, rows, reinterpret_cast<uint16_t*>(out), lse);

@@ -106,6 +106,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int si
   return mbar_wait_for(bar, parity, site, kWaitLimitNs);
 }
 
+// Drain wait before a CTA exits: asynchronous copies or MMAs this thread issued
+// must have landed before shared or tensor memory is released, even when
+// another CTA has already raised an error, so this wait does not give up on
+// the error word; it stops only at its own limit (0.2 s).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > 200ull * 1000ull * 1000ull) {
+      raise_error(0x100 | site);
+      return false;
+    }
+  }
+}
+
 // Whole-warp wait: every lane waits, and the warp leaves converged with one
 // verdict (false if any lane gave up), so .sync.aligned tcgen05 instructions
 // that follow see a converged warp.

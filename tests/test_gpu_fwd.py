@@ -72,6 +72,28 @@ def test_ragged_shapes(h, B, Hq, Hkv, Sq, Sk, causal):
     check_bf16(h, w)
 
 
+# More units (256 query rows x one (b, h)) than SMs and at most 8 KV tiles, no
+# mask: these launch the persistent kernel (one CTA per SM looping over units).
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk", [
+    (1, 40, 40, 1560, 512),
+    (2, 32, 8, 1000, 300),
+    (2, 48, 16, 520, 1024),
+])
+def test_persistent_short_kv(h, B, Hq, Hkv, Sq, Sk):
+    check_bf16(h, Workload("persist", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, seed=500 + Sq + Sk))
+
+
+def test_persistent_matches_one_cta_per_unit_bitwise(h):
+    # 280 units run persistently; three heads alone (21 units) run one CTA per unit
+    w = Workload("persist_bits", B=1, Hq=40, Hkv=40, Sq=1560, Sk=512, seed=77)
+    x = cuda(make_fwd_inputs(w))
+    o, l = run_fwd(h, x, False)
+    xs = {n: x[n][:, :3].contiguous() for n in ("q", "k", "v")}
+    o3, l3 = run_fwd(h, xs, False)
+    assert torch.equal(o3.view(torch.int16), o[:, :3].view(torch.int16))
+    assert torch.equal(l3, l[:, :3])
+
+
 def test_llm_config_sampled_rows(h):
     w = workloads.get("llm_gqa")
     check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
@@ -112,6 +134,10 @@ def check_fp8(h, w, rows=None):
 ])
 def test_fp8_small(h, B, Hq, Hkv, Sq, Sk, causal):
     check_fp8(h, Workload("f8", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, dtype="e4m3", seed=Sq))
+
+
+def test_fp8_persistent_short_kv(h):
+    check_fp8(h, Workload("f8p", B=1, Hq=40, Hkv=20, Sq=1200, Sk=640, dtype="e4m3", seed=41))
 
 
 def test_fp8_config_sampled_rows(h):
