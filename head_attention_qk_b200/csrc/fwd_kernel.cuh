@@ -16,7 +16,12 @@
 //   warps 4-7  softmax group 1: query tile 1 (rows q0+128 .. q0+255)
 //   warp 8     TMA producer: Q once, then K_j / V_j into one ring
 //   warp 9     MMA issuer (one thread) and tensor-memory owner
-//   warps 10-11  fp8 only: widen each e4m3 V tile to fp16 in shared memory
+//   warps 10-11  no role (they hold the registers the softmax groups give up)
+//
+// e4m3 inputs: Q and K stay e4m3 (S = Q K^T runs as an 8-bit MMA); V arrives
+// already widened to fp16 (exact) by a separate pass, so P V is an fp16 MMA with
+// P in fp16 and no conversion competes with the softmax for issue slots or
+// shared-memory bandwidth.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128) S0 = Q0 K_j^T   (P0 = softmax numerators, 16-bit, aliases its first 64 columns)
@@ -90,20 +95,18 @@ struct FwdArgs {
 
 template <bool kFp8>
 struct FwdSmemLayout {
-  static constexpr int kElt = kFp8 ? 1 : 2;
-  static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;      // Q, K or V tile as loaded
+  static constexpr int kElt = kFp8 ? 1 : 2;                            // Q and K element bytes
+  static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;         // Q or K tile as loaded
+  static constexpr int kVTileBytes = kBlockN * kHeadDim * 2;           // V tile: bf16, or fp16 widened from e4m3
+  static constexpr int kSlotBytes = kVTileBytes;
   // One ring holds the K and V tiles in load order K_0, V_0, K_1, V_1, ...; they
   // are also released in that order (K_j when S1_j completes, V_j when PV1_j
   // completes), so the producer can run kRing tiles ahead of the MMAs.
-  static constexpr int kRing = kFp8 ? 8 : 5;
-  static_assert(!kFp8 || kRing % 2 == 0, "fp8 ring slots must keep one role (K or V)");
-  static constexpr int kStagesV16 = kFp8 ? 2 : 0;                    // fp8: V widened to fp16
-  static constexpr int kV16Bytes = kBlockN * kHeadDim * 2;
+  static constexpr int kRing = kFp8 ? 6 : 5;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTilesPerCta * kTileBytes;
-  static constexpr int kV16Off = kRingOff + kRing * kTileBytes;
-  static constexpr int kBarOff = kV16Off + kStagesV16 * kV16Bytes;
-  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8;
+  static constexpr int kBarOff = kRingOff + kRing * kSlotBytes;
+  static constexpr int kNumBars = 3 + 2 * kRing + 8;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -115,8 +118,6 @@ struct FwdBars {
   uint64_t* mma_drain;  // every MMA of the CTA has completed (committed once, at exit)
   uint64_t* ring_full;   // [kRing]
   uint64_t* ring_empty;  // [kRing]
-  uint64_t* v16_full;
-  uint64_t* v16_empty;
   uint64_t* s_full;   // [2]: S_t ready
   uint64_t* p_full;   // [2 tiles][2 halves of 64 keys]: P_t,h written (128 arrivals)
   uint64_t* o_done;   // [2]: last P V of the tile completed
@@ -125,7 +126,7 @@ struct FwdBars {
 
 // Barrier sites recorded in the error word when a wait times out.
 enum : int {
-  kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty, kSiteV16Full, kSiteV16Empty,
+  kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty,
   kSiteSFull, kSitePFull, kSiteODone, kSiteDrain
 };
 
@@ -197,8 +198,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     bb.mma_drain = p; p += 1;
     bb.ring_full = p; p += L::kRing;
     bb.ring_empty = p; p += L::kRing;
-    bb.v16_full = p; p += L::kStagesV16;
-    bb.v16_empty = p; p += L::kStagesV16;
     bb.s_full = p; p += 2;
     bb.p_full = p; p += 4;
     bb.o_done = p; p += 2;
@@ -211,11 +210,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     mbar_init(bb.mma_drain, 1);
     for (int s = 0; s < L::kRing; ++s) {
       mbar_init(&bb.ring_full[s], 1);
-      // fp8: odd slots always hold V (even ring), released by the 2 widening warps;
-      // every other slot is released by one MMA commit.
-      mbar_init(&bb.ring_empty[s], (kFp8 && (s & 1)) ? 2 : 1);
+      mbar_init(&bb.ring_empty[s], 1);
     }
-    for (int s = 0; s < L::kStagesV16; ++s) { mbar_init(&bb.v16_full[s], 2); mbar_init(&bb.v16_empty[s], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bb.s_full[i], 1);
       // one arrival per softmax warp (elected after __syncwarp), not per thread:
@@ -239,18 +235,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sRing = smem + L::kRingOff;
-  uint8_t* sV16 = smem + L::kV16Off;
 
-  // Register split (see kRegsSoftmax): the producer / MMA / widening warpgroup
-  // gives registers up, the two softmax warpgroups take them.
+  // Register split (see kRegsSoftmax): the producer / MMA warpgroup gives
+  // registers up, the two softmax warpgroups take them.
   if (warp >= 8) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsOther) : "memory");
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      constexpr int kBoxes = kFp8 ? 1 : 2;                 // 128-byte-wide boxes per 128-column row
+      constexpr int kBoxes = kFp8 ? 1 : 2;                 // 128-byte-wide boxes per 128-column Q/K row
       constexpr int kBoxBytes = L::kTileBytes / kBoxes;
       constexpr int kBoxCols = 128 / L::kElt;
+      constexpr int kVBoxBytes = L::kVTileBytes / 2;       // V: two boxes of 64 16-bit columns
       bool ok = true;
       int slot = 0, units = 0;
       uint32_t ph = 0;
@@ -271,11 +267,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         for (int n = 0; n < 2 * w.n_kv && ok; ++n, ++nseq) {
           if (nseq >= L::kRing) ok = mbar_wait(&bb.ring_empty[slot], ph ^ 1u, kSiteKEmpty);
           if (!ok) break;
-          mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
-          const CUtensorMap* tm = (n & 1) ? tv : tk;
-          for (int x = 0; x < kBoxes; ++x)
-            tma_load_3d(sRing + slot * L::kTileBytes + x * kBoxBytes, tm, &bb.ring_full[slot], x * kBoxCols,
-                        (n >> 1) * kBlockN, w.kvh);
+          uint8_t* dst = sRing + slot * L::kSlotBytes;
+          if (n & 1) {
+            mbar_arrive_expect_tx(&bb.ring_full[slot], L::kVTileBytes);
+            for (int x = 0; x < 2; ++x)
+              tma_load_3d(dst + x * kVBoxBytes, tv, &bb.ring_full[slot], x * 64, (n >> 1) * kBlockN, w.kvh);
+          } else {
+            mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
+            for (int x = 0; x < kBoxes; ++x)
+              tma_load_3d(dst + x * kBoxBytes, tk, &bb.ring_full[slot], x * kBoxCols, (n >> 1) * kBlockN, w.kvh);
+          }
           if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
         }
       }
@@ -295,7 +296,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       constexpr int kQKSteps = kFp8 ? 4 : 8;               // K = 32 (e4m3) or 16 (bf16) per MMA
       constexpr int kQKStepBytes = 32;
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
-      const uint32_t sV16a = smem_u32(sV16);
       // Descriptor halves: Q / K tiles K-major (SBO 1024 B), V MN-major (LBO 16 KB
       // between the two 64-column halves of the head dim, SBO 1024 B).
       constexpr uint32_t kHi = sdesc_hi(1024);
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       auto issue_qk = [&](int t, int kslot) {
         const uint32_t d = tmem + t * 128;
         const uint32_t a_lo = q_lo0 + t * (L::kTileBytes >> 4);
-        const uint32_t b_lo = ring_lo0 + kslot * (L::kTileBytes >> 4);
+        const uint32_t b_lo = ring_lo0 + kslot * (L::kSlotBytes >> 4);
 #pragma unroll
         for (int k = 0; k < kQKSteps; ++k) {
           // bf16: two 64-column swizzle atoms of 16 KB; step k in atom k/4 at byte (k%4)*32.
@@ -339,8 +339,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       };
 
       bool ok = true;
-      int kslot = 0, vs16 = 0, units = 0;
-      uint32_t kph = 0, vph16 = 0, jg = 0;
+      int kslot = 0, units = 0;
+      uint32_t kph = 0, jg = 0;
       for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
         const FwdUnit w = fwd_unit(args, u);
         const int n_kv = w.n_kv;
@@ -358,14 +358,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           int vslot = kslot;
           uint32_t vph = kph;
           next_pos(vslot, vph);                            // V_j follows K_j
-          uint32_t vbase;
-          if (kFp8) {
-            ok = mbar_wait(&bb.v16_full[vs16], vph16, kSiteV16Full);
-            vbase = sV16a + vs16 * L::kV16Bytes;
-          } else {
-            ok = mbar_wait(&bb.ring_full[vslot], vph, kSiteVFull);
-            vbase = sRa + vslot * L::kTileBytes;
-          }
+          ok = mbar_wait(&bb.ring_full[vslot], vph, kSiteVFull);
+          const uint32_t vbase = sRa + vslot * L::kSlotBytes;
           if (ok) ok = pv(0, vbase, jg, j);
           if (!ok) break;
           if (j == n_kv - 1) mma_commit(&bb.o_done[0]);
@@ -382,12 +376,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           }
           ok = pv(1, vbase, jg, j);
           if (!ok) break;
-          if (kFp8) {
-            mma_commit(&bb.v16_empty[vs16]);
-            if (++vs16 == L::kStagesV16) { vs16 = 0; vph16 ^= 1u; }
-          } else {
-            mma_commit(&bb.ring_empty[vslot]);
-          }
+          mma_commit(&bb.ring_empty[vslot]);
           if (j == n_kv - 1) mma_commit(&bb.o_done[1]);
           if (more) {
             issue_qk(1, kslot);
@@ -403,55 +392,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_wait_drain(bb.mma_drain, 0, kSiteDrain);
     }
     __syncwarp();
-  } else if (warp >= 10) {
-    // ------------------------------------------------------------ fp8: widen V to fp16
-    if constexpr (kFp8) {
-      const int t = threadIdx.x - 320;                       // 0..63
-      bool ok = true;
-      uint32_t jg = 0;                                       // this CTA's tile count
-      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step) {
-        const int n_kv = fwd_unit(args, u).n_kv;
-        for (int j = 0; j < n_kv && ok; ++j, ++jg) {
-          // V of tile jg sits at ring position 2 jg + 1
-          const int vslot = (int)((2u * jg + 1u) % L::kRing);
-          const uint32_t vph = ((2u * jg + 1u) / L::kRing) & 1u;
-          const int s16 = jg % L::kStagesV16;
-          const uint32_t u16 = jg / L::kStagesV16;
-          ok = warp_wait(&bb.ring_full[vslot], vph, kSiteVFull);
-          if (ok && jg >= (uint32_t)L::kStagesV16) ok = warp_wait(&bb.v16_empty[s16], (u16 - 1) & 1, kSiteV16Empty);
-          if (!ok) break;
-          const uint8_t* src = sRing + vslot * L::kTileBytes;
-          uint8_t* dst = sV16 + s16 * L::kV16Bytes;
-          // e4m3 tile: row r (key) = 128 bytes, 16-byte chunk c holds head dims [16c, 16c+16),
-          // stored at chunk c ^ (r & 7).  fp16 tile: two 64-dim halves of 16 KB; row r of a
-          // half = 128 bytes, chunk c8 holds dims [8 c8, 8 c8 + 8) of the half at c8 ^ (r & 7).
-#pragma unroll 4
-          for (int it = 0; it < 16; ++it) {
-            const int idx = t + 64 * it;
-            const int r = idx >> 3, c = idx & 7;
-            const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + ((c ^ (r & 7)) << 4));
-            const uint32_t wv[4] = {in.x, in.y, in.z, in.w};
-            uint32_t o[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              o[2 * q] = e4m3x2_to_f16x2((uint16_t)(wv[q] & 0xFFFFu));
-              o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(wv[q] >> 16));
-            }
-            const int half = c >> 2;
-            const int c8 = (c & 3) * 2;
-            uint8_t* rowp = dst + half * 16384 + r * 128;
-            *reinterpret_cast<uint4*>(rowp + ((c8 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(rowp + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&bb.v16_full[s16]);
-            mbar_arrive(&bb.ring_empty[vslot]);   // this warp is done reading the e4m3 slot
-          }
-        }
-      }
-    }
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax) : "memory");
@@ -618,6 +558,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// e4m3 -> fp16 widening of the V operand of the e4m3 forward (exact: every
+// e4m3 value is an fp16 value).  One 16-byte group of codes per thread and
+// step, grid-stride; HBM-bound.
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                         long long n16) {
+  for (long long i = (long long)blockIdx.x * 256 + threadIdx.x; i < n16; i += (long long)gridDim.x * 256) {
+    const uint4 in = __ldg(&src[i]);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      o[2 * q] = e4m3x2_to_f16x2((uint16_t)(w[q] & 0xFFFFu));
+      o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(w[q] >> 16));
+    }
+    dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 

@@ -139,19 +139,61 @@ bool sizes_fit(long long B, long long H, long long S) {
 
 // 3-D view (D, S, heads) of a [.., heads, S, D] tensor, box (box_x, 128 rows, 1 head),
 // 128-byte swizzle.  box_x * elt_bytes == 128.
-bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uint64_t heads) {
+bool encode_rows_typed(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t heads) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const uint64_t eb = e4m3 ? 1 : 2;
+  const uint64_t eb = dt == CU_TENSOR_MAP_DATA_TYPE_UINT8 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)(kHeadDim * eb), (cuuint64_t)(rows * kHeadDim * eb)};
   cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)kBlockM, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uint64_t heads) {
+  return encode_rows_typed(m, base, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rows,
+                           heads);
+}
+
+namespace {
+
+// Stream-ordered scratch for the fp16 copy of an e4m3 V.  Outside graph capture
+// it comes from a private pool per device that keeps up to kPoolKeepBytes
+// mapped between calls (a larger block is returned to the device when the
+// stream synchronizes); under capture it becomes a graph allocation node.
+constexpr uint64_t kPoolKeepBytes = 256ull << 20;
+
+int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return HATTN_ELAUNCH;
+  if (cs != cudaStreamCaptureStatusNone) return cudaMallocAsync(p, bytes, st) == cudaSuccess ? HATTN_OK : HATTN_EDEVICE;
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HATTN_EDEVICE;
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    if (!pools[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t np;
+      if (cudaMemPoolCreate(&np, &props) != cudaSuccess) return HATTN_EDEVICE;
+      uint64_t keep = kPoolKeepBytes;
+      cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep);
+      pools[dev] = np;
+    }
+    pool = pools[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? HATTN_OK : HATTN_EDEVICE;
+}
+
+}  // namespace
 
 }  // namespace hattn
 
@@ -176,7 +218,25 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   memset(&a, 0, sizeof(a));
   if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
   if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
-  if (!encode_rows(&a.tm_v[0], v, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* v16 = nullptr;
+  if (fp8) {
+    // V widened to fp16 once (exact), read by the attention kernel's P V MMAs
+    const long long n16 = (long long)B * Hkv * Sk * kHeadDim / 16;
+    if ((rc = scratch_alloc(&v16, (size_t)n16 * 32, st))) return rc;
+    const int sms = device_sm_count();
+    const long long want = (n16 + 255) / 256;
+    const int grid = (int)(want < 8LL * sms ? want : 8LL * sms);
+    widen_e4m3_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(reinterpret_cast<const uint4*>(v),
+                                                          reinterpret_cast<uint4*>(v16), n16);
+    if (cudaGetLastError() != cudaSuccess || !encode_rows_typed(&a.tm_v[0], v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Sk,
+                                                               (uint64_t)B * Hkv)) {
+      cudaFreeAsync(v16, st);
+      return HATTN_ELAUNCH;
+    }
+  } else if (!encode_rows(&a.tm_v[0], v, false, Sk, (uint64_t)B * Hkv)) {
+    return HATTN_ELAUNCH;
+  }
   a.sk[0] = Sk;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
   a.causal = causal ? 1 : 0;
@@ -186,8 +246,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   a.lse = lse;
   a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
   a.block_offset = 0;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
+  rc = fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
+  if (v16 && cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_EDEVICE;
+  return rc;
 }
 
 size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks) {
