@@ -157,12 +157,62 @@ bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uin
                            heads);
 }
 
+}  // namespace hattn
+
+using namespace hattn;
+
+extern "C" {
+
+size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtype) {
+  if (B <= 0 || Hkv <= 0 || Sk <= 0 || D <= 0 || dtype != HATTN_E4M3) return 0;
+  return (size_t)B * Hkv * Sk * D * 2;
+}
+
+}  // extern "C"
+
 namespace {
 
-// Stream-ordered scratch for the fp16 copy of an e4m3 V.  Outside graph capture
-// it comes from a private pool per device that keeps up to kPoolKeepBytes
-// mapped between calls (a larger block is returned to the device when the
-// stream synchronizes); under capture it becomes a graph allocation node.
+// Forward with the e4m3 V widened to fp16 in `v16` (B*Hkv*Sk*D*2 bytes) when
+// dtype is e4m3; v16 is unused for bf16.
+int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                  int Sq, int Sk, float scale, int causal, int dtype, const float* q_descale,
+                  const float* k_descale, const float* v_descale, void* v16, cudaStream_t st) {
+  const bool fp8 = dtype == HATTN_E4M3;
+  static thread_local FwdArgs a;   // ~8 KB: kept off the stack
+  memset(&a, 0, sizeof(a));
+  if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+  if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+  if (fp8) {
+    // V widened to fp16 once (exact), read by the attention kernel's P V MMAs
+    const long long n16 = (long long)B * Hkv * Sk * kHeadDim / 16;
+    const int sms = device_sm_count();
+    if (sms <= 0) return HATTN_EDEVICE;
+    const long long want = (n16 + 255) / 256;
+    const int grid = (int)(want < 8LL * sms ? want : 8LL * sms);
+    widen_e4m3_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(v), reinterpret_cast<uint4*>(v16), n16);
+    if (cudaGetLastError() != cudaSuccess) return HATTN_ELAUNCH;
+    if (!encode_rows_typed(&a.tm_v[0], v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Sk, (uint64_t)B * Hkv))
+      return HATTN_ELAUNCH;
+  } else if (!encode_rows(&a.tm_v[0], v, false, Sk, (uint64_t)B * Hkv)) {
+    return HATTN_ELAUNCH;
+  }
+  a.sk[0] = Sk;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
+  a.causal = causal ? 1 : 0;
+  a.n_qpairs = (Sq + kQTilesPerCta * kBlockM - 1) / (kQTilesPerCta * kBlockM);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
+  a.block_offset = 0;
+  return fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
+}
+
+// Stream-ordered scratch for attn_fwd callers that pass no workspace.  Outside
+// graph capture it comes from a private pool per device that keeps up to
+// kPoolKeepBytes mapped between calls (a larger block goes back to the device
+// when the stream synchronizes; remapping ~100 MB costs about a millisecond);
+// under capture it becomes a graph allocation node.
 constexpr uint64_t kPoolKeepBytes = 256ull << 20;
 
 int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
@@ -193,17 +243,9 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? HATTN_OK : HATTN_EDEVICE;
 }
 
-}  // namespace
-
-}  // namespace hattn
-
-using namespace hattn;
-
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
-             int Sk, int D, float scale, int causal, int dtype, const float* q_descale, const float* k_descale,
-             const float* v_descale, void* stream) {
+int check_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+              int Sk, int D, float scale, int causal, int dtype, const float* q_descale, const float* k_descale,
+              const float* v_descale) {
   if (!q || !k || !v || !out || !lse) return HATTN_EINVAL;
   int rc = check_common(B, Hq, Hkv, Sq, D, scale);
   if (rc) return rc;
@@ -212,42 +254,45 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
   if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk)) return HATTN_EUNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse)) return HATTN_EALIGN;
+  return HATTN_OK;
+}
 
-  const bool fp8 = dtype == HATTN_E4M3;
-  static thread_local FwdArgs a;   // ~8 KB: kept off the stack
-  memset(&a, 0, sizeof(a));
-  if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
-  if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  void* v16 = nullptr;
-  if (fp8) {
-    // V widened to fp16 once (exact), read by the attention kernel's P V MMAs
-    const long long n16 = (long long)B * Hkv * Sk * kHeadDim / 16;
-    if ((rc = scratch_alloc(&v16, (size_t)n16 * 32, st))) return rc;
-    const int sms = device_sm_count();
-    const long long want = (n16 + 255) / 256;
-    const int grid = (int)(want < 8LL * sms ? want : 8LL * sms);
-    widen_e4m3_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(reinterpret_cast<const uint4*>(v),
-                                                          reinterpret_cast<uint4*>(v16), n16);
-    if (cudaGetLastError() != cudaSuccess || !encode_rows_typed(&a.tm_v[0], v16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Sk,
-                                                               (uint64_t)B * Hkv)) {
-      cudaFreeAsync(v16, st);
-      return HATTN_ELAUNCH;
-    }
-  } else if (!encode_rows(&a.tm_v[0], v, false, Sk, (uint64_t)B * Hkv)) {
-    return HATTN_ELAUNCH;
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+                int Sk, int D, float scale, int causal, int dtype, const float* q_descale, const float* k_descale,
+                const float* v_descale, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, dtype, q_descale, k_descale, v_descale);
+  if (rc) return rc;
+  const size_t need = attn_fwd_workspace_size(B, Hkv, Sk, D, dtype);
+  if (need) {
+    if (!workspace) return HATTN_EINVAL;
+    if (!aligned16(workspace)) return HATTN_EALIGN;
+    if (workspace_bytes < need) return HATTN_EWORKSPACE;
   }
-  a.sk[0] = Sk;
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
-  a.causal = causal ? 1 : 0;
-  a.n_qpairs = (Sq + kQTilesPerCta * kBlockM - 1) / (kQTilesPerCta * kBlockM);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.out = out;
-  a.lse = lse;
-  a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
-  a.block_offset = 0;
-  rc = fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
-  if (v16 && cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_EDEVICE;
+  return attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale, v_descale,
+                       workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+             int Sk, int D, float scale, int causal, int dtype, const float* q_descale, const float* k_descale,
+             const float* v_descale, void* stream) {
+  int rc = check_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, dtype, q_descale, k_descale, v_descale);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t need = attn_fwd_workspace_size(B, Hkv, Sk, D, dtype);
+  if (!need)
+    return attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale,
+                         v_descale, nullptr, st);
+  // e4m3 without a caller workspace: stream-ordered scratch, released on the
+  // same stream after the kernels.
+  void* v16 = nullptr;
+  if ((rc = scratch_alloc(&v16, need, st))) return rc;
+  rc = attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale, v_descale,
+                     v16, st);
+  if (cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_EDEVICE;
   return rc;
 }
 

@@ -25,6 +25,10 @@ lib = ctypes.CDLL(LIB_PATH)
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp, _vp, _vp]
 lib.attn_fwd.restype = _i
+lib.attn_fwd_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.attn_fwd_ws.restype = _i
+lib.attn_fwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+lib.attn_fwd_workspace_size.restype = _sz
 lib.attn_fwd_kvblocks.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp,
                                   _vp, _sz, _vp]
 lib.attn_fwd_kvblocks.restype = _i
@@ -44,7 +48,7 @@ lib.attn_error_string.argtypes = [_i]
 lib.attn_error_string.restype = ctypes.c_char_p
 
 BF16, E4M3 = 0, 1
-EXPORTED = ("attn_fwd", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
+EXPORTED = ("attn_fwd", "attn_fwd_ws", "attn_fwd_workspace_size", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
             "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_error", "attn_selftest_bounded_wait",
             "attn_error_string")
 NOALLOC_MAX_ROWS = 1 << 22
@@ -86,9 +90,18 @@ def _require(t: torch.Tensor, name: str):
         raise ValueError("%s must be contiguous" % name)
 
 
+def fwd_workspace_size(B, Hkv, Sk, D, dtype) -> int:
+    return lib.attn_fwd_workspace_size(B, Hkv, Sk, D, dtype)
+
+
 def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, v_descale=None,
-             out=None, lse=None, stream=None):
-    """O [B,Hq,Sq,D] bf16 and LSE [B,Hq,Sq] fp32 for q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D]."""
+             out=None, lse=None, workspace=None, stream=None):
+    """O [B,Hq,Sq,D] bf16 and LSE [B,Hq,Sq] fp32 for q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D].
+
+    e4m3 inputs need scratch for the fp16 copy of V: `workspace` (a CUDA byte
+    tensor of at least fwd_workspace_size() bytes), else one from torch's
+    allocator; the library itself then allocates nothing.
+    """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _require(t, n)
     B, Hq, Sq, D = q.shape
@@ -99,8 +112,15 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
         out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
-                      int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _stream(stream))
+    ws_bytes = fwd_workspace_size(B, Hkv, Sk, D, dt)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace is not None:
+        _require(workspace, "workspace")
+    rc = lib.attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+                         int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
+                         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                         _stream(stream))
     _check(rc, "attn_fwd")
     return out, lse
 

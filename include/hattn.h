@@ -20,9 +20,10 @@
  *  - causal != 0 masks key j for query i unless j <= i + (Sk - Sq)
  *    (bottom-right aligned); it requires Sq <= Sk so every row sees a key.
  *  - All device pointers must be 16-byte aligned.
- *  - The caller owns every buffer.  Calls allocate nothing, never synchronise
- *    the host, and enqueue their kernels on `stream` (a cudaStream_t; NULL is
- *    the legacy default stream), so they may be captured into a CUDA graph.
+ *  - The caller owns every buffer.  Calls allocate nothing (one exception:
+ *    attn_fwd with e4m3 inputs, see there), never synchronise the host, and
+ *    enqueue their kernels on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream), so they may be captured into a CUDA graph.
  *  - Results are bitwise reproducible: every output element is written by one
  *    thread block, reductions run in a fixed order, and tile sizes do not depend
  *    on B, H or the number of SMs, so a row's result does not change with the
@@ -71,12 +72,31 @@ enum {
  *     one value per tensor is the case where all entries are equal); all three
  *     must be NULL for bf16.  Descales must be positive.
  * Softmax statistics and both matrix products accumulate in fp32.  For e4m3
- * inputs the probabilities are rounded to fp16 before the P V product.
+ * inputs S = Q K^T is an 8-bit product; V is first widened to fp16 (exactly)
+ * in scratch memory, and the probabilities are rounded to fp16 before the P V
+ * product.  attn_fwd takes that scratch (attn_fwd_workspace_size() bytes)
+ * stream-ordered from a memory pool of the library's own, which keeps up to
+ * 256 MB mapped between calls, and releases it on `stream` (under graph capture
+ * it becomes a graph allocation); attn_fwd_ws takes it from the caller instead
+ * and allocates nothing.
  */
 HATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int dtype,
              const float* q_descale, const float* k_descale, const float* v_descale,
              void* stream);
+
+/*
+ * attn_fwd with caller-provided scratch: workspace must hold at least
+ * attn_fwd_workspace_size(B, Hkv, Sk, D, dtype) bytes (B*Hkv*Sk*D*2 for e4m3,
+ * 0 for bf16, where workspace may be NULL); its contents on entry do not
+ * matter.  Too small a workspace returns HATTN_EWORKSPACE.
+ */
+HATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* out, float* lse,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int dtype,
+             const float* q_descale, const float* k_descale, const float* v_descale,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+HATTN_API size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtype);
 
 /*
  * Streaming forward over a block KV cache (FlashDreams PR #486 section 1.2;

@@ -71,6 +71,20 @@ def test_fwd_fails_closed(h, kw, code):
     assert fwd(h, **kw) == code
 
 
+def test_fwd_workspace_size_and_checks(h):
+    assert h.fwd_workspace_size(1, 5, 75600, 128, 1) == 5 * 75600 * 128 * 2    # e4m3: fp16 copy of V
+    assert h.fwd_workspace_size(2, 8, 2048, 128, 0) == 0                       # bf16 needs none
+    need = h.fwd_workspace_size(1, 2, 128, 128, 1)
+
+    def call(ws=B_, wsb=need, dtype=1):
+        d = A if dtype == 1 else None
+        return h.lib.attn_fwd_ws(A, A, A, A, A, 1, 2, 2, 128, 128, 128, 0.088, 0, dtype, d, d, d, ws, wsb, None)
+
+    assert call(wsb=need - 1) == -4
+    assert call(ws=None) == -1
+    assert call(ws=MIS) == -3
+
+
 def test_kvblocks_fails_closed(h):
     lib = h.lib
     kp = (ctypes.c_void_p * 2)(0x10000, 0x20000)

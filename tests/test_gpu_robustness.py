@@ -70,6 +70,38 @@ def test_cuda_graph_capture_matches_eager(h):
     assert torch.equal(lse_g, lse_e)
 
 
+def test_cuda_graph_capture_fp8_stream_ordered_scratch(h):
+    # the C attn_fwd with e4m3 allocates its fp16 V scratch stream-ordered; under
+    # capture that becomes a graph allocation, and replays equal the eager result
+    w = Workload("graph8", B=1, Hq=4, Hkv=2, Sq=300, Sk=400, dtype="e4m3", seed=79)
+    x = {k: v.cuda() for k, v in make_fwd_inputs(w).items()}
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def call(out, lse, stream):
+        return h.lib.attn_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(out), P(lse), 1, 4, 2, 300, 400, 128, w.scale, 0, 1,
+                              P(x["q_descale"]), P(x["k_descale"]), P(x["v_descale"]),
+                              ctypes.c_void_p(stream.cuda_stream))
+
+    out_e = torch.empty(1, 4, 300, 128, dtype=torch.bfloat16, device="cuda")
+    lse_e = torch.empty(1, 4, 300, dtype=torch.float32, device="cuda")
+    assert call(out_e, lse_e, torch.cuda.current_stream()) == 0
+    torch.cuda.synchronize()
+    out_g = torch.zeros_like(out_e)
+    lse_g = torch.zeros_like(lse_e)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            assert call(out_g, lse_g, s) == 0
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    assert torch.equal(out_g.view(torch.int16), out_e.view(torch.int16)) and torch.equal(lse_g, lse_e)
+    del g
+
+
 def test_fail_closed_on_device(h):
     q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")     # head dim 64 is not offered
     with pytest.raises(h.HattnError) as ei:
