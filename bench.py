@@ -9,7 +9,9 @@ that is already resident in HBM:
   fp8        attn_fwd on e4m3 inputs with per-head descales, B=1 H=5 S=75600;
   llm_gqa    attn_fwd + attn_bwd, B=2 Hq=32 Hkv=8 S=2048 causal;
   streaming  attn_fwd_kvblocks over 21 blocks of 1560 keys + attn_fwd to 512
-             text keys, B=1 H=40 Sq=1560.
+             text keys, B=1 H=40 Sq=1560;
+  cross      attn_fwd, B=1 H=40 Sq=90000 Sk=512 (long-query cross-attention);
+  window     attn_fwd, B=1 H=12 Sq=4680 Sk=51480 (window / sink KV).
 The other workloads are measured too (``sub``) unless --no-sub.
 
 Timing: W untimed warm-up steps; then K steps, each preceded (outside its
@@ -50,7 +52,10 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "video": "video-DiT self-attention fwd (B1 H40 S32760 D128 bf16, Q/K RMS-norm)",
                   "fp8": "fp8 e4m3 attention fwd (B1 H5 S75600 D128, per-head descales)",
                   "llm_gqa": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16)",
-                  "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)"}
+                  "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)",
+                  "cross": "long-query cross-attention fwd (B1 H40 Sq90000 Sk512 D128 bf16)",
+                  "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)"}
+FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window")
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
 
@@ -88,7 +93,7 @@ def recorded_traffic(workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    """nvidia-smi clock / throttle-reason samples every 100 ms while running."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -104,7 +109,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -194,7 +199,7 @@ class Step:
             self.w = workloads.get(name, seed=self.w.seed + 7919 * rank, Hq=self.w.Hq, Hkv=self.w.Hkv)
         w = self.w
         self.launches = 1
-        if name in ("video", "fp8", "tiny"):
+        if name in FWD_WORKLOADS:
             x = make_fwd_inputs(w)
             self.host = x
             self.x = {k: v.cuda() for k, v in x.items()}
@@ -202,6 +207,8 @@ class Step:
             self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
             self.flops = w.fwd_flops()
             self.dtype = "e4m3" if name == "fp8" else "bf16"
+            if name == "fp8":
+                self.launches = 2          # V widened to fp16, then the attention kernel
         elif name == "llm_gqa":
             x = make_bwd_inputs(w)
             self.host = x
@@ -236,7 +243,7 @@ class Step:
 
     def __call__(self):
         h, w = self.h, self.w
-        if self.name in ("video", "fp8", "tiny"):
+        if self.name in FWD_WORKLOADS:
             x = self.x
             ds = {}
             if self.name == "fp8":
@@ -357,7 +364,7 @@ def run_reference(args, world, rank):
         return 0
     name = args.workload
     w = workloads.get(name)
-    rows = {"tiny": 256, "video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64}[name]
+    rows = {"tiny": 256, "video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64, "cross": 256, "window": 48}[name]
     vals = []
     for _ in range(args.warmup):
         oracle_sample_tflops(name, rows)
@@ -381,7 +388,7 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOAD_NAMES), default="video")
@@ -414,7 +421,9 @@ def main(argv=None):
 
     fp8 = step.dtype == "e4m3"
     peak_tensor = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
-    achieved = step.flops / (statistics.mean(ms) * 1e-3) / 1e12 if step.launches == 1 else None
+    # the dominant kernel is the attention kernel; an e4m3 step also widens V
+    # (an HBM-bound pass of about 0.5 % of the step), which this figure includes
+    achieved = step.flops / (statistics.mean(ms) * 1e-3) / 1e12 if name in FWD_WORKLOADS else None
     w = step.w
     roofline = None
     if achieved is not None:
@@ -435,7 +444,7 @@ def main(argv=None):
                        "l2": "256 MB write before each timed step, outside its CUDA events"},
             "gpu_launches": step.launches * args.steps,
             "clocks": clocks, "roofline": roofline}
-    if not args.no_e2e and name in ("video", "fp8", "tiny"):
+    if not args.no_e2e and name in FWD_WORKLOADS:
         e2e = e2e_video_like(step, max(2, args.steps // 2), 1)
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world)
         e2e["value"] = world * step.flops / (e2e["ms_per_step"] * 1e-3) / 1e12

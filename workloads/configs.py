@@ -15,6 +15,12 @@ Shapes follow the pages' workloads:
   block KV cache of 21 blocks, plus cross-attention to 512 text tokens
   (FlashDreams PR #486, section 1.2: streaming self-attention over a block KV
   cache and static cross-attention).
+
+Two more shapes from the pages' streaming workloads, measured beside these:
+- cross: long-query cross-attention, Sq=90000 video tokens against Sk=512 text
+  tokens with 40 heads (AITER PR #2911, the Wan 2.2 cross-attention report);
+- window: the raw SDPA call on the window-30 shape, 4680 queries against 51480
+  keys with 12 heads (FlashDreams issue #739, "SDPA kernels on gfx950").
 """
 from __future__ import annotations
 
@@ -64,6 +70,8 @@ CONFIGS = {
     "fp8": Workload("fp8", B=1, Hq=5, Hkv=5, Sq=75600, Sk=75600, dtype="e4m3", seed=3),
     "streaming": Workload("streaming", B=1, Hq=40, Hkv=40, Sq=1560, Sk=21 * 1560, seed=4,
                           n_blocks=21, text_len=512),
+    "cross": Workload("cross", B=1, Hq=40, Hkv=40, Sq=90000, Sk=512, seed=5),
+    "window": Workload("window", B=1, Hq=12, Hkv=12, Sq=4680, Sk=51480, seed=6),
 }
 
 
