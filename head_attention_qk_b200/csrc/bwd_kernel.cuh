@@ -248,28 +248,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      auto sQ_of = [&](int n) { return smem_u32(smem + L::kQ + (n & 1) * kTileBytesBf16); };
+      auto sDO_of = [&](int n) { return smem_u32(smem + L::kDO + (n & 1) * kTileBytesBf16); };
+      // Issue order per step n: dV_n (once P^T_n is written), S^T_{n+1} (its
+      // columns held P^T_n, which dV_n has read: one thread's MMAs run in
+      // order), dK_n (once dS^T_n is written), dP^T_{n+1}.  The next step's S^T
+      // thus runs while the compute warps form dS^T of this one.
       bool ok = mbar_wait(kv_full, 0, kSiteBwdKV);
-      for (int n = 0; n < steps && ok; ++n) {
-        const int s = n & 1, u = n >> 1;
-        ok = mbar_wait(&st_full[s], u & 1, kSiteBwdStFull);
-        if (!ok) break;
+      if (ok && steps > 0) ok = mbar_wait(&st_full[0], 0, kSiteBwdStFull);
+      if (ok && steps > 0) {
         tc_fence_after();
-        const uint32_t sQ = smem_u32(smem + L::kQ + s * kTileBytesBf16);
-        const uint32_t sDO = smem_u32(smem + L::kDO + s * kTileBytesBf16);
-        mma_tile_ss_kmajor(tmem + 256, sK, sQ, 0);        // S^T  = K Q^T
+        mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(0), 0);   // S^T  = K Q^T
         mma_commit(s_full);
-        mma_tile_ss_kmajor(tmem + 384, sV, sDO, 0);       // dP^T = V dO^T
+        mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(0), 0);  // dP^T = V dO^T
         mma_commit(dp_full);
-        // dV needs only P^T, so it runs while the compute warps form dS^T
+      }
+      for (int n = 0; n < steps && ok; ++n) {
+        const bool more = n + 1 < steps;
         ok = mbar_wait(p_full, n & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO, n > 0);    // dV += P^T dO
+        mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO_of(n), n > 0);    // dV += P^T dO
+        if (more) {
+          ok = mbar_wait(&st_full[(n + 1) & 1], ((n + 1) >> 1) & 1, kSiteBwdStFull);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step
+          mma_commit(s_full);
+        }
         ok = mbar_wait(ds_full, n & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ, n > 0);   // dK += dS^T Q
-        mma_commit(&st_empty[s]);
+        mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ_of(n), n > 0);   // dK += dS^T Q
+        mma_commit(&st_empty[n & 1]);
+        if (more) {
+          mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(n + 1), 0);         // dP^T of the next step
+          mma_commit(dp_full);
+        }
       }
       mma_commit(acc_done);
       mbar_wait(acc_done, 0, kSiteBwdDone);
@@ -411,11 +426,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   uint64_t* k_empty = bars + 3;   // [2]
   uint64_t* v_full = bars + 5;    // [2]
   uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;
-  uint64_t* dp_full = bars + 10;
-  uint64_t* ds_full = bars + 11;
-  uint64_t* dq_done = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* s_full = bars + 9;    // [2 S buffers]
+  uint64_t* dp_full = bars + 11;
+  uint64_t* ds_full = bars + 12;
+  uint64_t* dq_done = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -423,7 +438,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
     mbar_init(ds_full, kTile / 32);  // one arrival per compute warp
     mbar_init(dq_done, 1);
@@ -434,7 +450,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S / dS [0,128), dP [128,256), dQ [256,384)
+  // TMEM columns: S / dS buffer 0 [0,128), dP [128,256), dQ [256,384), S / dS buffer 1 [384,512)
+  auto s_col = [](int jj) { return (jj & 1) ? 384u : 0u; };
 
   if (warp == 4) {
     if (lane == 0) {
@@ -463,25 +480,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   } else if (warp == 5) {
     if (lane == 0) {
       const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-      bool ok = mbar_wait(q_full, 0, kSiteBwdKV);
-      for (int jj = 0; jj < n_kv && ok; ++jj) {
-        const int s = jj & 1, u = jj >> 1;
-        const uint32_t sK = smem_u32(smem + L::kK + s * kTileBytesBf16);
-        const uint32_t sV = smem_u32(smem + L::kV + s * kTileBytesBf16);
-        ok = mbar_wait(&k_full[s], u & 1, kSiteBwdStFull);
-        if (ok) ok = mbar_wait(&v_full[s], u & 1, kSiteBwdStFull);
-        if (!ok) break;
+      auto sK_of = [&](int jj) { return smem_u32(smem + L::kK + (jj & 1) * kTileBytesBf16); };
+      auto sV_of = [&](int jj) { return smem_u32(smem + L::kV + (jj & 1) * kTileBytesBf16); };
+      // S is double-buffered in TMEM: S_{j+1} is computed while the compute
+      // warps work on step j.  Issue order: S_0, dP_0, S_1, then per step j:
+      // dQ_j (once dS_j is written), dP_{j+1} (the compute warps have read dP_j),
+      // S_{j+2} into the buffer dQ_j has just read dS_j from.
+      auto issue_s = [&](int jj) -> bool {
+        if (!mbar_wait(&k_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull)) return false;
         tc_fence_after();
-        mma_tile_ss_kmajor(tmem + 0, sQ, sK, 0);          // S  = Q K^T
-        mma_commit(s_full);
-        mma_tile_ss_kmajor(tmem + 128, sDO, sV, 0);       // dP = dO V^T
+        mma_tile_ss_kmajor(tmem + s_col(jj), sQ, sK_of(jj), 0);         // S  = Q K^T
+        mma_commit(&s_full[jj & 1]);
+        return true;
+      };
+      auto issue_dp = [&](int jj) -> bool {
+        if (!mbar_wait(&v_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull)) return false;
+        tc_fence_after();
+        mma_tile_ss_kmajor(tmem + 128, sDO, sV_of(jj), 0);              // dP = dO V^T
         mma_commit(dp_full);
-        mma_commit(&v_empty[s]);
+        mma_commit(&v_empty[jj & 1]);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, kSiteBwdKV);
+      if (ok && n_kv > 0) ok = issue_s(0) && issue_dp(0);
+      if (ok && n_kv > 1) ok = issue_s(1);
+      for (int jj = 0; jj < n_kv && ok; ++jj) {
         ok = mbar_wait(ds_full, jj & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 256, tmem + 0, sK, jj > 0);   // dQ += dS K
-        mma_commit(&k_empty[s]);
+        mma_tile_ts_mnmajor(tmem + 256, tmem + s_col(jj), sK_of(jj), jj > 0);   // dQ += dS K
+        mma_commit(&k_empty[jj & 1]);
+        if (jj + 1 < n_kv) ok = issue_dp(jj + 1);
+        if (ok && jj + 2 < n_kv) ok = issue_s(jj + 2);
       }
       mma_commit(dq_done);
       mbar_wait(dq_done, 0, kSiteBwdDone);
@@ -499,11 +529,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     const float c = a.scale_log2;
     bool ok = true;
     for (int jj = 0; jj < n_kv && ok; ++jj) {
-      ok = warp_wait(s_full, jj & 1, kSiteBwdS);
+      ok = warp_wait(&s_full[jj & 1], (jj >> 1) & 1, kSiteBwdS);
       if (!ok) break;
       tc_fence_after();
       float p[128];
-      tmem_load_row128(tmem + lane_base + 0, p);
+      tmem_load_row128(tmem + lane_base + s_col(jj), p);
       const int kbase = jj * kTile;
       const bool need_mask = kbase + kTile - 1 > kv_limit;
 #pragma unroll
@@ -526,7 +556,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
           for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
         }
       }
-      tmem_store_bf16_row128(tmem + lane_base + 0, p);     // dS over S's first 64 columns
+      tmem_store_bf16_row128(tmem + lane_base + s_col(jj), p);   // dS over its S buffer's first 64 columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
