@@ -17,9 +17,16 @@
 //                     KV tiles (ascending).  Per step, three MMAs:
 //                       S = Q K^T, dP = dO V^T, dQ += dS K.
 //
-// Roles: warps 0-3 compute (one TMEM lane / tile row per thread), warp 4 TMA
-// producer, warp 5 MMA issuer and tensor-memory owner.  P and dS are rounded to
-// bf16 before their MMAs; S, dP and the dQ/dK/dV accumulators are fp32.
+// Roles: warps 0-7 compute, warp 8 TMA producer, warp 9 MMA issuer and
+// tensor-memory owner.  Compute warp w owns tile rows 32 (w % 4) .. +31 (its
+// TMEM lane quarter) and columns 64 (w / 4) .. +63 of S, dP: nothing in P or dS
+// needs a reduction along a row (the row statistics LSE and Delta come from the
+// forward), so the two warps of a lane quarter split the columns, and two
+// warps per SM sub-partition keep the MUFU exponentials fed.  Each writes its
+// 16-bit P or dS into the first 32 of its own 64 S / dP columns, so the MMAs
+// read them with a 32-column gap after the first 64 keys.  P and dS are
+// rounded to bf16 before their MMAs; S, dP and the dQ/dK/dV accumulators are
+// fp32.
 #pragma once
 
 #include "fwd_kernel.cuh"
@@ -27,7 +34,8 @@
 
 namespace hattn {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdComputeWarps = 8;
 constexpr int kTile = 128;
 constexpr int kTileBytesBf16 = kTile * kHeadDim * 2;     // 32 KB, two 16 KB swizzle halves
 
@@ -84,50 +92,22 @@ __device__ __forceinline__ void mma_tile_ss_kmajor(uint32_t d, uint32_t sa, uint
 
 // D (+)= A B where A (128 x 128, bf16 pairs) is in tensor memory and B is a
 // shared-memory tile read MN-major: the reduction runs over the tile's rows.
+// A's reduction elements 0..63 sit in columns [0, 32) and 64..127 in [64, 96)
+// (each half written by the warp that owns those 64 columns of S or dP).
 __device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
   constexpr uint32_t idesc = make_idesc(1, 1, 1, 128, 128);
   constexpr uint32_t hi = sdesc_hi(1024);
   const uint32_t b_lo = sdesc_lo(sb, 16384);
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    mma_f16_ts2(d, a_tmem + k * 8, b_lo + k * (2048 >> 4), hi, idesc, (acc || k > 0) ? 1u : 0u);
+    mma_f16_ts2(d, a_tmem + k * 8 + (k >> 2) * 32, b_lo + k * (2048 >> 4), hi, idesc, (acc || k > 0) ? 1u : 0u);
 }
 
-__device__ __forceinline__ void tmem_load_row128(uint32_t taddr, float (&x)[128]) {
-  uint32_t u[128];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[q * 32]));
-  tmem_wait_ld();
-#pragma unroll
-  for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
-}
-
-// Same, one 32-column chunk at a time (fewer live registers).
-__device__ __forceinline__ void tmem_load_row128_chunked(uint32_t taddr, float (&x)[128]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint32_t u[32];
-    tmem_ld32(taddr + q * 32, u);
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 32; ++e) x[q * 32 + e] = __uint_as_float(u[e]);
-  }
-}
-
-__device__ __forceinline__ void tmem_store_bf16_row128(uint32_t taddr, const float (&x)[128]) {
-  uint32_t u[32];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) u[e] = pack_bf16x2(x[q * 64 + 2 * e], x[q * 64 + 2 * e + 1]);
-    tmem_st32(taddr + q * 32, u);
-  }
-}
-
-// Read a 128-column fp32 TMEM row, scale it and store it as bf16 to global memory.
-__device__ __forceinline__ void store_row_bf16(uint32_t taddr, float mul, uint16_t* dst, bool store) {
+// Read 64 columns of an fp32 TMEM row (from taddr), scale them and store them as
+// bf16 to global memory at dst.
+__device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, uint16_t* dst, bool store) {
 #pragma unroll 1
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < 2; ++q) {
     uint32_t u[32];
     __syncwarp();
     tmem_ld32(taddr + q * 32, u);
@@ -196,19 +176,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], 1); }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, kTile / 32);   // one arrival per compute warp
-    mbar_init(ds_full, kTile / 32);
+    mbar_init(p_full, kBwdComputeWarps);   // one arrival per compute warp
+    mbar_init(ds_full, kBwdComputeWarps);
     mbar_init(acc_done, 1);
     fence_barrier_init();
   }
-  if (warp == 5) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384), dP^T / dS^T [384,512)
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * kTileBytesBf16);
@@ -244,7 +224,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       for (int n = max(0, steps - 2); n < steps; ++n) mbar_wait(&st_full[n & 1], (n >> 1) & 1, kSiteBwdStFull);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
@@ -291,9 +271,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- compute (warps 0-3)
-    const int r = threadIdx.x;                       // key row within the tile
+    // ---------------------------------------------------------------- compute (warps 0-7)
+    const int r = (warp & 3) * 32 + lane;            // key row within the tile
+    const int hc = warp >> 2;                        // column half: queries 64 hc .. 64 hc + 63
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + 256 + hc * 64;   // this warp's 64 S^T (then P^T) columns
+    const uint32_t tP = tmem + lane_base + 384 + hc * 64;   // this warp's 64 dP^T (then dS^T) columns
     const int kj = j * kTile + r;
     const float c = a.scale_log2;
     bool ok = true;
@@ -304,17 +287,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       if (ok) ok = warp_wait(s_full, n & 1, kSiteBwdS);
       if (!ok) break;
       tc_fence_after();
-      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + s * 2 * kTile * 4);
+      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + s * 2 * kTile * 4) + hc * 16;
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
-      const bool need_mask = a.causal && (i * kTile < lim);
+      const int q_first = i * kTile + hc * 64;       // first query of this warp's columns
+      const bool need_mask = a.causal && (q_first < lim);
       const float2 c2 = make_float2(c, c);
-      // P^T row as 64 bf16 pairs: the values dV's MMA consumes, reused for dS^T
-      uint32_t pk[64];
+      // P^T as 32 bf16 pairs: the values dV's MMA consumes, reused for dS^T
+      uint32_t pk[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         uint32_t u[32];
-        tmem_ld32(tmem + lane_base + 256 + q * 32, u);
+        tmem_ld32(tS + q * 32, u);
         tmem_wait_ld();
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
@@ -326,7 +310,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                                        c2, make_float2(-l4.z, -l4.w));
           float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x), p3 = ex2_approx(x1.y);
           if (need_mask) {
-            const int q0 = i * kTile + e;
+            const int q0 = q_first + e;
             p0 = q0 < lim ? 0.f : p0;
             p1 = q0 + 1 < lim ? 0.f : p1;
             p2 = q0 + 2 < lim ? 0.f : p2;
@@ -337,19 +321,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         }
       }
       __syncwarp();
-#pragma unroll
-      for (int q = 0; q < 2; ++q) tmem_st32(tmem + lane_base + 256 + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[q * 32]));
+      tmem_st32(tS, pk);                             // P^T over the first 32 of these columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);                // P^T over S^T's first 64 columns
+      if (lane == 0) mbar_arrive(p_full);
       ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         uint32_t uu[32];
-        tmem_ld32(tmem + lane_base + 384 + q * 32, uu);
+        tmem_ld32(tP + q * 32, uu);
         tmem_wait_ld();
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
@@ -367,8 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         }
       }
       __syncwarp();
-#pragma unroll
-      for (int q = 0; q < 2; ++q) tmem_st32(tmem + lane_base + 384 + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[q * 32]));
+      tmem_st32(tP, pk);                             // dS^T over the first 32 of these columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -377,16 +359,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
     if (ok) {
       tc_fence_after();
+      // this warp stores head dims 64 hc .. 64 hc + 63 of its rows of dV and dK
       const bool store = kj < a.Sk;
-      const size_t off = ((size_t)bkv * a.Sk + (store ? kj : 0)) * kHeadDim;
-      store_row_bf16(tmem + lane_base + 0, 1.f, a.dv + off, store);
-      store_row_bf16(tmem + lane_base + 128, a.scale, a.dk + off, store);
+      const size_t off = ((size_t)bkv * a.Sk + (store ? kj : 0)) * kHeadDim + hc * 64;
+      store_half_row_bf16(tmem + lane_base + 0 + hc * 64, 1.f, a.dv + off, store);
+      store_half_row_bf16(tmem + lane_base + 128 + hc * 64, a.scale, a.dk + off, store);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+  if (warp == 9) { tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
 // ---------------------------------------------------------------------------- dQ
@@ -441,11 +424,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, kTile / 32);  // one arrival per compute warp
+    mbar_init(ds_full, kBwdComputeWarps);  // one arrival per compute warp
     mbar_init(dq_done, 1);
     fence_barrier_init();
   }
-  if (warp == 5) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -453,7 +436,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   // TMEM columns: S / dS buffer 0 [0,128), dP [128,256), dQ [256,384), S / dS buffer 1 [384,512)
   auto s_col = [](int jj) { return (jj & 1) ? 384u : 0u; };
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * kTileBytesBf16);
       tma_tile_bf16(smem + L::kQ, &a.tm_q, q_full, i * kTile, bh);
@@ -477,7 +460,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
       auto sK_of = [&](int jj) { return smem_u32(smem + L::kK + (jj & 1) * kTileBytesBf16); };
@@ -518,7 +501,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     }
     __syncwarp();
   } else {
-    const int r = threadIdx.x;
+    const int r = (warp & 3) * 32 + lane;            // query row within the tile
+    const int hc = warp >> 2;                        // column half: keys 64 hc .. 64 hc + 63
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int qi = i * kTile + r;
     const bool valid = qi < a.Sq;
@@ -532,12 +516,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       ok = warp_wait(&s_full[jj & 1], (jj >> 1) & 1, kSiteBwdS);
       if (!ok) break;
       tc_fence_after();
-      float p[128];
-      tmem_load_row128(tmem + lane_base + s_col(jj), p);
-      const int kbase = jj * kTile;
-      const bool need_mask = kbase + kTile - 1 > kv_limit;
+      const uint32_t tS = tmem + lane_base + s_col(jj) + hc * 64;   // this warp's 64 S (then dS) columns
+      float p[64];
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
+      for (int q = 0; q < 2; ++q) {
+        uint32_t u[32];
+        tmem_ld32(tS + q * 32, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) p[q * 32 + e] = __uint_as_float(u[e]);
+      }
+      const int kbase = jj * kTile + hc * 64;
+      const bool need_mask = kbase + 63 > kv_limit;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
         float x = ex2_approx(fmaf(p[e], c, -lse2));
         if (need_mask && kbase + e > kv_limit) x = 0.f;
         p[e] = x;
@@ -549,14 +541,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       {
         uint32_t uu[32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          tmem_ld32(tmem + lane_base + 128 + q * 32, uu);
+        for (int q = 0; q < 2; ++q) {
+          tmem_ld32(tmem + lane_base + 128 + hc * 64 + q * 32, uu);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
         }
       }
-      tmem_store_bf16_row128(tmem + lane_base + s_col(jj), p);   // dS over its S buffer's first 64 columns
+      {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+        tmem_st32(tS, w);                            // dS over the first 32 of these columns
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -565,13 +562,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     if (ok) ok = warp_wait(dq_done, 0, kSiteBwdDone);
     if (ok) {
       tc_fence_after();
-      store_row_bf16(tmem + lane_base + 256, a.scale, a.dq + ridx * kHeadDim, valid);
+      store_half_row_bf16(tmem + lane_base + 256 + hc * 64, a.scale, a.dq + ridx * kHeadDim + hc * 64, valid);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+  if (warp == 9) { tc_fence_after(); tmem_dealloc(tmem, 512); }
 }
 
 // ---------------------------------------------------------------------------- host launch
