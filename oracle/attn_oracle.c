@@ -327,6 +327,90 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
     return failed ? -2 : 0;
 }
 
+/*
+ * e4m3 quantisation prologue: the step before fp8 attention.
+ * FlashDreams PR #486 "flashdreams.accelerated API v0": section 1.1
+ * Quantization toolkit (FP8 E4M3 with tensor- or slice-granularity scales)
+ * and section 1.2 (head-scoped Q/K normalization, optional FP8 SDPA); the
+ * clamp to the e4m3fn range +-448 as VeOmni PR #1363 describes its quantizers.
+ * The pages give no formula; the readings (listed in the design notes) are:
+ * the scale slice is one (batch, head); the optional normalisation is a plain
+ * RMS over the head dimension with eps and no weight; and each step is fixed
+ * in precision and order, so that every code is a function of the input:
+ *   sum_b   = sum over d = 0 .. D-1 ascending of x_d^2   (fp64, each square exact)
+ *   r       = 1 / sqrt(sum_b / D + eps)                  (fp64, correctly rounded)
+ *   y_d     = (float)(x_d * r)  (fp64 product, rounded to fp32); y = x without it
+ *   amax    = max |y| over the head's S x D values       (fp32)
+ *   descale = amax / 448 in fp32, or 1 when amax == 0
+ *   code    = e4m3 of y / descale (fp32 quotient), rounded to nearest with
+ *             ties to the even code, saturating at +-448; the sign bit is the
+ *             quotient's.
+ */
+
+/* The 127 non-negative finite e4m3fn values in code order (codes 0x00..0x7E),
+ * from the format definition; ascending. */
+static double e4m3_pos_value(int code) { return oracle_e4m3_to_double((uint8_t)code); }
+
+uint8_t oracle_e4m3_rne(float v) {
+    if (isnan(v)) return 0x7F;
+    const int neg = signbit(v) ? 1 : 0;
+    const double a = fabs((double)v);
+    int code;
+    if (a >= 448.0) {
+        code = 0x7E;                           /* saturate */
+    } else {
+        /* largest code whose value is <= a (binary search over ascending values) */
+        int lo = 0, hi = 0x7E;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) / 2;
+            if (e4m3_pos_value(mid) <= a) lo = mid; else hi = mid - 1;
+        }
+        code = lo;
+        if (e4m3_pos_value(code) < a) {        /* between code and code + 1 */
+            const double dl = a - e4m3_pos_value(code), dh = e4m3_pos_value(code + 1) - a;
+            if (dh < dl || (dh == dl && ((code + 1) & 1) == 0)) code = code + 1;
+        }
+    }
+    return (uint8_t)(code | (neg << 7));
+}
+
+int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int B, int H, int S, int D,
+                         int rmsnorm, double eps) {
+    if (B <= 0 || H <= 0 || S <= 0 || D <= 0 || !x || !codes || !descale) return -1;
+    const int64_t heads = (int64_t)B * H;
+    int failed = 0;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < heads; ++bh) {
+        float* y = (float*)malloc(sizeof(float) * (size_t)S * D);
+        if (!y) { failed = 1; continue; }
+        const uint16_t* xh = x + bh * (int64_t)S * D;
+        float amax = 0.f;
+        for (int64_t s = 0; s < S; ++s) {
+            double r = 1.0;
+            if (rmsnorm) {
+                double sum = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double v = bf16_to_double(xh[s * D + d]);
+                    sum += v * v;
+                }
+                r = 1.0 / sqrt(sum / (double)D + eps);
+            }
+            for (int d = 0; d < D; ++d) {
+                const double v = bf16_to_double(xh[s * D + d]);
+                const float yv = rmsnorm ? (float)(v * r) : (float)v;
+                y[s * D + d] = yv;
+                if (fabsf(yv) > amax) amax = fabsf(yv);
+            }
+        }
+        const float ds = amax > 0.f ? amax / 448.0f : 1.0f;
+        descale[bh] = ds;
+        uint8_t* ch = codes + bh * (int64_t)S * D;
+        for (int64_t i = 0; i < (int64_t)S * D; ++i) ch[i] = oracle_e4m3_rne(y[i] / ds);
+        free(y);
+    }
+    return failed ? -2 : 0;
+}
+
 /* Number of OpenMP threads a parallel region will use (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

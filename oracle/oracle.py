@@ -62,6 +62,10 @@ def _load():
             lib.oracle_e4m3_to_double.restype = cd
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ci
+            lib.oracle_e4m3_rne.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_rne.restype = ctypes.c_uint8
+            lib.oracle_quantize_e4m3.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd]
+            lib.oracle_quantize_e4m3.restype = ci
             _lib = lib
     return _lib
 
@@ -86,6 +90,27 @@ def num_threads() -> int:
 
 def e4m3_to_double(code: int) -> float:
     return _load().oracle_e4m3_to_double(int(code) & 0xFF)
+
+
+def e4m3_rne(v: float) -> int:
+    """e4m3fn code of an fp32 value: nearest, ties to the even code, saturating at +-448."""
+    return int(_load().oracle_e4m3_rne(float(np.float32(v))))
+
+
+def quantize_e4m3(x_bits, rmsnorm=False, eps=1e-6):
+    """e4m3 prologue (see attn_oracle.c): bf16 bits [B,H,S,D] -> (codes uint8 [B,H,S,D],
+    descale float32 [B,H])."""
+    x_bits = np.ascontiguousarray(x_bits)
+    if x_bits.dtype != np.uint16 or x_bits.ndim != 4:
+        raise TypeError("quantize_e4m3 takes [B,H,S,D] uint16 bf16 bit patterns")
+    B, H, S, D = x_bits.shape
+    codes = np.empty(x_bits.shape, dtype=np.uint8)
+    descale = np.empty((B, H), dtype=np.float32)
+    rc = _load().oracle_quantize_e4m3(_ptr(x_bits), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)),
+                                      float(eps))
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_e4m3 failed with code %d" % rc)
+    return codes, descale
 
 
 def attn_fwd(q, k, v, scale, causal=False, rows=None, descales=None):

@@ -1,0 +1,124 @@
+"""Pins of the oracle's e4m3 quantisation prologue (oracle/attn_oracle.c,
+oracle_quantize_e4m3 and oracle_e4m3_rne) against things other than itself:
+torch's own float8_e4m3fn cast, the e4m3fn value table, closed forms of the
+RMS normalisation on special rows, exact scale invariance, and the harness's
+independent torch quantiser."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import bf16_bits
+from workloads.gen import quantize_e4m3_per_head
+
+
+def torch_e4m3(v: torch.Tensor) -> np.ndarray:
+    return v.float().clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_rne_matches_torch_cast_across_magnitudes():
+    g = torch.Generator().manual_seed(5)
+    parts = [torch.randn(20000, generator=g) * s for s in (1e-3, 0.02, 1.0, 30.0, 300.0)]
+    # exact ties: midpoints between neighbouring codes (normal and subnormal ranges)
+    vals = torch.arange(0, 0x7E, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).float()
+    mids = (vals[:-1] + vals[1:]) / 2
+    v = torch.cat(parts + [mids, -mids, torch.tensor([0.0, -0.0, 448.0, 449.0, 1e6, -1e6, 2.0 ** -10, 2.0 ** -11])])
+    ours = np.array([oracle.e4m3_rne(float(x)) for x in v.numpy()], dtype=np.uint8)
+    assert np.array_equal(ours, torch_e4m3(v))
+
+
+def test_rne_known_codes():
+    # OCP e4m3fn: 1.0 = 0x38, 448 = 0x7E (largest finite), 2^-6 = 0x08 (smallest normal),
+    # 2^-9 = 0x01 (smallest subnormal), 1.125 = 0x39; ties go to the even code
+    assert oracle.e4m3_rne(1.0) == 0x38
+    assert oracle.e4m3_rne(448.0) == 0x7E and oracle.e4m3_rne(1e9) == 0x7E and oracle.e4m3_rne(-1e9) == 0xFE
+    assert oracle.e4m3_rne(2.0 ** -6) == 0x08 and oracle.e4m3_rne(2.0 ** -9) == 0x01
+    assert oracle.e4m3_rne(1.125) == 0x39
+    assert oracle.e4m3_rne(1.0625) == 0x38            # halfway 1.0 / 1.125 -> even code 0x38
+    assert oracle.e4m3_rne(1.1875) == 0x3A            # halfway 1.125 / 1.25 -> even code 0x3A
+    assert oracle.e4m3_rne(2.0 ** -10) == 0x00        # halfway 0 / 2^-9 -> 0
+    assert oracle.e4m3_rne(-2.0 ** -12) == 0x80       # underflow keeps the sign
+
+
+def _bits(x: torch.Tensor) -> np.ndarray:
+    return bf16_bits(x.to(torch.bfloat16))
+
+
+def test_plain_quantiser_matches_the_torch_harness():
+    # without normalisation the definition is the harness's (independent torch code)
+    g = torch.Generator().manual_seed(6)
+    x = (torch.randn(2, 3, 100, 128, generator=g) * 2.5).to(torch.bfloat16)
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=False)
+    ref_codes, ref_ds = quantize_e4m3_per_head(x)
+    assert np.array_equal(ds, ref_ds.numpy())
+    assert np.array_equal(codes, ref_codes.view(torch.uint8).numpy())
+
+
+def test_single_nonzero_element_takes_the_largest_code():
+    x = torch.zeros(1, 2, 7, 128)
+    x[0, 0, 3, 17] = -3.5
+    x[0, 1, 6, 127] = 0.25
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=False)
+    assert ds[0, 0] == np.float32(3.5) / np.float32(448) and ds[0, 1] == np.float32(0.25) / np.float32(448)
+    assert codes[0, 0, 3, 17] == 0xFE and codes[0, 1, 6, 127] == 0x7E
+    mask = np.ones(codes.shape, bool)
+    mask[0, 0, 3, 17] = mask[0, 1, 6, 127] = False
+    assert np.all(codes[mask] == 0)
+
+
+def test_all_zero_head_has_unit_descale():
+    x = torch.zeros(1, 1, 5, 128)
+    for rms in (False, True):
+        codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=rms)
+        assert ds[0, 0] == 1.0 and np.all(codes == 0)
+
+
+def test_rmsnorm_closed_form_one_spike_per_row():
+    # a row whose only nonzero value is a has y = a / sqrt(a^2 / 128 + eps) there
+    a_vals = [0.5, -1.0, 2.0, 3.0, -0.75, 1.5]
+    x = torch.zeros(1, 1, len(a_vals), 128)
+    for i, a in enumerate(a_vals):
+        x[0, 0, i, (7 * i) % 128] = a
+    eps = 1e-6
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=eps)
+    y = [np.float32(a / math.sqrt(a * a / 128 + eps)) for a in a_vals]
+    amax = max(abs(v) for v in y)
+    assert ds[0, 0] == np.float32(amax) / np.float32(448)
+    for i, v in enumerate(y):
+        assert codes[0, 0, i, (7 * i) % 128] == oracle.e4m3_rne(np.float32(v) / ds[0, 0])
+
+
+def test_rmsnorm_closed_form_constant_rows():
+    # a constant row a has y = a / sqrt(a^2 + eps) everywhere: all of a head's
+    # rows with the same |a| take the largest code
+    x = torch.full((1, 2, 4, 128), 0.75)
+    x[0, 1] = -2.0
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=1e-6)
+    y0 = np.float32(0.75 / math.sqrt(0.75 ** 2 + 1e-6))
+    assert ds[0, 0] == y0 / np.float32(448)
+    assert np.all(codes[0, 0] == 0x7E) and np.all(codes[0, 1] == 0xFE)
+
+
+def test_rmsnorm_removes_power_of_two_scales_exactly():
+    # with eps = 0 the normalised values of 2^k x equal those of x bit for bit
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn(1, 2, 33, 128, generator=g).to(torch.bfloat16)
+    c0, d0 = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=0.0)
+    for k in (-3, 5):
+        c1, d1 = oracle.quantize_e4m3(_bits(x.float() * 2.0 ** k), rmsnorm=True, eps=0.0)
+        assert np.array_equal(c0, c1) and np.array_equal(d0, d1)
+
+
+def test_dequantised_error_within_half_a_code_step():
+    g = torch.Generator().manual_seed(8)
+    x = torch.randn(1, 1, 64, 128, generator=g).to(torch.bfloat16)
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=False)
+    y = x.float().numpy()[0, 0]
+    q = y / ds[0, 0]
+    deq = np.vectorize(oracle.e4m3_to_double)(codes[0, 0]).astype(np.float64)
+    # code step at |q|: 2^(floor(log2|q|) - 3) in the normal range, 2^-9 below 2^-6
+    e = np.floor(np.log2(np.maximum(np.abs(q), 2.0 ** -6)))
+    step = np.exp2(e - 3)
+    assert np.all(np.abs(deq - q) <= step / 2 + 1e-12)
