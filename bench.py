@@ -12,7 +12,8 @@ that is already resident in HBM:
              text keys, B=1 H=40 Sq=1560;
   cross      attn_fwd, B=1 H=40 Sq=90000 Sk=512 (long-query cross-attention);
   window     attn_fwd, B=1 H=12 Sq=4680 Sk=51480 (window / sink KV).
-The other workloads are measured too (``sub``) unless --no-sub.
+The other workloads are measured too (``sub``) unless --no-sub, plus the e4m3
+prologue (quantize_e4m3 of the fp8 config's Q, K, V; HBM-bound, in GB/s).
 
 Timing: W untimed warm-up steps; then K steps, each preceded (outside its
 CUDA events) by a 256 MB write that flushes L2, bracketed by a barrier and a
@@ -54,7 +55,8 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "llm_gqa": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16)",
                   "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)",
                   "cross": "long-query cross-attention fwd (B1 H40 Sq90000 Sk512 D128 bf16)",
-                  "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)"}
+                  "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)",
+                  "fp8_prep": "e4m3 prologue of the fp8 config (Q, K RMS-normalised; V plain; per-head descales)"}
 FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window")
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
@@ -191,7 +193,7 @@ class Step:
     def __init__(self, name, h, heads=None, rank=0):
         self.name = name
         self.h = h
-        self.w = workloads.get(name)
+        self.w = workloads.get("fp8" if name == "fp8_prep" else name)
         if heads:
             self.w = workloads.get(name, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
         if rank:
@@ -222,6 +224,17 @@ class Step:
             self.flops = w.fwd_flops() + w.bwd_flops()
             self.launches = 4
             self.dtype = "bf16"
+        elif name == "fp8_prep":
+            # the step before the fp8 forward: bf16 Q, K, V of the fp8 shape -> e4m3 + descales
+            g = torch.Generator().manual_seed(w.seed)
+            self.src = [torch.randn(w.B, H, S, w.D, generator=g).to(torch.bfloat16).cuda()
+                        for H, S in ((w.Hq, w.Sq), (w.Hkv, w.Sk), (w.Hkv, w.Sk))]
+            self.dst = [(torch.empty(t.shape, dtype=torch.float8_e4m3fn, device="cuda"),
+                         torch.empty(t.shape[:2], dtype=torch.float32, device="cuda")) for t in self.src]
+            self.flops = 0.0
+            self.bytes = sum(5.0 * t.numel() for t in self.src)   # x read twice, codes written once
+            self.launches = 12                                      # 3 x (memset + 3 kernels)
+            self.dtype = "e4m3"
         elif name == "streaming":
             x = make_kvblock_inputs(w)
             self.host = x
@@ -249,6 +262,9 @@ class Step:
             if self.name == "fp8":
                 ds = dict(q_descale=x["q_descale"], k_descale=x["k_descale"], v_descale=x["v_descale"])
             h.attn_fwd(x["q"], x["k"], x["v"], out=self.out, lse=self.lse, **ds)
+        elif self.name == "fp8_prep":
+            for i, (t, (c, d)) in enumerate(zip(self.src, self.dst)):
+                h.quantize_e4m3(t, rmsnorm=i < 2, codes=c, descale=d)
         elif self.name == "llm_gqa":
             x = self.x
             h.attn_fwd(x["q"], x["k"], x["v"], causal=True, out=self.out, lse=self.lse)
@@ -391,7 +407,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOAD_NAMES), default="video")
+    ap.add_argument("--workload", choices=[n for n in WORKLOAD_NAMES if n != "fp8_prep"], default="video")
     ap.add_argument("--no-sub", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
@@ -462,11 +478,17 @@ def main(argv=None):
             if h.get_device_error() != 0:
                 raise RuntimeError("a kernel reported a bounded-wait timeout")
             t = statistics.mean(oms)
-            pk = peaks["bf16_tflops"] * (2.0 if st.dtype == "e4m3" else 1.0)
-            sub[other] = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t,
-                          "tflops": st.flops / (t * 1e-3) / 1e12,
-                          "frac_of_peak": st.flops / (t * 1e-3) / 1e12 / pk, "peak_tflops": pk,
-                          "dtype": st.dtype, "launches_per_step": st.launches}
+            if other == "fp8_prep":
+                gbs = st.bytes / (t * 1e-3) / 1e9
+                sub[other] = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t, "gbs": gbs,
+                              "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
+                              "bytes_per_step": st.bytes, "dtype": st.dtype, "launches_per_step": st.launches}
+            else:
+                pk = peaks["bf16_tflops"] * (2.0 if st.dtype == "e4m3" else 1.0)
+                sub[other] = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t,
+                              "tflops": st.flops / (t * 1e-3) / 1e12,
+                              "frac_of_peak": st.flops / (t * 1e-3) / 1e12 / pk, "peak_tflops": pk,
+                              "dtype": st.dtype, "launches_per_step": st.launches}
             del st
             torch.cuda.empty_cache()
         line["sub"] = sub

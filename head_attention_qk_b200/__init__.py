@@ -9,7 +9,7 @@ ImportError (there is no fallback).
 """
 _API = ("BF16", "E4M3", "EXPORTED", "NOALLOC_MAX_ROWS", "HattnError", "attn_bwd", "attn_bwd_noalloc", "attn_fwd",
         "attn_fwd_kvblocks", "bwd_workspace_size", "fwd_workspace_size", "get_device_error", "kvblocks_workspace_size",
-        "lib")
+        "lib", "quantize_e4m3")
 
 
 def __getattr__(name):

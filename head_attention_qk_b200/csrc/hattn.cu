@@ -18,6 +18,7 @@
 #include "../../include/hattn.h"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "prep_kernel.cuh"
 
 namespace hattn {
 
@@ -294,6 +295,27 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                      v16, st);
   if (cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_EDEVICE;
   return rc;
+}
+
+int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H, int S, int D, int rmsnorm,
+                       double eps, void* stream) {
+  if (!x || !codes || !descale) return HATTN_EINVAL;
+  if (B <= 0 || H <= 0 || S <= 0 || D <= 0) return HATTN_EINVAL;
+  if (rmsnorm && !(eps > 0.0 && eps < 1e300)) return HATTN_EINVAL;
+  if (D != kPrepD) return HATTN_EUNSUPPORTED;
+  if ((long long)B * H > 65535 || !sizes_fit(B, H, S)) return HATTN_EUNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(descale) & 3u)) return HATTN_EALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int bh = B * H;
+  const dim3 grid((S + kPrepThreads - 1) / kPrepThreads, bh);
+  if (cudaMemsetAsync(descale, 0, (size_t)bh * sizeof(float), st) != cudaSuccess) return HATTN_ELAUNCH;
+  prep_amax_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
+                                                   reinterpret_cast<unsigned int*>(descale), S, rmsnorm ? 1 : 0, eps);
+  prep_descale_kernel<<<(bh + 255) / 256, 256, 0, st>>>(descale, bh);
+  prep_quantize_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
+                                                       reinterpret_cast<uint8_t*>(codes), descale, S,
+                                                       rmsnorm ? 1 : 0, eps);
+  return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
 size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks) {

@@ -42,13 +42,15 @@ lib.attn_bwd_workspace_size.argtypes = [_i, _i, _i]
 lib.attn_bwd_workspace_size.restype = _sz
 lib.attn_get_device_error.argtypes = [_vp, ctypes.POINTER(_i)]
 lib.attn_get_device_error.restype = _i
+lib.attn_quantize_e4m3.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_double, _vp]
+lib.attn_quantize_e4m3.restype = _i
 lib.attn_selftest_bounded_wait.argtypes = [_vp, ctypes.c_uint]
 lib.attn_selftest_bounded_wait.restype = _i
 lib.attn_error_string.argtypes = [_i]
 lib.attn_error_string.restype = ctypes.c_char_p
 
 BF16, E4M3 = 0, 1
-EXPORTED = ("attn_fwd", "attn_fwd_ws", "attn_fwd_workspace_size", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
+EXPORTED = ("attn_fwd", "attn_fwd_ws", "attn_fwd_workspace_size", "attn_quantize_e4m3", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
             "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_error", "attn_selftest_bounded_wait",
             "attn_error_string")
 NOALLOC_MAX_ROWS = 1 << 22
@@ -123,6 +125,23 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
                          _stream(stream))
     _check(rc, "attn_fwd")
     return out, lse
+
+
+def quantize_e4m3(x, rmsnorm=False, eps=1e-6, codes=None, descale=None, stream=None):
+    """bf16 x [B,H,S,D] -> (e4m3fn codes [B,H,S,D], fp32 descale [B,H]) with an
+    optional per-row RMS normalisation first (see attn_quantize_e4m3 in hattn.h)."""
+    _require(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 4:
+        raise TypeError("quantize_e4m3 takes a [B,H,S,D] bfloat16 tensor")
+    B, H, S, D = x.shape
+    if codes is None:
+        codes = torch.empty((B, H, S, D), dtype=torch.float8_e4m3fn, device=x.device)
+    if descale is None:
+        descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    rc = lib.attn_quantize_e4m3(_ptr(x), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)), float(eps),
+                                _stream(stream))
+    _check(rc, "attn_quantize_e4m3")
+    return codes, descale
 
 
 def kvblocks_workspace_size(B, Hq, Sq, D, n_blocks) -> int:

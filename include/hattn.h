@@ -99,6 +99,26 @@ HATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* out
 HATTN_API size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtype);
 
 /*
+ * e4m3 quantisation prologue for the fp8 forward (FlashDreams PR #486 section
+ * 1.1 Quantization toolkit: FP8 E4M3 with per-slice scales, and section 1.2:
+ * head-scoped Q/K normalisation; e4m3fn range +-448 as in VeOmni PR #1363).
+ *   x       [B, H, S, D] bf16 in (D must be 128)
+ *   codes   [B, H, S, D] e4m3fn codes out
+ *   descale [B*H] fp32 out: the real value of code c of head (b, h) is
+ *           decode(c) * descale[b*H + h], ready for attn_fwd's descales.
+ * Per head: with rmsnorm != 0 each row is first divided by
+ * sqrt(mean over d of x_d^2 + eps) (eps > 0; the squares summed in fp64 in
+ * ascending d, the factor 1/sqrt(.) in fp64 and the product rounded to fp32),
+ * giving y; without it y = x.  descale = max |y| / 448 (fp32; 1 if the head is
+ * all zero), code = y / descale (fp32 quotient) rounded to the nearest e4m3fn
+ * value, ties to even, saturating at +-448.  The result is bitwise the same for
+ * any batch or head split.  Enqueues a memset of descale and three kernels;
+ * HBM traffic 5 bytes per element (x read twice, codes written once).
+ */
+HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H, int S, int D,
+                                 int rmsnorm, double eps, void* stream);
+
+/*
  * Streaming forward over a block KV cache (FlashDreams PR #486 section 1.2;
  * merge rule from RL-Kernel PR #319 Summary table).  Queries attend, without a
  * mask, to the concatenation of n_blocks caller-managed KV blocks.  Each block

@@ -85,6 +85,16 @@ def test_fwd_workspace_size_and_checks(h):
     assert call(ws=MIS) == -3
 
 
+def test_quantize_fails_closed(h):
+    def call(x=A, codes=B_, ds=A, B=1, H=2, S=64, D=128, rms=1, eps=1e-6):
+        return h.lib.attn_quantize_e4m3(x, codes, ds, B, H, S, D, rms, eps, None)
+
+    assert call(x=None) == -1 and call(ds=None) == -1 and call(S=0) == -1
+    assert call(eps=0.0) == -1 and call(eps=-1.0) == -1     # rmsnorm needs eps > 0
+    assert call(D=64) == -2
+    assert call(x=MIS) == -3 and call(codes=MIS) == -3
+
+
 def test_kvblocks_fails_closed(h):
     lib = h.lib
     kp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
