@@ -193,12 +193,13 @@ class Step:
     def __init__(self, name, h, heads=None, rank=0):
         self.name = name
         self.h = h
-        self.w = workloads.get("fp8" if name == "fp8_prep" else name)
+        base = "fp8" if name == "fp8_prep" else name
+        self.w = workloads.get(base)
         if heads:
-            self.w = workloads.get(name, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
+            self.w = workloads.get(base, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
         if rank:
             # weak scaling: each rank attends over its own units (its own seeded draws)
-            self.w = workloads.get(name, seed=self.w.seed + 7919 * rank, Hq=self.w.Hq, Hkv=self.w.Hkv)
+            self.w = workloads.get(base, seed=self.w.seed + 7919 * rank, Hq=self.w.Hq, Hkv=self.w.Hkv)
         w = self.w
         self.launches = 1
         if name in FWD_WORKLOADS:
@@ -401,6 +402,28 @@ def run_reference(args, world, rank):
     return 0
 
 
+def sub_result(other, h, flush, steps, warmup, peaks, heads=None):
+    """Time one workload on this GPU; its entry of the JSON line's ``sub``."""
+    st = Step(other, h, heads=heads)
+    oms, _ = time_steps(st, steps, warmup, 1, flush)
+    if h.get_device_error() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout")
+    t = statistics.mean(oms)
+    if other == "fp8_prep":
+        gbs = st.bytes / (t * 1e-3) / 1e9
+        r = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t, "gbs": gbs,
+             "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
+             "bytes_per_step": st.bytes, "dtype": st.dtype, "launches_per_step": st.launches}
+    else:
+        pk = peaks["bf16_tflops"] * (2.0 if st.dtype == "e4m3" else 1.0)
+        r = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t, "tflops": st.flops / (t * 1e-3) / 1e12,
+             "frac_of_peak": st.flops / (t * 1e-3) / 1e12 / pk, "peak_tflops": pk,
+             "dtype": st.dtype, "launches_per_step": st.launches}
+    del st
+    torch.cuda.empty_cache()
+    return r
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -412,6 +435,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="smaller case: override the query head count")
+    ap.add_argument("--only", choices=list(WORKLOAD_NAMES), default=None,
+                    help="time just this workload (one GPU) and print its sub-result line; for profiling")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -426,6 +451,10 @@ def main(argv=None):
     peaks, peak_src = load_peaks()
     torch.cuda.set_device(local)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    if args.only:
+        print(json.dumps({"only": args.only, **sub_result(args.only, h, flush, args.steps, args.warmup, peaks,
+                                                           heads=args.heads or None)}))
+        return 0
     name = args.workload
     step = Step(name, h, heads=args.heads or None, rank=rank)
     ms, clocks = time_steps(step, args.steps, args.warmup, world, flush,
@@ -473,24 +502,7 @@ def main(argv=None):
         for other in WORKLOAD_NAMES:
             if other == name or other == "tiny":
                 continue
-            st = Step(other, h)
-            oms, _ = time_steps(st, max(3, args.steps // 2), args.warmup, 1, flush)
-            if h.get_device_error() != 0:
-                raise RuntimeError("a kernel reported a bounded-wait timeout")
-            t = statistics.mean(oms)
-            if other == "fp8_prep":
-                gbs = st.bytes / (t * 1e-3) / 1e9
-                sub[other] = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t, "gbs": gbs,
-                              "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
-                              "bytes_per_step": st.bytes, "dtype": st.dtype, "launches_per_step": st.launches}
-            else:
-                pk = peaks["bf16_tflops"] * (2.0 if st.dtype == "e4m3" else 1.0)
-                sub[other] = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t,
-                              "tflops": st.flops / (t * 1e-3) / 1e12,
-                              "frac_of_peak": st.flops / (t * 1e-3) / 1e12 / pk, "peak_tflops": pk,
-                              "dtype": st.dtype, "launches_per_step": st.launches}
-            del st
-            torch.cuda.empty_cache()
+            sub[other] = sub_result(other, h, flush, max(3, args.steps // 2), args.warmup, peaks)
         line["sub"] = sub
 
     if rank == 0 and world == 1 and not args.no_cpu:

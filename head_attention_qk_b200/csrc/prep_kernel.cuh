@@ -26,29 +26,30 @@ namespace hattn {
 constexpr int kPrepD = 128;
 constexpr int kPrepThreads = 256;   // one row per thread
 
-// Per-row normalisation factor (1 without rmsnorm) and the row's 128 bf16 values
-// as 16 x 16-byte words.
-__device__ __forceinline__ double prep_row_factor(const uint4 (&w)[16], int rmsnorm, double eps) {
+// Per-row normalisation factor (1 without rmsnorm): squares summed in fp64 in
+// ascending d (each square is exact in fp64).  The row is streamed in 64-byte
+// pieces, so few registers stay live; the second pass over the row (y) hits L1.
+__device__ __forceinline__ double prep_row_factor(const uint4* __restrict__ row, int rmsnorm, double eps) {
   if (!rmsnorm) return 1.0;
   double sum = 0.0;
+#pragma unroll 2
+  for (int i = 0; i < 16; i += 4) {
+    uint4 w[4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t p[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+    for (int k = 0; k < 4; ++k) w[k] = __ldg(&row[i + k]);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const double lo = (double)__uint_as_float(p[k] << 16);
-      const double hi = (double)__uint_as_float(p[k] & 0xFFFF0000u);
-      sum += lo * lo;      // each square is exact in fp64; the adds run in d order
-      sum += hi * hi;
+      const uint32_t p[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const double lo = (double)__uint_as_float(p[t] << 16);
+        const double hi = (double)__uint_as_float(p[t] & 0xFFFF0000u);
+        sum += lo * lo;
+        sum += hi * hi;
+      }
     }
   }
   return 1.0 / sqrt(sum / (double)kPrepD + eps);
-}
-
-__device__ __forceinline__ void prep_load_row(const uint16_t* x, long long row, uint4 (&w)[16]) {
-  const uint4* src = reinterpret_cast<const uint4*>(x + row * kPrepD);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = __ldg(&src[i]);
 }
 
 __device__ __forceinline__ float prep_y(uint32_t bits16_as_f32, double r, int rmsnorm) {
@@ -57,19 +58,19 @@ __device__ __forceinline__ float prep_y(uint32_t bits16_as_f32, double r, int rm
 }
 
 // grid (ceil(S / 256), B*H): the largest |y| of each head into amax_bits (zeroed).
-__global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
-                                                                   unsigned int* __restrict__ amax_bits, int S,
-                                                                   int rmsnorm, double eps) {
+__global__ void __launch_bounds__(kPrepThreads, 4) prep_amax_kernel(const uint16_t* __restrict__ x,
+                                                                      unsigned int* __restrict__ amax_bits, int S,
+                                                                      int rmsnorm, double eps) {
   const int bh = blockIdx.y;
   const int s = blockIdx.x * kPrepThreads + threadIdx.x;
   float m = 0.f;
   if (s < S) {
-    uint4 w[16];
-    prep_load_row(x, (long long)bh * S + s, w);
-    const double r = prep_row_factor(w, rmsnorm, eps);
-#pragma unroll
+    const uint4* row = reinterpret_cast<const uint4*>(x) + ((long long)bh * S + s) * 16;
+    const double r = prep_row_factor(row, rmsnorm, eps);
+#pragma unroll 4
     for (int i = 0; i < 16; ++i) {
-      const uint32_t p[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+      const uint4 w = __ldg(&row[i]);
+      const uint32_t p[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         m = fmaxf(m, fabsf(prep_y(p[k] << 16, r, rmsnorm)));
@@ -99,6 +100,19 @@ __global__ void prep_descale_kernel(float* __restrict__ d, int n) {
   }
 }
 
+// y / ds rounded to fp32.  Fast path: y times a reciprocal, within 2 ulp of
+// the quotient; that can only change the e4m3 rounding when the result lies
+// within a few ulp of a midpoint between two e4m3 values (its low 20 mantissa
+// bits near 0x80000) or in the small range where e4m3 steps are subnormal, and
+// there the exactly rounded quotient is taken instead.
+__device__ __forceinline__ float prep_quotient(float y, float ds, float rcp) {
+  const float q = y * rcp;
+  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
+  const int low = (int)(b & 0xFFFFFu) - 0x80000;
+  if (b < 0x3D000000u /* 2^-5 */ || (low >= -4 && low <= 4)) return __fdiv_rn(y, ds);
+  return q;
+}
+
 __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
@@ -106,30 +120,31 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
 }
 
 // grid (ceil(S / 256), B*H): the codes of each row.
-__global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
-                                                                       uint8_t* __restrict__ codes,
-                                                                       const float* __restrict__ descale, int S,
-                                                                       int rmsnorm, double eps) {
+__global__ void __launch_bounds__(kPrepThreads, 4) prep_quantize_kernel(const uint16_t* __restrict__ x,
+                                                                          uint8_t* __restrict__ codes,
+                                                                          const float* __restrict__ descale, int S,
+                                                                          int rmsnorm, double eps) {
   const int bh = blockIdx.y;
   const int s = blockIdx.x * kPrepThreads + threadIdx.x;
   if (s >= S) return;
-  const long long row = (long long)bh * S + s;
-  uint4 w[16];
-  prep_load_row(x, row, w);
-  const double r = prep_row_factor(w, rmsnorm, eps);
+  const long long rowi = (long long)bh * S + s;
+  const uint4* row = reinterpret_cast<const uint4*>(x) + rowi * 16;
+  const double r = prep_row_factor(row, rmsnorm, eps);
   const float ds = __ldg(&descale[bh]);
-  uint4* dst = reinterpret_cast<uint4*>(codes + row * kPrepD);
-#pragma unroll
+  const float rcp = __frcp_rn(ds);
+  uint4* dst = reinterpret_cast<uint4*>(codes) + rowi * 8;
+#pragma unroll 2
   for (int i = 0; i < 16; i += 2) {
     uint32_t o[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t p[4] = {w[i + h].x, w[i + h].y, w[i + h].z, w[i + h].w};
+      const uint4 w = __ldg(&row[i + h]);
+      const uint32_t p[4] = {w.x, w.y, w.z, w.w};
       uint16_t c[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        c[k] = e4m3x2_rn_satfinite(__fdiv_rn(prep_y(p[k] << 16, r, rmsnorm), ds),
-                                   __fdiv_rn(prep_y(p[k] & 0xFFFF0000u, r, rmsnorm), ds));
+        c[k] = e4m3x2_rn_satfinite(prep_quotient(prep_y(p[k] << 16, r, rmsnorm), ds, rcp),
+                                   prep_quotient(prep_y(p[k] & 0xFFFF0000u, r, rmsnorm), ds, rcp));
       o[2 * h] = (uint32_t)c[0] | ((uint32_t)c[1] << 16);
       o[2 * h + 1] = (uint32_t)c[2] | ((uint32_t)c[3] << 16);
     }
