@@ -90,7 +90,9 @@ struct FwdArgs {
   const float* k_descale;
   const float* v_descale;
   int block_offset;              // index of this launch's first block among all blocks
-  int total_units;               // n_qpairs * B * Hq * (blocks in this launch); CTAs loop over them
+  int total_units;               // work units of this launch; CTAs loop over them
+  int fused_blocks;              // > 1: one unit runs over all these blocks in order (no partials)
+  int fused_tiles;               // KV tiles over all fused blocks
 };
 
 template <bool kFp8>
@@ -137,10 +139,14 @@ __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int 
   return max_key / kBlockN + 1;
 }
 
-// One work unit: 256 query rows of one (b, h) against one KV block.
+// One work unit: 256 query rows of one (b, h) against one KV block, or against
+// all the launch's blocks in ascending order when they are fused.
 struct FwdUnit {
   int bh, kvh, q_row0, blk, sk, n_kv;
 };
+
+// KV tiles of a block of sk keys.
+__device__ __forceinline__ int fwd_block_tiles(int sk) { return (sk + kBlockN - 1) / kBlockN; }
 
 // Units are numbered block-major.  Without a mask, consecutive units share a
 // head (its K/V stays hot in L2); under a causal mask the order is rank-major
@@ -150,7 +156,7 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdArgs& a, int u) {
   FwdUnit w;
   const int nbh = a.B * a.Hq;
   const int per_blk = a.n_qpairs * nbh;
-  w.blk = u / per_blk;
+  w.blk = a.fused_blocks > 1 ? 0 : u / per_blk;
   const int r = u - w.blk * per_blk;
   int qpair;
   if (a.causal) {
@@ -165,7 +171,7 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdArgs& a, int u) {
   w.kvh = b * a.Hkv + h / (a.Hq / a.Hkv);
   w.q_row0 = qpair * (kQTilesPerCta * kBlockM);
   w.sk = a.sk[w.blk];
-  w.n_kv = fwd_num_kv_tiles(w.sk, a.Sq, a.causal, w.q_row0);
+  w.n_kv = a.fused_blocks > 1 ? a.fused_tiles : fwd_num_kv_tiles(w.sk, a.Sq, a.causal, w.q_row0);
   return w;
 }
 
@@ -253,8 +259,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       long long nseq = 0;                                  // K/V tiles loaded by this CTA
       for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
         const FwdUnit w = fwd_unit(args, u);
-        const CUtensorMap* tk = &args.tm_k[w.blk];
-        const CUtensorMap* tv = &args.tm_v[w.blk];
+        // K/V tile j of the unit: tile lt of block b (fused blocks run in order)
+        int b = w.blk, lt = 0, nt = fwd_block_tiles(args.sk[b]);
         // the previous unit's last S has been issued before Q is overwritten
         if (units > 0) ok = mbar_wait(bb.q_empty, (units - 1) & 1, kSiteQFull);
         if (!ok) break;
@@ -271,11 +277,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           if (n & 1) {
             mbar_arrive_expect_tx(&bb.ring_full[slot], L::kVTileBytes);
             for (int x = 0; x < 2; ++x)
-              tma_load_3d(dst + x * kVBoxBytes, tv, &bb.ring_full[slot], x * 64, (n >> 1) * kBlockN, w.kvh);
+              tma_load_3d(dst + x * kVBoxBytes, &args.tm_v[b], &bb.ring_full[slot], x * 64, lt * kBlockN, w.kvh);
+            if (++lt == nt && n + 1 < 2 * w.n_kv) {         // next block
+              ++b;
+              lt = 0;
+              nt = fwd_block_tiles(args.sk[b]);
+            }
           } else {
             mbar_arrive_expect_tx(&bb.ring_full[slot], L::kTileBytes);
             for (int x = 0; x < kBoxes; ++x)
-              tma_load_3d(dst + x * kBoxBytes, tk, &bb.ring_full[slot], x * kBoxCols, (n >> 1) * kBlockN, w.kvh);
+              tma_load_3d(dst + x * kBoxBytes, &args.tm_k[b], &bb.ring_full[slot], x * kBoxCols, lt * kBlockN,
+                          w.kvh);
           }
           if (++slot == L::kRing) { slot = 0; ph ^= 1u; }
         }
@@ -420,7 +432,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
       float m = -INFINITY;     // running max of x = s * c (base-2 units)
       float l = 0.f;           // running sum of 2^(x - m)
+      const bool fused = args.fused_blocks > 1;
+      int fb = 0, flt = 0, fsk = args.sk[0], fnt = fwd_block_tiles(fsk);   // fused: block / tile walk
       for (int j = 0; j < n_kv; ++j, ++jg) {
+        // last unmasked key column of this tile (>= 127: none masked)
+        int lim;
+        if (fused) {
+          lim = fsk - flt * kBlockN - 1;
+          if (++flt == fnt && j + 1 < n_kv) {
+            ++fb;
+            flt = 0;
+            fsk = args.sk[fb];
+            fnt = fwd_block_tiles(fsk);
+          }
+        } else {
+          lim = kv_limit - j * kBlockN;
+        }
         ok = warp_wait(&bb.s_full[tile], jg & 1, kSiteSFull);
         if (!ok) break;
         tc_fence_after();
@@ -433,12 +460,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 #pragma unroll
           for (int e = 0; e < 128; ++e) s[e] = __uint_as_float(uu[e]);
         }
-        const int kbase = j * kBlockN;
-        const bool masked = kbase + kBlockN - 1 > kv_limit;
+        const bool masked = lim < kBlockN - 1;
         if (masked) {
 #pragma unroll
           for (int e = 0; e < 128; ++e)
-            if (kbase + e > kv_limit) s[e] = -INFINITY;
+            if (e > lim) s[e] = -INFINITY;
         }
         // row max: eight independent three-input chains
         float mx[8];
@@ -490,8 +516,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
               // fp16 P (fp8 path) tolerates the quadratic, bf16 P takes the cubic
               p = exp2_poly2<kFp8 ? 2 : 3>(x);
               if (masked) {                               // the polynomial is never exactly 0
-                p.x = kbase + e > kv_limit ? 0.f : p.x;
-                p.y = kbase + e + 1 > kv_limit ? 0.f : p.y;
+                p.x = e > lim ? 0.f : p.x;
+                p.y = e + 1 > lim ? 0.f : p.y;
               }
             } else {
               p = make_float2(ex2_approx(x.x), ex2_approx(x.y));

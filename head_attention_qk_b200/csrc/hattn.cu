@@ -320,6 +320,7 @@ int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H,
 
 size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks) {
   if (B <= 0 || Hq <= 0 || Sq <= 0 || D <= 0 || n_blocks <= 0) return 0;
+  if (n_blocks <= kMaxKvBlocks) return 0;   // one launch folds the blocks in order: no partials
   return (size_t)n_blocks * (size_t)B * Hq * Sq * ((size_t)D + 1) * sizeof(float);
 }
 
@@ -327,7 +328,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
                       int n_blocks, void* out, float* lse, int B, int Hq, int Hkv, int Sq, int D, float scale,
                       int dtype, const float* q_descale, const float* k_descale, const float* v_descale,
                       void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k_blocks || !v_blocks || !blk_len || !out || !lse || !workspace) return HATTN_EINVAL;
+  if (!q || !k_blocks || !v_blocks || !blk_len || !out || !lse) return HATTN_EINVAL;
   if (n_blocks <= 0) return HATTN_EINVAL;
   int rc = check_common(B, Hq, Hkv, Sq, D, scale);
   if (rc) return rc;
@@ -340,15 +341,41 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     if (!sizes_fit(B, Hkv, blk_len[i])) return HATTN_EUNSUPPORTED;
     if (!aligned16(k_blocks[i]) || !aligned16(v_blocks[i])) return HATTN_EALIGN;
   }
-  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(workspace)) return HATTN_EALIGN;
-  if (workspace_bytes < attn_fwd_kvblocks_workspace_size(B, Hq, Sq, D, n_blocks)) return HATTN_EWORKSPACE;
+  const size_t need = attn_fwd_kvblocks_workspace_size(B, Hq, Sq, D, n_blocks);
+  if (need && !workspace) return HATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (need && !aligned16(workspace))) return HATTN_EALIGN;
+  if (workspace_bytes < need) return HATTN_EWORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  static thread_local FwdArgs a;
+
+  if (n_blocks <= kMaxKvBlocks) {
+    // One unit per (256 query rows, b, h) runs over all blocks in ascending
+    // order: its online softmax folds block after block, so no per-block
+    // partials are written and no merge pass is needed.
+    memset(&a, 0, sizeof(a));
+    if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    int tiles = 0;
+    for (int i = 0; i < n_blocks; ++i) {
+      if (!encode_rows(&a.tm_k[i], k_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+      if (!encode_rows(&a.tm_v[i], v_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+      a.sk[i] = blk_len[i];
+      tiles += (blk_len[i] + kBlockN - 1) / kBlockN;
+    }
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Sq = Sq;
+    a.causal = 0;
+    a.n_qpairs = (Sq + kQTilesPerCta * kBlockM - 1) / (kQTilesPerCta * kBlockM);
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.out = out;
+    a.lse = lse;
+    a.fused_blocks = n_blocks;
+    a.fused_tiles = tiles;
+    if (n_blocks == 1) a.fused_blocks = 0;   // a single block is a plain forward
+    return launch_fwd<false, false>(a, 1, tiles * kBlockN, st);
+  }
 
   const long long rows = (long long)B * Hq * Sq;
   float* o_parts = reinterpret_cast<float*>(workspace);
   float* lse_parts = o_parts + (size_t)n_blocks * rows * kHeadDim;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-
-  static thread_local FwdArgs a;
   for (int first = 0; first < n_blocks; first += kMaxKvBlocks) {
     const int cnt = n_blocks - first < kMaxKvBlocks ? n_blocks - first : kMaxKvBlocks;
     memset(&a, 0, sizeof(a));

@@ -163,7 +163,7 @@ def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=Non
     vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in v_blocks])
     lens = (ctypes.c_int * n)(*[int(t.shape[2]) for t in k_blocks])
     ws_bytes = kvblocks_workspace_size(B, Hq, Sq, D, n)
-    if workspace is None:
+    if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
@@ -172,7 +172,8 @@ def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=Non
     rc = lib.attn_fwd_kvblocks(_ptr(q), ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
                                ctypes.cast(lens, ctypes.c_void_p), n, _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, D,
                                scale, _dtype_code(q), None, None, None, _ptr(workspace),
-                               workspace.numel() * workspace.element_size(), _stream(stream))
+                               0 if workspace is None else workspace.numel() * workspace.element_size(),
+                               _stream(stream))
     _check(rc, "attn_fwd_kvblocks")
     return out, lse
 

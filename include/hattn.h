@@ -121,9 +121,12 @@ HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int
 /*
  * Streaming forward over a block KV cache (FlashDreams PR #486 section 1.2;
  * merge rule from RL-Kernel PR #319 Summary table).  Queries attend, without a
- * mask, to the concatenation of n_blocks caller-managed KV blocks.  Each block
- * is computed separately into the workspace as (O_b, LSE_b), then the blocks
- * are folded in ascending order:
+ * mask, to the concatenation of n_blocks caller-managed KV blocks, folded in
+ * ascending block order.  Up to 32 blocks are folded inside one launch: each
+ * unit of 256 query rows runs its online softmax over block 0, then block 1,
+ * and so on (no workspace: attn_fwd_kvblocks_workspace_size() returns 0).
+ * With more blocks, each is computed separately into the workspace as
+ * (O_b, LSE_b), then the blocks are folded in ascending order:
  *     M = max(L, L_b); w = e^(L - M); w_b = e^(L_b - M);
  *     L = M + ln(w + w_b); O = (w O + w_b O_b) / (w + w_b),  from (O, L) = (0, -inf).
  *   q          [B, Hq, Sq, D] bf16 (dtype must be HATTN_BF16 in this version)
@@ -131,8 +134,8 @@ HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int
  *              [B, Hkv, blk_len[i], D] bf16
  *   blk_len    HOST array of n_blocks lengths, each > 0
  *   out, lse   as for attn_fwd
- *   workspace  device buffer of at least attn_fwd_kvblocks_workspace_size() bytes;
- *              its contents on entry do not matter.
+ *   workspace  device buffer of at least attn_fwd_kvblocks_workspace_size() bytes
+ *              (may be NULL when that is 0); its contents on entry do not matter.
  */
 HATTN_API int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* const* v_blocks,
                       const int* blk_len, int n_blocks, void* out, float* lse,

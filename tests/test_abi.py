@@ -39,7 +39,8 @@ def test_library_exports_every_declared_symbol(h):
 
 
 def test_workspace_sizes(h):
-    assert h.kvblocks_workspace_size(1, 40, 1560, 128, 21) == 21 * 40 * 1560 * 129 * 4
+    assert h.kvblocks_workspace_size(1, 40, 1560, 128, 21) == 0          # folded in one launch
+    assert h.kvblocks_workspace_size(1, 40, 1560, 128, 40) == 40 * 40 * 1560 * 129 * 4
     assert h.bwd_workspace_size(2, 32, 2048) == 2 * 32 * 2048 * 4
     assert h.kvblocks_workspace_size(0, 1, 1, 128, 1) == 0
 
@@ -97,22 +98,25 @@ def test_quantize_fails_closed(h):
 
 def test_kvblocks_fails_closed(h):
     lib = h.lib
-    kp = (ctypes.c_void_p * 2)(0x10000, 0x20000)
-    lens = (ctypes.c_int * 2)(100, 0)
-    need = h.kvblocks_workspace_size(1, 2, 64, 128, 2)
 
-    def call(lens=lens, n=2, ws=A, wsb=need, dtype=0, D=128, qd=None):
+    def call(lens, n, ws=A, wsb=0, dtype=0, D=128, qd=None):
+        kp = (ctypes.c_void_p * len(lens))(*([0x10000] * len(lens)))
+        ln = (ctypes.c_int * len(lens))(*lens)
         return lib.attn_fwd_kvblocks(A, ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(kp, ctypes.c_void_p),
-                                     ctypes.cast(lens, ctypes.c_void_p), n, A, A, 1, 2, 2, 64, D, 0.088, dtype,
+                                     ctypes.cast(ln, ctypes.c_void_p), n, A, A, 1, 2, 2, 64, D, 0.088, dtype,
                                      qd, qd, qd, ws, wsb, None)
 
-    assert call() == -2                                   # a zero-length block
-    ok_lens = (ctypes.c_int * 2)(100, 50)
-    assert call(lens=ok_lens, n=0) == -1
-    assert call(lens=ok_lens, wsb=need - 1) == -4          # workspace too small
-    assert call(lens=ok_lens, ws=MIS) == -3
-    assert call(lens=ok_lens, D=64) == -2
-    assert call(lens=ok_lens, dtype=1, qd=A) == -2         # fp8 block-KV not offered
+    assert call([100, 0], 2) == -2                       # a zero-length block
+    assert call([100, 50], 0) == -1
+    assert call([100, 50], 2, D=64) == -2
+    assert call([100, 50], 2, dtype=1, qd=A) == -2       # fp8 block-KV not offered
+    # more blocks than one launch folds: per-block partials need the workspace
+    many = [40 + i for i in range(33)]
+    need = h.kvblocks_workspace_size(1, 2, 64, 128, 33)
+    assert need > 0 and h.kvblocks_workspace_size(1, 2, 64, 128, 32) == 0
+    assert call(many, 33, wsb=need - 1) == -4            # workspace too small
+    assert call(many, 33, ws=MIS, wsb=need) == -3
+    assert call(many, 33, ws=None, wsb=need) == -1
 
 
 def test_bwd_fails_closed(h):
