@@ -52,7 +52,9 @@ struct BwdArgs {
   uint16_t* dv;
 };
 
-enum : int { kSiteBwdKV = 20, kSiteBwdStFull, kSiteBwdStEmpty, kSiteBwdS, kSiteBwdDP, kSiteBwdP, kSiteBwdDone };
+enum : int {
+  kSiteBwdKV = 20, kSiteBwdStFull, kSiteBwdStEmpty, kSiteBwdS, kSiteBwdDP, kSiteBwdP, kSiteBwdDone, kSiteBwdAlign
+};
 
 // ---------------------------------------------------------------------------- Delta
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
@@ -128,14 +130,23 @@ __device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, u
 
 // ---------------------------------------------------------------------------- dK / dV
 struct DkdvSmem {
+  // Q is read by S^T_n early in a step and by dK_n at its end, so it gets a
+  // third stage: Q_{n+1} can load while dK_{n-1} still reads Q_{n-1}.
+  static constexpr int kQStages = 3;
+  static constexpr int kDOStages = 2;
+  static constexpr int kStatStages = 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytesBf16;
-  static constexpr int kQ = kV + kTileBytesBf16;               // 2 stages
-  static constexpr int kDO = kQ + 2 * kTileBytesBf16;          // 2 stages
-  static constexpr int kStats = kDO + 2 * kTileBytesBf16;      // 2 stages x (128 lse2 + 128 delta) fp32
-  static constexpr int kBars = kStats + 2 * 2 * kTile * 4;
-  static constexpr int kBytes = kBars + 16 * 8;
-  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kQ = kV + kTileBytesBf16;
+  static constexpr int kDO = kQ + kQStages * kTileBytesBf16;
+  static constexpr int kStats = kDO + kDOStages * kTileBytesBf16;   // [stage] x (128 lse2 + 128 delta) fp32
+  static constexpr int kBars = kStats + kStatStages * 2 * kTile * 4;
+  static constexpr int kBytes = kBars + 24 * 8;
+  // No alignment slack: this layout fills the 227 KB a CTA may hold.  The
+  // dynamic shared window starts 1024-byte aligned on sm_100a (after the 1 KB
+  // the driver reserves); the kernel checks that and refuses to run otherwise.
+  static constexpr int kAlloc = kBytes;
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
 __device__ __forceinline__ int bwd_first_q_tile(int j, int Sq, int Sk, int causal) {
@@ -147,7 +158,11 @@ __device__ __forceinline__ int bwd_first_q_tile(int j, int Sq, int Sk, int causa
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using L = DkdvSmem;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem_u32(smem_raw) & 1023u) {              // the layout needs a 1024-byte aligned window
+    if (threadIdx.x == 0) raise_error(0x100 | kSiteBwdAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int warp = warp_id(), lane = lane_id();
 
   // Key tiles are the slow grid index so that, under a causal mask, the tiles
@@ -162,18 +177,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* kv_full = bars + 0;
-  uint64_t* st_full = bars + 1;      // [2]
-  uint64_t* st_empty = bars + 3;     // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* p_full = bars + 7;       // P^T written
-  uint64_t* acc_done = bars + 8;
-  uint64_t* ds_full = bars + 9;      // dS^T written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* q_full = bars + 1;       // [3]
+  uint64_t* q_empty = bars + 4;      // [3]
+  uint64_t* do_full = bars + 7;      // [2]
+  uint64_t* do_empty = bars + 9;     // [2]
+  uint64_t* s_full = bars + 11;
+  uint64_t* dp_full = bars + 12;
+  uint64_t* p_full = bars + 13;      // P^T written
+  uint64_t* acc_done = bars + 14;
+  uint64_t* ds_full = bars + 15;     // dS^T written
+  uint64_t* st_full = bars + 16;     // [2] LSE / Delta of a step staged (32 producer lanes)
+  uint64_t* st_empty = bars + 18;    // [2] the compute warps are done with them (one arrival per warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], 1); }
+    for (int s = 0; s < L::kQStages; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int s = 0; s < L::kDOStages; ++s) { mbar_init(&do_full[s], 1); mbar_init(&do_empty[s], 1); }
+    for (int s = 0; s < L::kStatStages; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], kBwdComputeWarps); }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, kBwdComputeWarps);   // one arrival per compute warp
@@ -197,18 +218,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     }
     bool ok = true;
     for (int n = 0; n < steps && ok; ++n) {
-      const int s = n & 1, u = n >> 1;
       const int g = n / (nq - i0), i = i0 + n % (nq - i0);
-      const int h = kvh * G + g;
-      const int bh = b * a.Hq + h;
-      if (n >= 2) ok = warp_wait(&st_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+      const int bh = b * a.Hq + kvh * G + g;
+      const int qs = n % L::kQStages, qu = n / L::kQStages;
+      if (n >= L::kQStages) ok = warp_wait(&q_empty[qs], (qu - 1) & 1, kSiteBwdStEmpty);
       if (!ok) break;
       if (lane == 0) {
-        mbar_expect_tx(&st_full[s], 2 * kTileBytesBf16);
-        tma_tile_bf16(smem + L::kQ + s * kTileBytesBf16, &a.tm_q, &st_full[s], i * kTile, bh);
-        tma_tile_bf16(smem + L::kDO + s * kTileBytesBf16, &a.tm_do, &st_full[s], i * kTile, bh);
+        mbar_arrive_expect_tx(&q_full[qs], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kQ + qs * kTileBytesBf16, &a.tm_q, &q_full[qs], i * kTile, bh);
       }
-      float* stats = reinterpret_cast<float*>(smem + L::kStats + s * 2 * kTile * 4);
+      const int ds = n % L::kDOStages, du = n / L::kDOStages;
+      if (n >= L::kDOStages) ok = warp_wait(&do_empty[ds], (du - 1) & 1, kSiteBwdStEmpty);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&do_full[ds], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kDO + ds * kTileBytesBf16, &a.tm_do, &do_full[ds], i * kTile, bh);
+      }
+      const int ss = n % L::kStatStages, su = n / L::kStatStages;
+      if (n >= L::kStatStages) ok = warp_wait(&st_empty[ss], (su - 1) & 1, kSiteBwdStEmpty);
+      if (!ok) break;
+      float* stats = reinterpret_cast<float*>(smem + L::kStats + ss * 2 * kTile * 4);
       for (int r = lane; r < kTile; r += 32) {
         const int qi = i * kTile + r;
         const bool valid = qi < a.Sq;
@@ -216,26 +245,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         stats[r] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
         stats[kTile + r] = valid ? __ldg(&a.delta[idx]) : 0.f;
       }
-      mbar_arrive(&st_full[s]);
+      mbar_arrive(&st_full[ss]);
     }
-    // drain outstanding loads
+    // drain: every load issued must land before the CTA exits
     if (lane == 0) {
-      mbar_wait(kv_full, 0, kSiteBwdKV);
-      for (int n = max(0, steps - 2); n < steps; ++n) mbar_wait(&st_full[n & 1], (n >> 1) & 1, kSiteBwdStFull);
+      mbar_wait_drain(kv_full, 0, kSiteBwdKV);
+      for (int n = max(0, steps - L::kQStages); n < steps; ++n)
+        mbar_wait_drain(&q_full[n % L::kQStages], (n / L::kQStages) & 1, kSiteBwdStFull);
+      for (int n = max(0, steps - L::kDOStages); n < steps; ++n)
+        mbar_wait_drain(&do_full[n % L::kDOStages], (n / L::kDOStages) & 1, kSiteBwdStFull);
     }
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-      auto sQ_of = [&](int n) { return smem_u32(smem + L::kQ + (n & 1) * kTileBytesBf16); };
-      auto sDO_of = [&](int n) { return smem_u32(smem + L::kDO + (n & 1) * kTileBytesBf16); };
+      auto sQ_of = [&](int n) { return smem_u32(smem + L::kQ + (n % L::kQStages) * kTileBytesBf16); };
+      auto sDO_of = [&](int n) { return smem_u32(smem + L::kDO + (n % L::kDOStages) * kTileBytesBf16); };
+      auto wait_q = [&](int n) { return mbar_wait(&q_full[n % L::kQStages], (n / L::kQStages) & 1, kSiteBwdStFull); };
+      auto wait_do = [&](int n) {
+        return mbar_wait(&do_full[n % L::kDOStages], (n / L::kDOStages) & 1, kSiteBwdStFull);
+      };
       // Issue order per step n: dV_n (once P^T_n is written), S^T_{n+1} (its
       // columns held P^T_n, which dV_n has read: one thread's MMAs run in
       // order), dK_n (once dS^T_n is written), dP^T_{n+1}.  The next step's S^T
       // thus runs while the compute warps form dS^T of this one.
       bool ok = mbar_wait(kv_full, 0, kSiteBwdKV);
-      if (ok && steps > 0) ok = mbar_wait(&st_full[0], 0, kSiteBwdStFull);
+      if (ok && steps > 0) ok = wait_q(0) && wait_do(0);
       if (ok && steps > 0) {
         tc_fence_after();
         mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(0), 0);   // S^T  = K Q^T
@@ -249,8 +285,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         if (!ok) break;
         tc_fence_after();
         mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO_of(n), n > 0);    // dV += P^T dO
+        mma_commit(&do_empty[n % L::kDOStages]);
         if (more) {
-          ok = mbar_wait(&st_full[(n + 1) & 1], ((n + 1) >> 1) & 1, kSiteBwdStFull);
+          ok = wait_q(n + 1);
           if (!ok) break;
           tc_fence_after();
           mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step
@@ -260,8 +297,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         if (!ok) break;
         tc_fence_after();
         mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ_of(n), n > 0);   // dK += dS^T Q
-        mma_commit(&st_empty[n & 1]);
+        mma_commit(&q_empty[n % L::kQStages]);
         if (more) {
+          ok = wait_do(n + 1);
+          if (!ok) break;
+          tc_fence_after();
           mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(n + 1), 0);         // dP^T of the next step
           mma_commit(dp_full);
         }
@@ -281,16 +321,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     const float c = a.scale_log2;
     bool ok = true;
     for (int n = 0; n < steps && ok; ++n) {
-      const int s = n & 1, u = n >> 1;
       const int i = i0 + n % (nq - i0);
-      ok = warp_wait(&st_full[s], u & 1, kSiteBwdStFull);
+      const int ss = n % L::kStatStages;
+      ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
       if (ok) ok = warp_wait(s_full, n & 1, kSiteBwdS);
       if (!ok) break;
       tc_fence_after();
-      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + s * 2 * kTile * 4) + hc * 16;
+      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + ss * 2 * kTile * 4) + hc * 16;
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
       const int q_first = i * kTile + hc * 64;       // first query of this warp's columns
+
       const bool need_mask = a.causal && (q_first < lim);
       const float2 c2 = make_float2(c, c);
       // P^T as 32 bf16 pairs: the values dV's MMA consumes, reused for dS^T
@@ -354,7 +395,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) {
+        mbar_arrive(ds_full);
+        mbar_arrive(&st_empty[ss]);                  // done with this step's LSE / Delta
+      }
     }
     if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
     if (ok) {
@@ -374,13 +418,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 
 // ---------------------------------------------------------------------------- dQ
 struct DqSmem {
+  // K is read by S_j and again by dQ_j two steps of MMAs later, so it gets a
+  // third stage: K_{j+2} can load while dQ_j still reads K_j.
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 2;
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + kTileBytesBf16;
-  static constexpr int kK = kDO + kTileBytesBf16;              // 2 stages
-  static constexpr int kV = kK + 2 * kTileBytesBf16;           // 2 stages
-  static constexpr int kBars = kV + 2 * kTileBytesBf16;
-  static constexpr int kBytes = kBars + 16 * 8;
+  static constexpr int kK = kDO + kTileBytesBf16;
+  static constexpr int kV = kK + kKStages * kTileBytesBf16;
+  static constexpr int kBars = kV + kVStages * kTileBytesBf16;
+  static constexpr int kBytes = kBars + 18 * 8;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
@@ -405,22 +454,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2 S buffers]
-  uint64_t* dp_full = bars + 11;
-  uint64_t* ds_full = bars + 12;
-  uint64_t* dq_done = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* k_full = bars + 1;    // [3]
+  uint64_t* k_empty = bars + 4;   // [3]
+  uint64_t* v_full = bars + 7;    // [2]
+  uint64_t* v_empty = bars + 9;   // [2]
+  uint64_t* s_full = bars + 11;   // [2 S buffers]
+  uint64_t* dp_full = bars + 13;
+  uint64_t* ds_full = bars + 14;
+  uint64_t* dq_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
-    }
+    for (int s = 0; s < L::kKStages; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < L::kVStages; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
@@ -443,45 +490,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       tma_tile_bf16(smem + L::kDO, &a.tm_do, q_full, i * kTile, bh);
       bool ok = true;
       for (int jj = 0; jj < n_kv && ok; ++jj) {
-        const int s = jj & 1, u = jj >> 1;
-        if (jj >= 2) ok = mbar_wait(&k_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+        const int ks = jj % L::kKStages, ku = jj / L::kKStages;
+        if (jj >= L::kKStages) ok = mbar_wait(&k_empty[ks], (ku - 1) & 1, kSiteBwdStEmpty);
         if (!ok) break;
-        mbar_arrive_expect_tx(&k_full[s], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kK + s * kTileBytesBf16, &a.tm_k, &k_full[s], jj * kTile, bkv);
-        if (jj >= 2) ok = mbar_wait(&v_empty[s], (u - 1) & 1, kSiteBwdStEmpty);
+        mbar_arrive_expect_tx(&k_full[ks], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kK + ks * kTileBytesBf16, &a.tm_k, &k_full[ks], jj * kTile, bkv);
+        const int vs = jj % L::kVStages, vu = jj / L::kVStages;
+        if (jj >= L::kVStages) ok = mbar_wait(&v_empty[vs], (vu - 1) & 1, kSiteBwdStEmpty);
         if (!ok) break;
-        mbar_arrive_expect_tx(&v_full[s], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kV + s * kTileBytesBf16, &a.tm_v, &v_full[s], jj * kTile, bkv);
+        mbar_arrive_expect_tx(&v_full[vs], kTileBytesBf16);
+        tma_tile_bf16(smem + L::kV + vs * kTileBytesBf16, &a.tm_v, &v_full[vs], jj * kTile, bkv);
       }
-      mbar_wait(q_full, 0, kSiteBwdKV);
-      for (int jj = max(0, n_kv - 2); jj < n_kv; ++jj) {
-        mbar_wait(&k_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull);
-        mbar_wait(&v_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull);
-      }
+      // drain: every load issued must land before the CTA exits
+      mbar_wait_drain(q_full, 0, kSiteBwdKV);
+      for (int jj = max(0, n_kv - L::kKStages); jj < n_kv; ++jj)
+        mbar_wait_drain(&k_full[jj % L::kKStages], (jj / L::kKStages) & 1, kSiteBwdStFull);
+      for (int jj = max(0, n_kv - L::kVStages); jj < n_kv; ++jj)
+        mbar_wait_drain(&v_full[jj % L::kVStages], (jj / L::kVStages) & 1, kSiteBwdStFull);
     }
     __syncwarp();
   } else if (warp == 9) {
     if (lane == 0) {
       const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-      auto sK_of = [&](int jj) { return smem_u32(smem + L::kK + (jj & 1) * kTileBytesBf16); };
-      auto sV_of = [&](int jj) { return smem_u32(smem + L::kV + (jj & 1) * kTileBytesBf16); };
+      auto sK_of = [&](int jj) { return smem_u32(smem + L::kK + (jj % L::kKStages) * kTileBytesBf16); };
+      auto sV_of = [&](int jj) { return smem_u32(smem + L::kV + (jj % L::kVStages) * kTileBytesBf16); };
       // S is double-buffered in TMEM: S_{j+1} is computed while the compute
       // warps work on step j.  Issue order: S_0, dP_0, S_1, then per step j:
       // dQ_j (once dS_j is written), dP_{j+1} (the compute warps have read dP_j),
       // S_{j+2} into the buffer dQ_j has just read dS_j from.
       auto issue_s = [&](int jj) -> bool {
-        if (!mbar_wait(&k_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull)) return false;
+        if (!mbar_wait(&k_full[jj % L::kKStages], (jj / L::kKStages) & 1, kSiteBwdStFull)) return false;
         tc_fence_after();
         mma_tile_ss_kmajor(tmem + s_col(jj), sQ, sK_of(jj), 0);         // S  = Q K^T
         mma_commit(&s_full[jj & 1]);
         return true;
       };
       auto issue_dp = [&](int jj) -> bool {
-        if (!mbar_wait(&v_full[jj & 1], (jj >> 1) & 1, kSiteBwdStFull)) return false;
+        if (!mbar_wait(&v_full[jj % L::kVStages], (jj / L::kVStages) & 1, kSiteBwdStFull)) return false;
         tc_fence_after();
         mma_tile_ss_kmajor(tmem + 128, sDO, sV_of(jj), 0);              // dP = dO V^T
         mma_commit(dp_full);
-        mma_commit(&v_empty[jj & 1]);
+        mma_commit(&v_empty[jj % L::kVStages]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, kSiteBwdKV);
@@ -492,7 +541,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         if (!ok) break;
         tc_fence_after();
         mma_tile_ts_mnmajor(tmem + 256, tmem + s_col(jj), sK_of(jj), jj > 0);   // dQ += dS K
-        mma_commit(&k_empty[jj & 1]);
+        mma_commit(&k_empty[jj % L::kKStages]);
         if (jj + 1 < n_kv) ok = issue_dp(jj + 1);
         if (ok && jj + 2 < n_kv) ok = issue_s(jj + 2);
       }
