@@ -301,40 +301,63 @@ def time_steps(step, K, W, world, flush, sampler_index=None):
 
 
 def e2e_video_like(step, K, W):
-    """Same metric through the public API with pinned HOST buffers: H2D of the
-    step's inputs, the call, D2H of O and LSE, all inside the timed region."""
+    """Same metric through the public API with pinned HOST buffers: every step
+    copies its inputs host -> device, calls attn_fwd and copies O and LSE back;
+    all of it inside the timed region.  Steps are pipelined the way a server
+    would run them: two buffer sets, the copy in of step k+1 and the copy out
+    of step k-1 overlap the kernel of step k (separate streams, event-ordered)."""
     h = step.h
     names = ["q", "k", "v"] + (["q_descale", "k_descale", "v_descale"] if step.name == "fp8" else [])
     host = {n: step.host[n].pin_memory() for n in names}
-    dev = {n: torch.empty_like(step.x[n]) for n in names}
-    out_h = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    lse_h = torch.empty(step.lse.shape, dtype=step.lse.dtype).pin_memory()
-    stream = torch.cuda.current_stream()
+    sets = []
+    for _ in range(2):
+        sets.append({"in": {n: torch.empty_like(step.x[n]) for n in names},
+                     "out": torch.empty_like(step.out), "lse": torch.empty_like(step.lse),
+                     "out_h": torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory(),
+                     "lse_h": torch.empty(step.lse.shape, dtype=step.lse.dtype).pin_memory(),
+                     "in_done": torch.cuda.Event(), "run_done": torch.cuda.Event(), "out_done": torch.cuda.Event()})
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def one():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
+    def one(k):
+        b = sets[k % 2]
+        if k >= 2:
+            s_in.wait_event(b["run_done"])          # step k-2 is done reading these inputs
+        with torch.cuda.stream(s_in):
+            for n in names:
+                b["in"][n].copy_(host[n], non_blocking=True)
+        b["in_done"].record(s_in)
+        s_run.wait_event(b["in_done"])
+        if k >= 2:
+            s_run.wait_event(b["out_done"])         # step k-2's outputs have left the device
         ds = {}
         if step.name == "fp8":
-            ds = dict(q_descale=dev["q_descale"], k_descale=dev["k_descale"], v_descale=dev["v_descale"])
-        h.attn_fwd(dev["q"], dev["k"], dev["v"], out=step.out, lse=step.lse, **ds)
-        out_h.copy_(step.out, non_blocking=True)
-        lse_h.copy_(step.lse, non_blocking=True)
+            ds = dict(q_descale=b["in"]["q_descale"], k_descale=b["in"]["k_descale"], v_descale=b["in"]["v_descale"])
+        with torch.cuda.stream(s_run):
+            h.attn_fwd(b["in"]["q"], b["in"]["k"], b["in"]["v"], out=b["out"], lse=b["lse"], stream=s_run, **ds)
+        b["run_done"].record(s_run)
+        s_out.wait_event(b["run_done"])
+        with torch.cuda.stream(s_out):
+            b["out_h"].copy_(b["out"], non_blocking=True)
+            b["lse_h"].copy_(b["lse"], non_blocking=True)
+        b["out_done"].record(s_out)
 
-    for _ in range(W):
-        one()
+    for k in range(W):
+        one(k)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(K):
-        one()
-    b.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for k in range(K):
+        one(k)
+    s_out.wait_event(sets[(K - 1) % 2]["out_done"])
+    end.record(s_out)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / K
+    ms = start.elapsed_time(end) / K
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    d2h = sets[0]["out_h"].numel() * sets[0]["out_h"].element_size() + \
+        sets[0]["lse_h"].numel() * sets[0]["lse_h"].element_size()
     return {"value": step.flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelining": "2 buffer sets; copy in of step k+1 and copy out of step k-1 overlap step k's kernel"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing
