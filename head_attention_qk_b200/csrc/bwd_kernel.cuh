@@ -238,12 +238,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       if (n >= L::kStatStages) ok = warp_wait(&st_empty[ss], (su - 1) & 1, kSiteBwdStEmpty);
       if (!ok) break;
       float* stats = reinterpret_cast<float*>(smem + L::kStats + ss * 2 * kTile * 4);
-      for (int r = lane; r < kTile; r += 32) {
-        const int qi = i * kTile + r;
-        const bool valid = qi < a.Sq;
-        const size_t idx = (size_t)bh * a.Sq + (valid ? qi : 0);
-        stats[r] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
-        stats[kTile + r] = valid ? __ldg(&a.delta[idx]) : 0.f;
+      {
+        // all eight global loads in flight before the first store
+        float lv[kTile / 32], dv[kTile / 32];
+#pragma unroll
+        for (int k = 0; k < kTile / 32; ++k) {
+          const int qi = i * kTile + lane + 32 * k;
+          const bool valid = qi < a.Sq;
+          const size_t idx = (size_t)bh * a.Sq + (valid ? qi : 0);
+          lv[k] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
+          dv[k] = valid ? __ldg(&a.delta[idx]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kTile / 32; ++k) {
+          stats[lane + 32 * k] = lv[k];
+          stats[kTile + lane + 32 * k] = dv[k];
+        }
       }
       mbar_arrive(&st_full[ss]);
     }
