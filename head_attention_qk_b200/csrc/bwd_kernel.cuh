@@ -12,21 +12,24 @@
 //   bwd_dkdv_kernel   one CTA per (b, kv head, 128-key tile); loops over the
 //                     group's query heads (ascending) and their 128-row query
 //                     tiles (ascending).  Per step, four tcgen05 MMAs:
-//                       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q.
+//                       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q
+//                     (S^T of the next step and dV in two query halves).
 //   bwd_dq_kernel     one CTA per (b, q head, 128-row query tile); loops over
 //                     KV tiles (ascending).  Per step, three MMAs:
 //                       S = Q K^T, dP = dO V^T, dQ += dS K.
 //
 // Roles: warps 0-7 compute, warp 8 TMA producer, warp 9 MMA issuer and
 // tensor-memory owner.  Compute warp w owns tile rows 32 (w % 4) .. +31 (its
-// TMEM lane quarter) and columns 64 (w / 4) .. +63 of S, dP: nothing in P or dS
+// TMEM lane quarter) and half of the columns of S, dP: nothing in P or dS
 // needs a reduction along a row (the row statistics LSE and Delta come from the
 // forward), so the two warps of a lane quarter split the columns, and two
-// warps per SM sub-partition keep the MUFU exponentials fed.  Each writes its
-// 16-bit P or dS into the first 32 of its own 64 S / dP columns, so the MMAs
-// read them with a 32-column gap after the first 64 keys.  P and dS are
-// rounded to bf16 before their MMAs; S, dP and the dQ/dK/dV accumulators are
-// fp32.
+// warps per SM sub-partition keep the MUFU exponentials fed.  Each packs its
+// 16-bit P or dS over the first half of the fp32 columns it read.  In dQ warp
+// w holds columns 64 (w / 4) .. +63; in dK/dV it holds columns 32 (w / 4) +
+// 64 c .. +31 for chunks c = 0, 1, so that all eight warps finish the P^T of
+// queries 0..63 first and the MMAs of that half start while they form the
+// other.  P and dS are rounded to bf16 before their MMAs; S, dP and the
+// dQ/dK/dV accumulators are fp32.
 #pragma once
 
 #include "fwd_kernel.cuh"
@@ -96,13 +99,48 @@ __device__ __forceinline__ void mma_tile_ss_kmajor(uint32_t d, uint32_t sa, uint
 // shared-memory tile read MN-major: the reduction runs over the tile's rows.
 // A's reduction elements 0..63 sit in columns [0, 32) and 64..127 in [64, 96)
 // (each half written by the warp that owns those 64 columns of S or dP).
-__device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
+__device__ __forceinline__ void mma_tile_ts_mnmajor_halves(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
   constexpr uint32_t idesc = make_idesc(1, 1, 1, 128, 128);
   constexpr uint32_t hi = sdesc_hi(1024);
   const uint32_t b_lo = sdesc_lo(sb, 16384);
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     mma_f16_ts2(d, a_tmem + k * 8 + (k >> 2) * 32, b_lo + k * (2048 >> 4), hi, idesc, (acc || k > 0) ? 1u : 0u);
+}
+
+// D = A B^T for the 64 B rows 64 h .. 64 h + 63 only (M = 128, N = 64, K = 128),
+// both operands K-major bf16 tiles in shared memory.  Row 64 of a swizzled
+// tile starts 8 KB into each 16 KB half, a whole number of swizzle atoms.
+__device__ __forceinline__ void mma_tile_ss_kmajor_n64(uint32_t d, uint32_t sa, uint32_t sb, int h) {
+  constexpr uint32_t idesc = make_idesc(1, 1, 0, 128, 64);
+  constexpr uint32_t hi = sdesc_hi(1024);
+  const uint32_t a_lo = sdesc_lo(sa, 16), b_lo = sdesc_lo(sb + h * 8192, 16);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+    mma_f16_ss2(d, a_lo + off, hi, b_lo + off, hi, idesc, k > 0 ? 1u : 0u);
+  }
+}
+
+// TMEM column (relative to the S^T or dP^T block) of the bf16 pairs that hold
+// reduction elements 16 k .. 16 k + 15 of P^T or dS^T.  Reduction element q
+// (a query) is computed by the warp with column half (q / 32) % 2 in its chunk
+// q / 64, which packs its 32 values over the first 16 of its 32 fp32 columns.
+__device__ __forceinline__ constexpr uint32_t bwd_pair_col(int k) {
+  return (uint32_t)((k >> 2) * 64 + ((k >> 1) & 1) * 32 + (k & 1) * 8);
+}
+
+// D (+)= A B over reduction groups K0 .. K1-1 (16 elements each), where A
+// (128 rows of bf16 pairs, laid out by bwd_pair_col) is in tensor memory and
+// B is a shared-memory tile read MN-major: the reduction runs over its rows.
+template <int K0, int K1>
+__device__ __forceinline__ void mma_tile_ts_mnmajor(uint32_t d, uint32_t a_tmem, uint32_t sb, uint32_t acc) {
+  constexpr uint32_t idesc = make_idesc(1, 1, 1, 128, 128);
+  constexpr uint32_t hi = sdesc_hi(1024);
+  const uint32_t b_lo = sdesc_lo(sb, 16384);
+#pragma unroll
+  for (int k = K0; k < K1; ++k)
+    mma_f16_ts2(d, a_tmem + bwd_pair_col(k), b_lo + k * (2048 >> 4), hi, idesc, (acc || k > K0) ? 1u : 0u);
 }
 
 // Read 64 columns of an fp32 TMEM row (from taddr), scale them and store them as
@@ -181,23 +219,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   uint64_t* q_empty = bars + 4;      // [3]
   uint64_t* do_full = bars + 7;      // [2]
   uint64_t* do_empty = bars + 9;     // [2]
-  uint64_t* s_full = bars + 11;
-  uint64_t* dp_full = bars + 12;
-  uint64_t* p_full = bars + 13;      // P^T written
-  uint64_t* acc_done = bars + 14;
-  uint64_t* ds_full = bars + 15;     // dS^T written
-  uint64_t* st_full = bars + 16;     // [2] LSE / Delta of a step staged (32 producer lanes)
-  uint64_t* st_empty = bars + 18;    // [2] the compute warps are done with them (one arrival per warp)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* s_full = bars + 11;      // [2] S^T columns of query half 0 / 1
+  uint64_t* dp_full = bars + 13;
+  uint64_t* p_full = bars + 14;      // [2] P^T of query half 0 / 1 written
+  uint64_t* acc_done = bars + 16;
+  uint64_t* ds_full = bars + 17;     // dS^T written
+  uint64_t* st_full = bars + 18;     // [2] LSE / Delta of a step staged (32 producer lanes)
+  uint64_t* st_empty = bars + 20;    // [2] the compute warps are done with them (one arrival per warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < L::kQStages; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < L::kDOStages; ++s) { mbar_init(&do_full[s], 1); mbar_init(&do_empty[s], 1); }
     for (int s = 0; s < L::kStatStages; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], kBwdComputeWarps); }
-    mbar_init(s_full, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&s_full[h], 1);
+      mbar_init(&p_full[h], kBwdComputeWarps);   // one arrival per compute warp
+    }
     mbar_init(dp_full, 1);
-    mbar_init(p_full, kBwdComputeWarps);   // one arrival per compute warp
     mbar_init(ds_full, kBwdComputeWarps);
     mbar_init(acc_done, 1);
     fence_barrier_init();
@@ -276,37 +316,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       auto wait_do = [&](int n) {
         return mbar_wait(&do_full[n % L::kDOStages], (n / L::kDOStages) & 1, kSiteBwdStFull);
       };
-      // Issue order per step n: dV_n (once P^T_n is written), S^T_{n+1} (its
-      // columns held P^T_n, which dV_n has read: one thread's MMAs run in
-      // order), dK_n (once dS^T_n is written), dP^T_{n+1}.  The next step's S^T
-      // thus runs while the compute warps form dS^T of this one.
+      // Issue order per step n, by query halves h = 0, 1: dV_n over the
+      // queries of half h (once P^T_n of that half is written), then S^T_{n+1}
+      // of half h (its columns held that half of P^T_n, which dV_n has read:
+      // one thread's MMAs run in order); then dK_n (once dS^T_n is written)
+      // and dP^T_{n+1}.  The next step's first half of S^T thus runs while the
+      // compute warps form the second half of P^T and then dS^T of this one.
       bool ok = mbar_wait(kv_full, 0, kSiteBwdKV);
       if (ok && steps > 0) ok = wait_q(0) && wait_do(0);
       if (ok && steps > 0) {
         tc_fence_after();
         mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(0), 0);   // S^T  = K Q^T
-        mma_commit(s_full);
+        mma_commit(&s_full[0]);
+        mma_commit(&s_full[1]);
         mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(0), 0);  // dP^T = V dO^T
         mma_commit(dp_full);
       }
       for (int n = 0; n < steps && ok; ++n) {
         const bool more = n + 1 < steps;
-        ok = mbar_wait(p_full, n & 1, kSiteBwdP);
+        ok = mbar_wait(&p_full[0], n & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 0, tmem + 256, sDO_of(n), n > 0);    // dV += P^T dO
-        mma_commit(&do_empty[n % L::kDOStages]);
+        mma_tile_ts_mnmajor<0, 4>(tmem + 0, tmem + 256, sDO_of(n), n > 0);   // dV += P^T dO, queries 0..63
         if (more) {
           ok = wait_q(n + 1);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step
-          mma_commit(s_full);
+          mma_tile_ss_kmajor_n64(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step, half 0
+          mma_commit(&s_full[0]);
+        }
+        ok = mbar_wait(&p_full[1], n & 1, kSiteBwdP);
+        if (!ok) break;
+        tc_fence_after();
+        mma_tile_ts_mnmajor<4, 8>(tmem + 0, tmem + 256, sDO_of(n), 1);       // queries 64..127
+        mma_commit(&do_empty[n % L::kDOStages]);
+        if (more) {
+          mma_tile_ss_kmajor_n64(tmem + 320, sK, sQ_of(n + 1), 1);          // half 1
+          mma_commit(&s_full[1]);
         }
         ok = mbar_wait(ds_full, n & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 128, tmem + 384, sQ_of(n), n > 0);   // dK += dS^T Q
+        mma_tile_ts_mnmajor<0, 8>(tmem + 128, tmem + 384, sQ_of(n), n > 0);  // dK += dS^T Q
         mma_commit(&q_empty[n % L::kQStages]);
         if (more) {
           ok = wait_do(n + 1);
@@ -323,42 +374,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   } else {
     // ---------------------------------------------------------------- compute (warps 0-7)
     const int r = (warp & 3) * 32 + lane;            // key row within the tile
-    const int hc = warp >> 2;                        // column half: queries 64 hc .. 64 hc + 63
+    const int hc = warp >> 2;                        // queries 64 c + 32 hc .. +31 in chunk c = 0, 1
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + 256 + hc * 64;   // this warp's 64 S^T (then P^T) columns
-    const uint32_t tP = tmem + lane_base + 384 + hc * 64;   // this warp's 64 dP^T (then dS^T) columns
+    const uint32_t tS = tmem + lane_base + 256 + hc * 32;   // S^T (then P^T) columns of chunk 0; chunk 1 at +64
+    const uint32_t tP = tmem + lane_base + 384 + hc * 32;   // dP^T (then dS^T) columns, same layout
     const int kj = j * kTile + r;
     const float c = a.scale_log2;
+    const float2 c2 = make_float2(c, c);
     bool ok = true;
     for (int n = 0; n < steps && ok; ++n) {
       const int i = i0 + n % (nq - i0);
       const int ss = n % L::kStatStages;
       ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
-      if (ok) ok = warp_wait(s_full, n & 1, kSiteBwdS);
       if (!ok) break;
-      tc_fence_after();
-      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + ss * 2 * kTile * 4) + hc * 16;
+      // LSE (log2 domain) then Delta of the tile's 128 queries
+      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + ss * 2 * kTile * 4) + hc * 8;
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
-      const int q_first = i * kTile + hc * 64;       // first query of this warp's columns
-
-      const bool need_mask = a.causal && (q_first < lim);
-      const float2 c2 = make_float2(c, c);
-      // P^T as 32 bf16 pairs: the values dV's MMA consumes, reused for dS^T
-      uint32_t pk[32];
+      // P^T as bf16 pairs, per chunk: the values dV's MMA consumes, reused for dS^T
+      uint32_t pk[2][16];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int ch = 0; ch < 2; ++ch) {
+        ok = warp_wait(&s_full[ch], n & 1, kSiteBwdS);
+        if (!ok) break;
+        tc_fence_after();
+        const int q_first = i * kTile + ch * 64 + hc * 32;   // first query of these 32 columns
+        const bool need_mask = a.causal && (q_first < lim);
         uint32_t u[32];
-        tmem_ld32(tS + q * 32, u);
+        tmem_ld32(tS + ch * 64, u);
         tmem_wait_ld();
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-          const int e = q * 32 + 4 * k4;
-          const float4 l4 = lds128(&stats4[e / 4]); // log2-domain LSE of queries e .. e+3 (broadcast)
-          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(u[4 * k4]), __uint_as_float(u[4 * k4 + 1])), c2,
+          const int e = 4 * k4;
+          const float4 l4 = lds128(&stats4[ch * 16 + k4]);   // queries e .. e+3 of the chunk (broadcast)
+          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
                                        make_float2(-l4.x, -l4.y));
-          const float2 x1 = __ffma2_rn(make_float2(__uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3])),
-                                       c2, make_float2(-l4.z, -l4.w));
+          const float2 x1 = __ffma2_rn(make_float2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3])), c2,
+                                       make_float2(-l4.z, -l4.w));
           float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x), p3 = ex2_approx(x1.y);
           if (need_mask) {
             const int q0 = q_first + e;
@@ -367,41 +419,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             p2 = q0 + 2 < lim ? 0.f : p2;
             p3 = q0 + 3 < lim ? 0.f : p3;
           }
-          pk[e / 2] = pack_bf16x2(p0, p1);
-          pk[e / 2 + 1] = pack_bf16x2(p2, p3);
+          pk[ch][e / 2] = pack_bf16x2(p0, p1);
+          pk[ch][e / 2 + 1] = pack_bf16x2(p2, p3);
         }
+        __syncwarp();
+        tmem_st16(tS + ch * 64, pk[ch]);             // P^T over the first 16 of these columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[ch]);
       }
-      __syncwarp();
-      tmem_st32(tS, pk);                             // P^T over the first 32 of these columns
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (!ok) break;
       ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t uu[32];
-        tmem_ld32(tP + q * 32, uu);
+        tmem_ld32(tP + ch * 64, uu);
         tmem_wait_ld();
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-          const int e = q * 32 + 4 * k4;
-          const float4 d4 = lds128(&stats4[kTile / 4 + e / 4]);  // Delta of queries e .. e+3
-          const uint32_t w0 = pk[e / 2], w1 = pk[e / 2 + 1];
+          const int e = 4 * k4;
+          const float4 d4 = lds128(&stats4[kTile / 4 + ch * 16 + k4]);   // Delta of queries e .. e+3
+          const uint32_t w0 = pk[ch][e / 2], w1 = pk[ch][e / 2 + 1];
           const float2 pa = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
           const float2 pb = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
-          const float2 a0 = __fmul2_rn(pa, __fadd2_rn(make_float2(__uint_as_float(uu[4 * k4]), __uint_as_float(uu[4 * k4 + 1])),
+          const float2 a0 = __fmul2_rn(pa, __fadd2_rn(make_float2(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1])),
                                                       make_float2(-d4.x, -d4.y)));
-          const float2 a1 = __fmul2_rn(pb, __fadd2_rn(make_float2(__uint_as_float(uu[4 * k4 + 2]), __uint_as_float(uu[4 * k4 + 3])),
+          const float2 a1 = __fmul2_rn(pb, __fadd2_rn(make_float2(__uint_as_float(uu[e + 2]), __uint_as_float(uu[e + 3])),
                                                       make_float2(-d4.z, -d4.w)));
-          pk[e / 2] = pack_bf16x2(a0.x, a0.y);
-          pk[e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
+          pk[ch][e / 2] = pack_bf16x2(a0.x, a0.y);
+          pk[ch][e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
         }
+        __syncwarp();
+        tmem_st16(tP + ch * 64, pk[ch]);             // dS^T over the first 16 of these columns
       }
-      __syncwarp();
-      tmem_st32(tP, pk);                             // dS^T over the first 32 of these columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -550,7 +603,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         ok = mbar_wait(ds_full, jj & 1, kSiteBwdP);
         if (!ok) break;
         tc_fence_after();
-        mma_tile_ts_mnmajor(tmem + 256, tmem + s_col(jj), sK_of(jj), jj > 0);   // dQ += dS K
+        mma_tile_ts_mnmajor_halves(tmem + 256, tmem + s_col(jj), sK_of(jj), jj > 0);   // dQ += dS K
         mma_commit(&k_empty[jj % L::kKStages]);
         if (jj + 1 < n_kv) ok = issue_dp(jj + 1);
         if (ok && jj + 2 < n_kv) ok = issue_s(jj + 2);
