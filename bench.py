@@ -56,8 +56,10 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)",
                   "cross": "long-query cross-attention fwd (B1 H40 Sq90000 Sk512 D128 bf16)",
                   "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)",
+                  "bf16_75600": "bf16 attention fwd at the fp8 shape (B1 H5 S75600 D128)",
+                  "fp8_32760": "fp8 e4m3 attention fwd at the video shape (B1 H40 S32760 D128, Q/K RMS-norm)",
                   "fp8_prep": "e4m3 prologue of the fp8 config (Q, K RMS-normalised; V plain; per-head descales)"}
-FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window")
+FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window", "bf16_75600", "fp8_32760")
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
 
@@ -209,8 +211,8 @@ class Step:
             self.out = torch.empty((w.B, w.Hq, w.Sq, w.D), dtype=torch.bfloat16, device="cuda")
             self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
             self.flops = w.fwd_flops()
-            self.dtype = "e4m3" if name == "fp8" else "bf16"
-            if name == "fp8":
+            self.dtype = w.dtype
+            if w.dtype == "e4m3":
                 self.launches = 2          # V widened to fp16, then the attention kernel
         elif name == "llm_gqa":
             x = make_bwd_inputs(w)
@@ -260,7 +262,7 @@ class Step:
         if self.name in FWD_WORKLOADS:
             x = self.x
             ds = {}
-            if self.name == "fp8":
+            if w.dtype == "e4m3":
                 ds = dict(q_descale=x["q_descale"], k_descale=x["k_descale"], v_descale=x["v_descale"])
             h.attn_fwd(x["q"], x["k"], x["v"], out=self.out, lse=self.lse, **ds)
         elif self.name == "fp8_prep":
@@ -307,7 +309,7 @@ def e2e_video_like(step, K, W):
     would run them: two buffer sets, the copy in of step k+1 and the copy out
     of step k-1 overlap the kernel of step k (separate streams, event-ordered)."""
     h = step.h
-    names = ["q", "k", "v"] + (["q_descale", "k_descale", "v_descale"] if step.name == "fp8" else [])
+    names = ["q", "k", "v"] + (["q_descale", "k_descale", "v_descale"] if step.dtype == "e4m3" else [])
     host = {n: step.host[n].pin_memory() for n in names}
     sets = []
     for _ in range(2):
@@ -330,7 +332,7 @@ def e2e_video_like(step, K, W):
         if k >= 2:
             s_run.wait_event(b["out_done"])         # step k-2's outputs have left the device
         ds = {}
-        if step.name == "fp8":
+        if step.dtype == "e4m3":
             ds = dict(q_descale=b["in"]["q_descale"], k_descale=b["in"]["k_descale"], v_descale=b["in"]["v_descale"])
         with torch.cuda.stream(s_run):
             h.attn_fwd(b["in"]["q"], b["in"]["k"], b["in"]["v"], out=b["out"], lse=b["lse"], stream=s_run, **ds)
@@ -404,7 +406,8 @@ def run_reference(args, world, rank):
         return 0
     name = args.workload
     w = workloads.get(name)
-    rows = {"tiny": 256, "video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64, "cross": 256, "window": 48}[name]
+    rows = {"tiny": 256, "video": 16, "fp8": 32, "llm_gqa": 256, "streaming": 64, "cross": 256, "window": 48,
+            "bf16_75600": 32, "fp8_32760": 16}[name]
     vals = []
     for _ in range(args.warmup):
         oracle_sample_tflops(name, rows)

@@ -72,6 +72,11 @@ CONFIGS = {
                           n_blocks=21, text_len=512),
     "cross": Workload("cross", B=1, Hq=40, Hkv=40, Sq=90000, Sk=512, seed=5),
     "window": Workload("window", B=1, Hq=12, Hkv=12, Sq=4680, Sk=51480, seed=6),
+    # the precision pair the FP8 page compares (AITER PR #2911, Test Result:
+    # bf16 and fp8 fmha on the same 75600-token shape), measured on both shapes
+    "bf16_75600": Workload("bf16_75600", B=1, Hq=5, Hkv=5, Sq=75600, Sk=75600, seed=7),
+    "fp8_32760": Workload("fp8_32760", B=1, Hq=40, Hkv=40, Sq=32760, Sk=32760, dtype="e4m3", seed=8,
+                          qk_rmsnorm=True),
 }
 
 
