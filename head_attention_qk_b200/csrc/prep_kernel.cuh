@@ -5,9 +5,13 @@
 // tensor- or slice-granularity scales) and section 1.2 (head-scoped Q/K
 // normalisation, optional FP8 SDPA), with the clamp to the e4m3fn range +-448
 // that VeOmni PR #1363 describes for its quantizers.  Per (batch, head):
-//   r       = 1 / sqrt(mean_d x_d^2 + eps)   per row (only with rmsnorm), fp64,
-//             the squares summed over d = 0 .. 127 in ascending order
-//   y_d     = (float)(x_d * r), or x_d without rmsnorm
+//   ss      = sum of x_d^2 over the row (fp32, every operation rounded to
+//             nearest): lane k of the row's 16 threads adds the squares of
+//             d = 8k .. 8k+7 in ascending order, then the 16 partial sums are
+//             added pairwise, neighbours first (k with k^1, then pairs with
+//             pairs, ...); the squares of bf16 values are exact in fp32
+//   r       = 1 / sqrt(ss / 128 + eps)          per row (only with rmsnorm), fp32
+//   y_d     = x_d * r (fp32), or x_d without rmsnorm
 //   descale = max |y| / 448 over the head (1 if that max is 0), fp32
 //   code    = e4m3 of y / descale: fp32 quotient, round to nearest even,
 //             saturating at +-448
@@ -16,7 +20,9 @@
 // head split.  Three launches (after a memset of the descale array): the head
 // maxima (atomicMax on the non-negative fp32 bit patterns, which order like
 // integers, so the result does not depend on the order), max -> descale in
-// place, and the codes.  HBM-bound: x is read twice and the codes written once.
+// place, and the codes.  HBM-bound: x is read twice and the codes written once;
+// 16 threads share a row, so a warp reads two whole rows (512 contiguous
+// bytes) per load and writes two rows of codes (256 bytes) per store.
 #pragma once
 
 #include "sm100.cuh"
@@ -24,59 +30,59 @@
 namespace hattn {
 
 constexpr int kPrepD = 128;
-constexpr int kPrepThreads = 256;   // one row per thread
+constexpr int kPrepThreads = 256;     // 16 rows at a time: 16 threads per row, 8 values each
+constexpr int kPrepRowsPerCta = 64;   // 4 rows per thread, their loads issued together
 
-// Per-row normalisation factor (1 without rmsnorm): squares summed in fp64 in
-// ascending d (each square is exact in fp64).  The row is streamed in 64-byte
-// pieces, so few registers stay live; the second pass over the row (y) hits L1.
-__device__ __forceinline__ double prep_row_factor(const uint4* __restrict__ row, int rmsnorm, double eps) {
-  if (!rmsnorm) return 1.0;
-  double sum = 0.0;
-#pragma unroll 2
-  for (int i = 0; i < 16; i += 4) {
-    uint4 w[4];
+// This lane's 8 values (d = 8 (lane % 16) .. +7 of its row) as fp32.
+struct PrepVals {
+  float v[8];
+};
+
+__device__ __forceinline__ PrepVals prep_unpack(uint4 w) {
+  PrepVals p;
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k] = __ldg(&row[i + k]);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t p[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const double lo = (double)__uint_as_float(p[t] << 16);
-        const double hi = (double)__uint_as_float(p[t] & 0xFFFF0000u);
-        sum += lo * lo;
-        sum += hi * hi;
-      }
-    }
+  for (int t = 0; t < 4; ++t) {
+    p.v[2 * t] = __uint_as_float(u[t] << 16);
+    p.v[2 * t + 1] = __uint_as_float(u[t] & 0xFFFF0000u);
   }
-  return 1.0 / sqrt(sum / (double)kPrepD + eps);
+  return p;
 }
 
-__device__ __forceinline__ float prep_y(uint32_t bits16_as_f32, double r, int rmsnorm) {
-  const float v = __uint_as_float(bits16_as_f32);
-  return rmsnorm ? (float)((double)v * r) : v;
-}
-
-// grid (ceil(S / 256), B*H): the largest |y| of each head into amax_bits (zeroed).
-__global__ void __launch_bounds__(kPrepThreads, 4) prep_amax_kernel(const uint16_t* __restrict__ x,
-                                                                      unsigned int* __restrict__ amax_bits, int S,
-                                                                      int rmsnorm, double eps) {
-  const int bh = blockIdx.y;
-  const int s = blockIdx.x * kPrepThreads + threadIdx.x;
-  float m = 0.f;
-  if (s < S) {
-    const uint4* row = reinterpret_cast<const uint4*>(x) + ((long long)bh * S + s) * 16;
-    const double r = prep_row_factor(row, rmsnorm, eps);
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-      const uint4 w = __ldg(&row[i]);
-      const uint32_t p[4] = {w.x, w.y, w.z, w.w};
+// Row factor r = 1 / sqrt(ss / 128 + eps) (1 without rmsnorm); every lane of
+// the row's 16 gets the same bits (fp32 addition is commutative).  Rounded
+// operations are spelt out so that no multiply-add is contracted.
+__device__ __forceinline__ float prep_row_factor(const PrepVals& p, int rmsnorm, float eps) {
+  if (!rmsnorm) return 1.f;
+  float s = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        m = fmaxf(m, fabsf(prep_y(p[k] << 16, r, rmsnorm)));
-        m = fmaxf(m, fabsf(prep_y(p[k] & 0xFFFF0000u, r, rmsnorm)));
-      }
-    }
+  for (int t = 0; t < 8; ++t) s = __fadd_rn(s, __fmul_rn(p.v[t], p.v[t]));
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+  return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fmul_rn(s, 0.0078125f), eps)));
+}
+
+// grid (ceil(S / 64), B*H): the largest |y| of each head into amax_bits (zeroed).
+__global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
+                                                                   unsigned int* __restrict__ amax_bits, int S,
+                                                                   int rmsnorm, float eps) {
+  const int bh = blockIdx.y;
+  const int sub = threadIdx.x & 15;               // which 8 values of the row
+  const int r0 = blockIdx.x * kPrepRowsPerCta + (threadIdx.x >> 4);
+  const uint4* base = reinterpret_cast<const uint4*>(x) + (long long)bh * S * 16 + sub;
+  uint4 w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int s = r0 + 16 * k;
+    w[k] = s < S ? __ldg(base + (long long)s * 16) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const PrepVals p = prep_unpack(w[k]);
+    const float r = prep_row_factor(p, rmsnorm, eps);   // rows past S are zero: y = 0
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m = fmaxf(m, fabsf(rmsnorm ? __fmul_rn(p.v[t], r) : p.v[t]));
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -119,36 +125,38 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   return r;
 }
 
-// grid (ceil(S / 256), B*H): the codes of each row.
-__global__ void __launch_bounds__(kPrepThreads, 4) prep_quantize_kernel(const uint16_t* __restrict__ x,
-                                                                          uint8_t* __restrict__ codes,
-                                                                          const float* __restrict__ descale, int S,
-                                                                          int rmsnorm, double eps) {
+// grid (ceil(S / 64), B*H): the codes of each row.
+__global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
+                                                                       uint8_t* __restrict__ codes,
+                                                                       const float* __restrict__ descale, int S,
+                                                                       int rmsnorm, float eps) {
   const int bh = blockIdx.y;
-  const int s = blockIdx.x * kPrepThreads + threadIdx.x;
-  if (s >= S) return;
-  const long long rowi = (long long)bh * S + s;
-  const uint4* row = reinterpret_cast<const uint4*>(x) + rowi * 16;
-  const double r = prep_row_factor(row, rmsnorm, eps);
+  const int sub = threadIdx.x & 15;
+  const int r0 = blockIdx.x * kPrepRowsPerCta + (threadIdx.x >> 4);
+  const uint4* base = reinterpret_cast<const uint4*>(x) + (long long)bh * S * 16 + sub;
+  uint2* dst = reinterpret_cast<uint2*>(codes) + (long long)bh * S * 16 + sub;
+  uint4 w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int s = r0 + 16 * k;
+    w[k] = s < S ? __ldg(base + (long long)s * 16) : make_uint4(0u, 0u, 0u, 0u);
+  }
   const float ds = __ldg(&descale[bh]);
   const float rcp = __frcp_rn(ds);
-  uint4* dst = reinterpret_cast<uint4*>(codes) + rowi * 8;
-#pragma unroll 2
-  for (int i = 0; i < 16; i += 2) {
-    uint32_t o[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 w = __ldg(&row[i + h]);
-      const uint32_t p[4] = {w.x, w.y, w.z, w.w};
-      uint16_t c[4];
+  for (int k = 0; k < 4; ++k) {
+    const PrepVals p = prep_unpack(w[k]);
+    const float r = prep_row_factor(p, rmsnorm, eps);   // all 16 lanes of the row take part
+    uint16_t c[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        c[k] = e4m3x2_rn_satfinite(prep_quotient(prep_y(p[k] << 16, r, rmsnorm), ds, rcp),
-                                   prep_quotient(prep_y(p[k] & 0xFFFF0000u, r, rmsnorm), ds, rcp));
-      o[2 * h] = (uint32_t)c[0] | ((uint32_t)c[1] << 16);
-      o[2 * h + 1] = (uint32_t)c[2] | ((uint32_t)c[3] << 16);
+    for (int t = 0; t < 4; ++t) {
+      const float y0 = rmsnorm ? __fmul_rn(p.v[2 * t], r) : p.v[2 * t];
+      const float y1 = rmsnorm ? __fmul_rn(p.v[2 * t + 1], r) : p.v[2 * t + 1];
+      c[t] = e4m3x2_rn_satfinite(prep_quotient(y0, ds, rcp), prep_quotient(y1, ds, rcp));
     }
-    dst[i / 2] = make_uint4(o[0], o[1], o[2], o[3]);
+    const int s = r0 + 16 * k;
+    if (s < S)
+      dst[(long long)s * 16] = make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
   }
 }
 

@@ -106,10 +106,13 @@ HATTN_API size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtyp
  *   codes   [B, H, S, D] e4m3fn codes out
  *   descale [B*H] fp32 out: the real value of code c of head (b, h) is
  *           decode(c) * descale[b*H + h], ready for attn_fwd's descales.
- * Per head: with rmsnorm != 0 each row is first divided by
- * sqrt(mean over d of x_d^2 + eps) (eps > 0; the squares summed in fp64 in
- * ascending d, the factor 1/sqrt(.) in fp64 and the product rounded to fp32),
- * giving y; without it y = x.  descale = max |y| / 448 (fp32; 1 if the head is
+ * Per head: with rmsnorm != 0 each row is first multiplied by
+ * r = 1 / sqrt(ss / 128 + eps), giving y; without it y = x.  All in fp32 with
+ * every operation rounded to nearest (eps > 0 is taken as fp32; ss is the sum
+ * of the row's squares: the squares of d = 8k .. 8k+7 added in ascending d for
+ * k = 0 .. 15, then those 16 partial sums added pairwise, neighbours first:
+ * (s0 + s1), (s2 + s3), ..., then ((s0 + s1) + (s2 + s3)), ... up to one sum).
+ * descale = max |y| / 448 (fp32; 1 if the head is
  * all zero), code = y / descale (fp32 quotient) rounded to the nearest e4m3fn
  * value, ties to even, saturating at +-448.  The result is bitwise the same for
  * any batch or head split.  Enqueues a memset of descale and three kernels;

@@ -337,9 +337,15 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
  * the scale slice is one (batch, head); the optional normalisation is a plain
  * RMS over the head dimension with eps and no weight; and each step is fixed
  * in precision and order, so that every code is a function of the input:
- *   sum_b   = sum over d = 0 .. D-1 ascending of x_d^2   (fp64, each square exact)
- *   r       = 1 / sqrt(sum_b / D + eps)                  (fp64, correctly rounded)
- *   y_d     = (float)(x_d * r)  (fp64 product, rounded to fp32); y = x without it
+ *   ss      = sum of the row's x_d^2 in fp32, each operation rounded to nearest:
+ *             sixteen partial sums s_k over d = 8k .. 8k+7 (ascending d), then
+ *             added pairwise, neighbours first: (s0 + s1), (s2 + s3), ...,
+ *             ((s0 + s1) + (s2 + s3)), ... down to one value (D = 128)
+ *   r       = 1 / sqrt(ss / 128 + eps)    (fp32: multiply by 2^-7, add the fp32
+ *             eps, square root and division, each correctly rounded)
+ *   y_d     = x_d * r rounded to fp32; y = x without the normalisation
+ * (the norm's precision is the kernel's: the pages fix none, and these values
+ * decide integer codes, so both sides take them in the same fp32 steps)
  *   amax    = max |y| over the head's S x D values       (fp32)
  *   descale = amax / 448 in fp32, or 1 when amax == 0
  *   code    = e4m3 of y / descale (fp32 quotient), rounded to nearest with
@@ -377,6 +383,8 @@ uint8_t oracle_e4m3_rne(float v) {
 int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int B, int H, int S, int D,
                          int rmsnorm, double eps) {
     if (B <= 0 || H <= 0 || S <= 0 || D <= 0 || !x || !codes || !descale) return -1;
+    if (rmsnorm && D != 128) return -1;
+    const float eps32 = (float)eps;
     const int64_t heads = (int64_t)B * H;
     int failed = 0;
     #pragma omp parallel for schedule(dynamic, 1)
@@ -386,18 +394,27 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
         const uint16_t* xh = x + bh * (int64_t)S * D;
         float amax = 0.f;
         for (int64_t s = 0; s < S; ++s) {
-            double r = 1.0;
+            float r = 1.0f;
             if (rmsnorm) {
-                double sum = 0.0;
-                for (int d = 0; d < D; ++d) {
-                    const double v = bf16_to_double(xh[s * D + d]);
-                    sum += v * v;
+                volatile float part[16];               /* volatile: every step rounded to fp32 */
+                for (int k = 0; k < 16; ++k) {
+                    float acc = 0.0f;
+                    for (int t = 0; t < 8; ++t) {
+                        const float v = (float)bf16_to_double(xh[s * D + 8 * k + t]);
+                        const float sq = v * v;
+                        acc = acc + sq;
+                    }
+                    part[k] = acc;
                 }
-                r = 1.0 / sqrt(sum / (double)D + eps);
+                for (int width = 1; width < 16; width *= 2)
+                    for (int k = 0; k < 16; k += 2 * width) part[k] = part[k] + part[k + width];
+                const float mean = part[0] * 0.0078125f;
+                const float den = sqrtf(mean + eps32);
+                r = 1.0f / den;
             }
             for (int d = 0; d < D; ++d) {
-                const double v = bf16_to_double(xh[s * D + d]);
-                const float yv = rmsnorm ? (float)(v * r) : (float)v;
+                const float v = (float)bf16_to_double(xh[s * D + d]);
+                const float yv = rmsnorm ? v * r : v;
                 y[s * D + d] = yv;
                 if (fabsf(yv) > amax) amax = fabsf(yv);
             }

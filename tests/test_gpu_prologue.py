@@ -53,6 +53,18 @@ def test_prologue_special_rows(h):
     check_exact(h, torch.zeros(1, 1, 9, 128, dtype=torch.bfloat16), True)   # all-zero head: descale 1
 
 
+def test_prologue_extreme_magnitudes(h):
+    # squares that underflow to fp32 subnormals (2^-70 scale), large rows (2^60),
+    # and a mix inside one row: every fp32 step of the norm is IEEE on both sides
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn(1, 2, 48, 128, generator=g)
+    x[0, 0, :16] *= 2.0 ** -70
+    x[0, 0, 16:32] *= 2.0 ** 60
+    x[0, 1, :, ::3] *= 2.0 ** -64
+    for rms in (False, True):
+        check_exact(h, x.to(torch.bfloat16), rms)
+
+
 def test_prologue_fp8_config_q_bit_exact(h):
     w = workloads.get("fp8")
     g = torch.Generator().manual_seed(w.seed)

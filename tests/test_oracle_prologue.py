@@ -75,15 +75,23 @@ def test_all_zero_head_has_unit_descale():
         assert ds[0, 0] == 1.0 and np.all(codes == 0)
 
 
+def _f32_factor(ss, eps):
+    """r = 1 / sqrt(ss / 128 + eps) with each fp32 step rounded (numpy float32
+    arithmetic and sqrt are IEEE correctly rounded)."""
+    mean = np.float32(ss) * np.float32(1.0 / 128)
+    return np.float32(1.0) / np.sqrt(np.float32(mean + np.float32(eps)))
+
+
 def test_rmsnorm_closed_form_one_spike_per_row():
-    # a row whose only nonzero value is a has y = a / sqrt(a^2 / 128 + eps) there
+    # a row whose only nonzero value is a has the exact sum of squares a^2, so
+    # y = a / sqrt(a^2 / 128 + eps) there, in fp32 steps
     a_vals = [0.5, -1.0, 2.0, 3.0, -0.75, 1.5]
     x = torch.zeros(1, 1, len(a_vals), 128)
     for i, a in enumerate(a_vals):
         x[0, 0, i, (7 * i) % 128] = a
     eps = 1e-6
     codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=eps)
-    y = [np.float32(a / math.sqrt(a * a / 128 + eps)) for a in a_vals]
+    y = [np.float32(a) * _f32_factor(a * a, eps) for a in a_vals]
     amax = max(abs(v) for v in y)
     assert ds[0, 0] == np.float32(amax) / np.float32(448)
     for i, v in enumerate(y):
@@ -96,9 +104,28 @@ def test_rmsnorm_closed_form_constant_rows():
     x = torch.full((1, 2, 4, 128), 0.75)
     x[0, 1] = -2.0
     codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=1e-6)
-    y0 = np.float32(0.75 / math.sqrt(0.75 ** 2 + 1e-6))
+    y0 = np.float32(0.75) * _f32_factor(128 * 0.75 ** 2, 1e-6)   # 128 a^2 is exact in fp32
     assert ds[0, 0] == y0 / np.float32(448)
     assert np.all(codes[0, 0] == 0x7E) and np.all(codes[0, 1] == 0xFE)
+
+
+def test_rmsnorm_exact_sum_in_any_order():
+    # squares that are distinct powers of two spread over the row sum exactly in
+    # fp32, whatever the order: the factor is the closed form of that sum
+    x = torch.zeros(1, 1, 3, 128)
+    for d in range(0, 128, 8):
+        x[0, 0, 0, d] = 2.0 ** (d // 8 - 8)            # squares 2^-16 .. 2^14, each once
+    x[0, 0, 1, 5] = 1.0
+    x[0, 0, 1, 77] = -4.0                              # 1 + 16
+    x[0, 0, 2, :] = torch.tensor([(-1.0) ** d * 0.5 for d in range(128)])   # 128 / 4
+    sums = [sum(4.0 ** (k - 8) for k in range(16)), 17.0, 32.0]
+    codes, ds = oracle.quantize_e4m3(_bits(x), rmsnorm=True, eps=1e-6)
+    ys = [x[0, 0, i].numpy().astype(np.float32) * _f32_factor(sums[i], 1e-6) for i in range(3)]
+    amax = max(float(np.abs(y).max()) for y in ys)
+    assert ds[0, 0] == np.float32(amax) / np.float32(448)
+    for i in range(3):
+        want = [oracle.e4m3_rne(np.float32(v) / ds[0, 0]) for v in ys[i]]
+        assert list(codes[0, 0, i]) == want
 
 
 def test_rmsnorm_removes_power_of_two_scales_exactly():
