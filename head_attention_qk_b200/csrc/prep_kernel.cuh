@@ -106,17 +106,20 @@ __global__ void prep_descale_kernel(float* __restrict__ d, int n) {
   }
 }
 
-// y / ds rounded to fp32.  Fast path: y times a reciprocal, within 2 ulp of
-// the quotient; that can only change the e4m3 rounding when the result lies
-// within a few ulp of a midpoint between two e4m3 values (its low 20 mantissa
-// bits near 0x80000) or in the small range where e4m3 steps are subnormal, and
-// there the exactly rounded quotient is taken instead.
-__device__ __forceinline__ float prep_quotient(float y, float ds, float rcp) {
-  const float q = y * rcp;
-  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
-  const int low = (int)(b & 0xFFFFFu) - 0x80000;
-  if (b < 0x3D000000u /* 2^-5 */ || (low >= -4 && low <= 4)) return __fdiv_rn(y, ds);
-  return q;
+// y / ds rounded to fp32, for a pair (rcp = 1/ds correctly rounded, ds >= 2^-60
+// so that no residual below is subnormal).  q0 = y * rcp is within an ulp of
+// the quotient; with the exact residual r = y - q0 ds (one fused multiply-add)
+// the correction q0 + r * rcp is the correctly rounded quotient (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990).  Below 2^-11 the correction is skipped: every value
+// there, exact or not, takes the e4m3 code of a signed zero (the smallest
+// e4m3 step is 2^-9), and the sign is the quotient's either way.
+__device__ __forceinline__ float2 prep_quotient2(float2 y, float ds, float rcp) {
+  const float2 r2 = make_float2(rcp, rcp);
+  const float2 q0 = __fmul2_rn(y, r2);
+  const float2 res = __ffma2_rn(q0, make_float2(-ds, -ds), y);
+  const float2 q = __ffma2_rn(res, r2, q0);
+  return make_float2(fabsf(q0.x) < 0x1p-11f ? q0.x : q.x, fabsf(q0.y) < 0x1p-11f ? q0.y : q.y);
 }
 
 __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
@@ -143,6 +146,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint1
   }
   const float ds = __ldg(&descale[bh]);
   const float rcp = __frcp_rn(ds);
+  const bool tiny_ds = ds < 0x1p-60f;    // a head of tiny values: exact division throughout
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const PrepVals p = prep_unpack(w[k]);
@@ -150,9 +154,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint1
     uint16_t c[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const float y0 = rmsnorm ? __fmul_rn(p.v[2 * t], r) : p.v[2 * t];
-      const float y1 = rmsnorm ? __fmul_rn(p.v[2 * t + 1], r) : p.v[2 * t + 1];
-      c[t] = e4m3x2_rn_satfinite(prep_quotient(y0, ds, rcp), prep_quotient(y1, ds, rcp));
+      float2 y = make_float2(p.v[2 * t], p.v[2 * t + 1]);
+      if (rmsnorm) y = __fmul2_rn(y, make_float2(r, r));
+      const float2 q = tiny_ds ? make_float2(__fdiv_rn(y.x, ds), __fdiv_rn(y.y, ds)) : prep_quotient2(y, ds, rcp);
+      c[t] = e4m3x2_rn_satfinite(q.x, q.y);
     }
     const int s = r0 + 16 * k;
     if (s < S)

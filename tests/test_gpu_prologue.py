@@ -55,12 +55,14 @@ def test_prologue_special_rows(h):
 
 def test_prologue_extreme_magnitudes(h):
     # squares that underflow to fp32 subnormals (2^-70 scale), large rows (2^60),
-    # and a mix inside one row: every fp32 step of the norm is IEEE on both sides
+    # a mix inside one row, and a head whose descale is tiny: every fp32 step of
+    # the norm and of the quotient is IEEE on both sides
     g = torch.Generator().manual_seed(31)
-    x = torch.randn(1, 2, 48, 128, generator=g)
+    x = torch.randn(1, 3, 48, 128, generator=g)
     x[0, 0, :16] *= 2.0 ** -70
     x[0, 0, 16:32] *= 2.0 ** 60
     x[0, 1, :, ::3] *= 2.0 ** -64
+    x[0, 2] *= 2.0 ** -80                           # a whole head of tiny values: tiny descale
     for rms in (False, True):
         check_exact(h, x.to(torch.bfloat16), rms)
 
