@@ -236,7 +236,7 @@ class Step:
                          torch.empty(t.shape[:2], dtype=torch.float32, device="cuda")) for t in self.src]
             self.flops = 0.0
             self.bytes = sum(5.0 * t.numel() for t in self.src)   # x read twice, codes written once
-            self.launches = 12                                      # 3 x (memset + 3 kernels)
+            self.launches = 6                                       # 3 x 2 kernels (and a memset each)
             self.dtype = "e4m3"
         elif name == "streaming":
             x = make_kvblock_inputs(w)

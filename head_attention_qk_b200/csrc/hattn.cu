@@ -312,7 +312,6 @@ int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H,
   if (cudaMemsetAsync(descale, 0, (size_t)bh * sizeof(float), st) != cudaSuccess) return HATTN_ELAUNCH;
   prep_amax_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
                                                    reinterpret_cast<unsigned int*>(descale), S, rmsnorm ? 1 : 0, eps32);
-  prep_descale_kernel<<<(bh + 255) / 256, 256, 0, st>>>(descale, bh);
   prep_quantize_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
                                                        reinterpret_cast<uint8_t*>(codes), descale, S,
                                                        rmsnorm ? 1 : 0, eps32);

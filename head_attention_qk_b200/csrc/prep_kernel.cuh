@@ -17,10 +17,10 @@
 //             saturating at +-448
 // Every step is fixed in precision and order, so the codes and descales are a
 // function of the input alone: bit for bit the same for any grid, batch or
-// head split.  Three launches (after a memset of the descale array): the head
-// maxima (atomicMax on the non-negative fp32 bit patterns, which order like
-// integers, so the result does not depend on the order), max -> descale in
-// place, and the codes.  HBM-bound: x is read twice and the codes written once;
+// head split.  Two launches (after a memset of the descale array): the head
+// maxima (atomicMax on fp32 bit patterns, which order like integers, so the
+// result does not depend on the order) and the codes, which also turn each
+// head's maximum into its descale.  HBM-bound: x is read twice and the codes written once;
 // 16 threads share a row, so a warp reads two whole rows (512 contiguous
 // bytes) per load and writes two rows of codes (256 bytes) per store.
 #pragma once
@@ -62,7 +62,10 @@ __device__ __forceinline__ float prep_row_factor(const PrepVals& p, int rmsnorm,
   return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fmul_rn(s, 0.0078125f), eps)));
 }
 
-// grid (ceil(S / 64), B*H): the largest |y| of each head into amax_bits (zeroed).
+// grid (ceil(S / 64), B*H): the largest |y| of each head, stored negated into
+// amax_bits (zeroed): the bit patterns of non-positive floats order like
+// unsigned integers by magnitude, so atomicMax keeps the largest, and the
+// sign bit tells this value apart from a finished descale.
 __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
                                                                    unsigned int* __restrict__ amax_bits, int S,
                                                                    int rmsnorm, float eps) {
@@ -93,17 +96,16 @@ __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t*
     float bm = wmax[0];
 #pragma unroll
     for (int i = 1; i < kPrepThreads / 32; ++i) bm = fmaxf(bm, wmax[i]);
-    atomicMax(&amax_bits[bh], __float_as_uint(bm));
+    atomicMax(&amax_bits[bh], __float_as_uint(-bm));
   }
 }
 
-// In place: descale = amax / 448 (1 when amax == 0).
-__global__ void prep_descale_kernel(float* __restrict__ d, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) {
-    const float amax = d[i];
-    d[i] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  }
+// descale of a head from its slot: either -amax (sign bit set, as the maxima
+// kernel left it) or the descale already written there; both give the same.
+__device__ __forceinline__ float prep_descale_of(float slot) {
+  if (!signbit(slot)) return slot;
+  const float amax = -slot;
+  return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
 // y / ds rounded to fp32, for a pair (rcp = 1/ds correctly rounded, ds >= 2^-60
@@ -128,14 +130,17 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   return r;
 }
 
-// grid (ceil(S / 64), B*H): the codes of each row.
+// grid (ceil(S / 64), B*H): the codes of each row, and the descale of each
+// head in place of its maximum.  CTAs walk the rows in the reverse of the
+// maxima kernel's order, so the rows it read last, still in L2, come first.
 __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
                                                                        uint8_t* __restrict__ codes,
-                                                                       const float* __restrict__ descale, int S,
+                                                                       float* __restrict__ descale, int S,
                                                                        int rmsnorm, float eps) {
-  const int bh = blockIdx.y;
+  const int bh = gridDim.y - 1 - blockIdx.y;
+  const int tile = gridDim.x - 1 - blockIdx.x;
   const int sub = threadIdx.x & 15;
-  const int r0 = blockIdx.x * kPrepRowsPerCta + (threadIdx.x >> 4);
+  const int r0 = tile * kPrepRowsPerCta + (threadIdx.x >> 4);
   const uint4* base = reinterpret_cast<const uint4*>(x) + (long long)bh * S * 16 + sub;
   uint2* dst = reinterpret_cast<uint2*>(codes) + (long long)bh * S * 16 + sub;
   uint4 w[4];
@@ -144,7 +149,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint1
     const int s = r0 + 16 * k;
     w[k] = s < S ? __ldg(base + (long long)s * 16) : make_uint4(0u, 0u, 0u, 0u);
   }
-  const float ds = __ldg(&descale[bh]);
+  const float ds = prep_descale_of(*reinterpret_cast<volatile float*>(&descale[bh]));
+  if (tile == 0 && threadIdx.x == 0) descale[bh] = ds;   // the other CTAs read either form
   const float rcp = __frcp_rn(ds);
   const bool tiny_ds = ds < 0x1p-60f;    // a head of tiny values: exact division throughout
 #pragma unroll

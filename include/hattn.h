@@ -115,8 +115,11 @@ HATTN_API size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtyp
  * descale = max |y| / 448 (fp32; 1 if the head is
  * all zero), code = y / descale (fp32 quotient) rounded to the nearest e4m3fn
  * value, ties to even, saturating at +-448.  The result is bitwise the same for
- * any batch or head split.  Enqueues a memset of descale and three kernels;
- * HBM traffic 5 bytes per element (x read twice, codes written once).
+ * any batch or head split.  Enqueues a memset of descale and two kernels
+ * (head maxima; codes, which also turn each maximum into its descale); x is
+ * read twice (the second pass starts with the rows read last, which L2 may
+ * still hold) and the codes are written once: at most 5 bytes of HBM traffic
+ * per element.
  */
 HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H, int S, int D,
                                  int rmsnorm, double eps, void* stream);
