@@ -14,8 +14,9 @@
 //                     tiles (ascending).  Per step, four tcgen05 MMAs:
 //                       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q
 //                     (S^T of the next step and dV in two query halves).
-//   bwd_dq_kernel     one CTA per (b, q head, 128-row query tile); loops over
-//                     KV tiles (ascending).  Per step, three MMAs:
+//   bwd_dq_kernel     persistent, one CTA per SM; each (b, q head, 128-row query
+//                     tile) unit loops over KV tiles (ascending).  Per step,
+//                     three MMAs:
 //                       S = Q K^T, dP = dO V^T, dQ += dS K.
 //
 // Roles: warps 0-7 compute, warp 8 TMA producer, warp 9 MMA issuer and
@@ -490,30 +491,55 @@ struct DqSmem {
   static constexpr int kK = kDO + kTileBytesBf16;
   static constexpr int kV = kK + kKStages * kTileBytesBf16;
   static constexpr int kBars = kV + kVStages * kTileBytesBf16;
-  static constexpr int kBytes = kBars + 18 * 8;
+  static constexpr int kBytes = kBars + 20 * 8;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
+// One unit of dQ work: query tile i of head bh (KV head bkv), n_kv KV tiles.
+struct DqUnit {
+  int i, bh, bkv, n_kv;
+};
+
+// Unit t of the work list, heaviest first: query-tile rank t / (B*Hq), counted
+// from the last tile under a causal mask (the last tiles see the most keys).
+__device__ __forceinline__ DqUnit dq_unit(const BwdArgs& a, int t) {
+  const int BH = a.B * a.Hq;
+  const int nq = (a.Sq + kTile - 1) / kTile;
+  const int rank = t / BH;
+  DqUnit u;
+  u.bh = t - rank * BH;
+  u.i = a.causal ? nq - 1 - rank : rank;
+  const int b = u.bh / a.Hq, h = u.bh - b * a.Hq;
+  u.bkv = b * a.Hkv + h / (a.Hq / a.Hkv);
+  if (!a.causal) {
+    u.n_kv = (a.Sk + kTile - 1) / kTile;
+  } else {
+    const int last_row = min(u.i * kTile + kTile - 1, a.Sq - 1);
+    u.n_kv = min(last_row + (a.Sk - a.Sq), a.Sk - 1) / kTile + 1;
+  }
+  return u;
+}
+
+// The k-th unit of CTA c among G persistent CTAs: the heaviest-first list is
+// dealt out in snake order (c, then 2G-1-c, then 2G+c, ...), which evens out
+// the causal unit sizes.  Increasing in k, so the first index past the list
+// ends the CTA's loop.
+__device__ __forceinline__ int dq_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
+
+// Persistent: one CTA per SM walks its units.  Every unit's dQ rows are summed
+// over its KV tiles in ascending order by one CTA, as before; only which CTA
+// does a unit depends on the grid.  Across units the K/V ring, the S buffers
+// and every barrier phase continue with a global step count, so the next
+// unit's Q/dO load (once the last S and dP of a unit have read them) and its
+// first S and dP overlap the end of the current unit and its dQ epilogue.
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
   using L = DqSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
-
-  const int nq = (a.Sq + kTile - 1) / kTile;
-  const int i = a.causal ? nq - 1 - (int)blockIdx.x : (int)blockIdx.x;   // heaviest first under a mask
-  const int bh = blockIdx.y;
-  const int b = bh / a.Hq, h = bh - b * a.Hq;
-  const int G = a.Hq / a.Hkv;
-  const int bkv = b * a.Hkv + h / G;
-  int n_kv;
-  if (!a.causal) {
-    n_kv = (a.Sk + kTile - 1) / kTile;
-  } else {
-    const int last_row = min(i * kTile + kTile - 1, a.Sq - 1);
-    n_kv = min(last_row + (a.Sk - a.Sq), a.Sk - 1) / kTile + 1;
-  }
+  const int n_units = ((a.Sq + kTile - 1) / kTile) * a.B * a.Hq;
+  const int cta = blockIdx.x, n_cta = gridDim.x;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
@@ -524,8 +550,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   uint64_t* s_full = bars + 11;   // [2 S buffers]
   uint64_t* dp_full = bars + 13;
   uint64_t* ds_full = bars + 14;
-  uint64_t* dq_done = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* dq_done = bars + 15;  // a unit's dQ MMAs have completed
+  uint64_t* q_empty = bars + 16;  // a unit's last S and dP have read Q and dO
+  uint64_t* mma_drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -536,6 +564,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     mbar_init(dp_full, 1);
     mbar_init(ds_full, kBwdComputeWarps);  // one arrival per compute warp
     mbar_init(dq_done, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(mma_drain, 1);
     fence_barrier_init();
   }
   if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
@@ -544,137 +574,179 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S / dS buffer 0 [0,128), dP [128,256), dQ [256,384), S / dS buffer 1 [384,512)
-  auto s_col = [](int jj) { return (jj & 1) ? 384u : 0u; };
+  auto s_col = [](int g) { return (g & 1) ? 384u : 0u; };
 
   if (warp == 8) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * kTileBytesBf16);
-      tma_tile_bf16(smem + L::kQ, &a.tm_q, q_full, i * kTile, bh);
-      tma_tile_bf16(smem + L::kDO, &a.tm_do, q_full, i * kTile, bh);
       bool ok = true;
-      for (int jj = 0; jj < n_kv && ok; ++jj) {
-        const int ks = jj % L::kKStages, ku = jj / L::kKStages;
-        if (jj >= L::kKStages) ok = mbar_wait(&k_empty[ks], (ku - 1) & 1, kSiteBwdStEmpty);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&k_full[ks], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kK + ks * kTileBytesBf16, &a.tm_k, &k_full[ks], jj * kTile, bkv);
-        const int vs = jj % L::kVStages, vu = jj / L::kVStages;
-        if (jj >= L::kVStages) ok = mbar_wait(&v_empty[vs], (vu - 1) & 1, kSiteBwdStEmpty);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&v_full[vs], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kV + vs * kTileBytesBf16, &a.tm_v, &v_full[vs], jj * kTile, bkv);
+      int ul = 0, gk = 0, gv = 0;   // units started, K and V tiles requested
+      for (int k = 0; ok; ++k) {
+        const int t = dq_unit_index(k, cta, n_cta);
+        if (t >= n_units) break;
+        const DqUnit u = dq_unit(a, t);
+        // K_0 and V_0 go first: their ring stages free up while the previous
+        // unit still runs, before its last S and dP release Q and dO
+        for (int jj = 0; jj < u.n_kv && ok; ++jj) {
+          if (jj == 1 || u.n_kv == 1) {
+            if (ul > 0) ok = mbar_wait(q_empty, (ul - 1) & 1, kSiteBwdStEmpty);
+            if (!ok) break;
+            mbar_arrive_expect_tx(q_full, 2 * kTileBytesBf16);
+            tma_tile_bf16(smem + L::kQ, &a.tm_q, q_full, u.i * kTile, u.bh);
+            tma_tile_bf16(smem + L::kDO, &a.tm_do, q_full, u.i * kTile, u.bh);
+            ++ul;
+          }
+          const int ks = gk % L::kKStages, ku = gk / L::kKStages;
+          if (gk >= L::kKStages) ok = mbar_wait(&k_empty[ks], (ku - 1) & 1, kSiteBwdStEmpty);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&k_full[ks], kTileBytesBf16);
+          tma_tile_bf16(smem + L::kK + ks * kTileBytesBf16, &a.tm_k, &k_full[ks], jj * kTile, u.bkv);
+          ++gk;
+          const int vs = gv % L::kVStages, vu = gv / L::kVStages;
+          if (gv >= L::kVStages) ok = mbar_wait(&v_empty[vs], (vu - 1) & 1, kSiteBwdStEmpty);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&v_full[vs], kTileBytesBf16);
+          tma_tile_bf16(smem + L::kV + vs * kTileBytesBf16, &a.tm_v, &v_full[vs], jj * kTile, u.bkv);
+          ++gv;
+        }
       }
       // drain: every load issued must land before the CTA exits
-      mbar_wait_drain(q_full, 0, kSiteBwdKV);
-      for (int jj = max(0, n_kv - L::kKStages); jj < n_kv; ++jj)
-        mbar_wait_drain(&k_full[jj % L::kKStages], (jj / L::kKStages) & 1, kSiteBwdStFull);
-      for (int jj = max(0, n_kv - L::kVStages); jj < n_kv; ++jj)
-        mbar_wait_drain(&v_full[jj % L::kVStages], (jj / L::kVStages) & 1, kSiteBwdStFull);
+      if (ul > 0) mbar_wait_drain(q_full, (ul - 1) & 1, kSiteBwdKV);
+      for (int g = max(0, gk - L::kKStages); g < gk; ++g)
+        mbar_wait_drain(&k_full[g % L::kKStages], (g / L::kKStages) & 1, kSiteBwdStFull);
+      for (int g = max(0, gv - L::kVStages); g < gv; ++g)
+        mbar_wait_drain(&v_full[g % L::kVStages], (g / L::kVStages) & 1, kSiteBwdStFull);
     }
     __syncwarp();
   } else if (warp == 9) {
     if (lane == 0) {
       const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-      auto sK_of = [&](int jj) { return smem_u32(smem + L::kK + (jj % L::kKStages) * kTileBytesBf16); };
-      auto sV_of = [&](int jj) { return smem_u32(smem + L::kV + (jj % L::kVStages) * kTileBytesBf16); };
+      auto sK_of = [&](int g) { return smem_u32(smem + L::kK + (g % L::kKStages) * kTileBytesBf16); };
+      auto sV_of = [&](int g) { return smem_u32(smem + L::kV + (g % L::kVStages) * kTileBytesBf16); };
       // S is double-buffered in TMEM: S_{j+1} is computed while the compute
-      // warps work on step j.  Issue order: S_0, dP_0, S_1, then per step j:
-      // dQ_j (once dS_j is written), dP_{j+1} (the compute warps have read dP_j),
-      // S_{j+2} into the buffer dQ_j has just read dS_j from.
-      auto issue_s = [&](int jj) -> bool {
-        if (!mbar_wait(&k_full[jj % L::kKStages], (jj / L::kKStages) & 1, kSiteBwdStFull)) return false;
+      // warps work on step j.  Issue order per unit: S_0, dP_0, S_1, then per
+      // step j: dQ_j (once dS_j is written), dP_{j+1} (the compute warps have
+      // read dP_j), S_{j+2} into the buffer dQ_j has just read dS_j from.  g
+      // counts steps over all of this CTA's units.
+      auto issue_s = [&](int g) -> bool {
+        if (!mbar_wait(&k_full[g % L::kKStages], (g / L::kKStages) & 1, kSiteBwdStFull)) return false;
         tc_fence_after();
-        mma_tile_ss_kmajor(tmem + s_col(jj), sQ, sK_of(jj), 0);         // S  = Q K^T
-        mma_commit(&s_full[jj & 1]);
+        mma_tile_ss_kmajor(tmem + s_col(g), sQ, sK_of(g), 0);           // S  = Q K^T
+        mma_commit(&s_full[g & 1]);
         return true;
       };
-      auto issue_dp = [&](int jj) -> bool {
-        if (!mbar_wait(&v_full[jj % L::kVStages], (jj / L::kVStages) & 1, kSiteBwdStFull)) return false;
+      auto issue_dp = [&](int g) -> bool {
+        if (!mbar_wait(&v_full[g % L::kVStages], (g / L::kVStages) & 1, kSiteBwdStFull)) return false;
         tc_fence_after();
-        mma_tile_ss_kmajor(tmem + 128, sDO, sV_of(jj), 0);              // dP = dO V^T
+        mma_tile_ss_kmajor(tmem + 128, sDO, sV_of(g), 0);               // dP = dO V^T
         mma_commit(dp_full);
-        mma_commit(&v_empty[jj % L::kVStages]);
+        mma_commit(&v_empty[g % L::kVStages]);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, kSiteBwdKV);
-      if (ok && n_kv > 0) ok = issue_s(0) && issue_dp(0);
-      if (ok && n_kv > 1) ok = issue_s(1);
-      for (int jj = 0; jj < n_kv && ok; ++jj) {
-        ok = mbar_wait(ds_full, jj & 1, kSiteBwdP);
+      bool ok = true;
+      int ul = 0, g0 = 0;
+      for (int k = 0; ok; ++k) {
+        const int t = dq_unit_index(k, cta, n_cta);
+        if (t >= n_units) break;
+        const int n = dq_unit(a, t).n_kv;
+        ok = mbar_wait(q_full, ul & 1, kSiteBwdKV);
+        if (ok) ok = issue_s(g0) && issue_dp(g0);
+        if (ok && n == 1) mma_commit(q_empty);                           // Q and dO read for the last time
+        if (ok && n > 1) ok = issue_s(g0 + 1);
+        for (int jj = 0; jj < n && ok; ++jj) {
+          const int g = g0 + jj;
+          ok = mbar_wait(ds_full, g & 1, kSiteBwdP);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ts_mnmajor_halves(tmem + 256, tmem + s_col(g), sK_of(g), jj > 0);   // dQ += dS K
+          mma_commit(&k_empty[g % L::kKStages]);
+          if (jj + 1 < n) {
+            ok = issue_dp(g + 1);
+            if (ok && jj + 1 == n - 1) mma_commit(q_empty);
+          }
+          if (ok && jj + 2 < n) ok = issue_s(g + 2);
+        }
         if (!ok) break;
-        tc_fence_after();
-        mma_tile_ts_mnmajor_halves(tmem + 256, tmem + s_col(jj), sK_of(jj), jj > 0);   // dQ += dS K
-        mma_commit(&k_empty[jj % L::kKStages]);
-        if (jj + 1 < n_kv) ok = issue_dp(jj + 1);
-        if (ok && jj + 2 < n_kv) ok = issue_s(jj + 2);
+        mma_commit(dq_done);
+        g0 += n;
+        ++ul;
       }
-      mma_commit(dq_done);
-      mbar_wait(dq_done, 0, kSiteBwdDone);
+      mma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0, kSiteBwdDone);
     }
     __syncwarp();
   } else {
     const int r = (warp & 3) * 32 + lane;            // query row within the tile
     const int hc = warp >> 2;                        // column half: keys 64 hc .. 64 hc + 63
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const int qi = i * kTile + r;
-    const bool valid = qi < a.Sq;
-    const size_t ridx = (size_t)bh * a.Sq + (valid ? qi : 0);
-    const float lse2 = valid ? __ldg(&a.lse[ridx]) * 1.4426950408889634f : INFINITY;
-    const float dlt = valid ? __ldg(&a.delta[ridx]) : 0.f;
-    const int kv_limit = a.causal ? min(a.Sk - 1, qi + (a.Sk - a.Sq)) : a.Sk - 1;
     const float c = a.scale_log2;
     bool ok = true;
-    for (int jj = 0; jj < n_kv && ok; ++jj) {
-      ok = warp_wait(&s_full[jj & 1], (jj >> 1) & 1, kSiteBwdS);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tS = tmem + lane_base + s_col(jj) + hc * 64;   // this warp's 64 S (then dS) columns
-      float p[64];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t u[32];
-        tmem_ld32(tS + q * 32, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) p[q * 32 + e] = __uint_as_float(u[e]);
-      }
-      const int kbase = jj * kTile + hc * 64;
-      const bool need_mask = kbase + 63 > kv_limit;
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        float x = ex2_approx(fmaf(p[e], c, -lse2));
-        if (need_mask && kbase + e > kv_limit) x = 0.f;
-        p[e] = x;
-      }
-      __syncwarp();
-      ok = warp_wait(dp_full, jj & 1, kSiteBwdDP);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        uint32_t uu[32];
+    int ul = 0, g0 = 0;
+    for (int k = 0; ok; ++k) {
+      const int t = dq_unit_index(k, cta, n_cta);
+      if (t >= n_units) break;
+      const DqUnit u = dq_unit(a, t);
+      const int qi = u.i * kTile + r;
+      const bool valid = qi < a.Sq;
+      const size_t ridx = (size_t)u.bh * a.Sq + (valid ? qi : 0);
+      const float lse2 = valid ? __ldg(&a.lse[ridx]) * 1.4426950408889634f : INFINITY;
+      const float dlt = valid ? __ldg(&a.delta[ridx]) : 0.f;
+      const int kv_limit = a.causal ? min(a.Sk - 1, qi + (a.Sk - a.Sq)) : a.Sk - 1;
+      for (int jj = 0; jj < u.n_kv && ok; ++jj) {
+        const int g = g0 + jj;
+        ok = warp_wait(&s_full[g & 1], (g >> 1) & 1, kSiteBwdS);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = tmem + lane_base + s_col(g) + hc * 64;   // this warp's 64 S (then dS) columns
+        float p[64];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          tmem_ld32(tmem + lane_base + 128 + hc * 64 + q * 32, uu);
+          uint32_t uu[32];
+          tmem_ld32(tS + q * 32, uu);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
+          for (int e = 0; e < 32; ++e) p[q * 32 + e] = __uint_as_float(uu[e]);
         }
-      }
-      {
-        uint32_t w[32];
+        const int kbase = jj * kTile + hc * 64;
+        const bool need_mask = kbase + 63 > kv_limit;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-        tmem_st32(tS, w);                            // dS over the first 32 of these columns
+        for (int e = 0; e < 64; ++e) {
+          float x = ex2_approx(fmaf(p[e], c, -lse2));
+          if (need_mask && kbase + e > kv_limit) x = 0.f;
+          p[e] = x;
+        }
+        __syncwarp();
+        ok = warp_wait(dp_full, g & 1, kSiteBwdDP);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          uint32_t uu[32];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            tmem_ld32(tmem + lane_base + 128 + hc * 64 + q * 32, uu);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
+          }
+        }
+        {
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+          tmem_st32(tS, w);                          // dS over the first 32 of these columns
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    if (ok) ok = warp_wait(dq_done, 0, kSiteBwdDone);
-    if (ok) {
+      if (ok) ok = warp_wait(dq_done, ul & 1, kSiteBwdDone);
+      if (!ok) break;
       tc_fence_after();
+      // The next unit's first dQ MMA overwrites these columns only after this
+      // warp's first dS of that unit, i.e. after these loads have completed.
       store_half_row_bf16(tmem + lane_base + 256 + hc * 64, a.scale, a.dq + ridx * kHeadDim + hc * 64, valid);
+      g0 += u.n_kv;
+      ++ul;
     }
   }
 
@@ -688,7 +760,7 @@ bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uin
 
 inline int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
-                      float scale, bool causal, float* delta, cudaStream_t st) {
+                      float scale, bool causal, float* delta, int n_sm, cudaStream_t st) {
   static bool attr_ok = [] {
     return cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvSmem::kAlloc) ==
                cudaSuccess &&
@@ -715,7 +787,9 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   bwd_delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(reinterpret_cast<const uint16_t*>(out),
                                                                 reinterpret_cast<const uint16_t*>(dout), delta, rows);
   bwd_dkdv_kernel<<<dim3(B * Hkv, (Sk + kTile - 1) / kTile), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
-  bwd_dq_kernel<<<dim3((Sq + kTile - 1) / kTile, B * Hq), kBwdThreads, DqSmem::kAlloc, st>>>(a);
+  const long long dq_units = (long long)((Sq + kTile - 1) / kTile) * B * Hq;
+  const int dq_grid = (int)std::min<long long>(dq_units, n_sm);
+  bwd_dq_kernel<<<dq_grid, kBwdThreads, DqSmem::kAlloc, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 

@@ -422,8 +422,10 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   for (const void* p : ptrs)
     if (!aligned16(p)) return HATTN_EALIGN;
   if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq)) return HATTN_EWORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HATTN_EDEVICE;
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
-                    reinterpret_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+                    reinterpret_cast<float*>(workspace), sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- allocation-free backward
@@ -471,7 +473,9 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   if (!delta) return HATTN_ELAUNCH;
   // Delta is fully rewritten for every row this call reads, so the array needs
   // no clearing between calls.
-  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta,
+  const int sms = device_sm_count();
+  if (sms <= 0) return HATTN_EDEVICE;
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta, sms,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
