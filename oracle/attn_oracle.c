@@ -8,7 +8,9 @@
  * head_attention_qk_b200/csrc, and it never includes or links it.
  *
  * Everything is computed in double precision with plain loops (no blocking, no
- * fusion, no reordering beyond the definition).  OpenMP splits independent
+ * fusion, no reordering beyond the definition), except the e4m3 prologue's
+ * RMS norm, which takes the kernel's fp32 steps in a stated order because its
+ * values decide integer codes (see oracle_quantize_e4m3).  OpenMP splits independent
  * (batch, head, query-row) units across host threads; each unit is summed in a
  * fixed ascending order, so results do not depend on the thread count.
  *
