@@ -50,6 +50,10 @@ def check(h, w):
     (2, 4, 2, 300, 300, True),
     (1, 2, 2, 129, 1100, True),
     (1, 4, 1, 513, 257, False),
+    # more query-tile units than SMs, ragged tails: the persistent dQ CTAs each
+    # take several units of different lengths
+    (1, 24, 3, 1000, 1000, True),
+    (2, 12, 4, 1100, 700, False),
 ])
 def test_bwd_ragged(h, B, Hq, Hkv, Sq, Sk, causal):
     check(h, Workload("bw", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, seed=200 + Sq + Sk, backward=True))
