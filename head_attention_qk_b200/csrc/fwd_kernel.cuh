@@ -175,6 +175,18 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdArgs& a, int u) {
   return w;
 }
 
+// The units of one CTA.  Persistent: the (heaviest-first) unit list is dealt
+// out in snake order, unit k of CTA c being k G + c for even k and
+// k G + G - 1 - c for odd k (G = gridDim.x), which evens out unequal causal
+// units; increasing in k, so the loop ends at the first index past the list.
+// One unit per CTA: blockIdx.x, then past it.
+template <bool kPersist>
+__device__ __forceinline__ int fwd_unit_index(int k) {
+  if (!kPersist) return (int)blockIdx.x + k;
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * G + ((k & 1) ? G - 1 - c : c);
+}
+
 // Unit loop condition.  Persistent launches loop while units remain; a
 // one-unit-per-CTA launch runs the body exactly once (the compiler sees a single
 // iteration, so the per-tile code is the same as a kernel without the loop).
@@ -191,9 +203,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
   const int warp = warp_id();
   const int lane = lane_id();
-  // Persistent: this CTA takes units blockIdx.x, blockIdx.x + gridDim.x, ...
-  // otherwise the grid holds one CTA per unit.
-  const int u_first = blockIdx.x, u_step = kPersist ? (int)gridDim.x : 1, u_end = args.total_units;
+  // Persistent: this CTA takes units fwd_unit_index(0), (1), ...; otherwise
+  // the grid holds one CTA per unit.
+  const int u_first = blockIdx.x, u_end = args.total_units;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   FwdBars bb;
@@ -257,7 +269,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       int slot = 0, units = 0;
       uint32_t ph = 0;
       long long nseq = 0;                                  // K/V tiles loaded by this CTA
-      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u = fwd_unit_index<kPersist>(++units)) {
         const FwdUnit w = fwd_unit(args, u);
         // K/V tile j of the unit: tile lt of block b (fused blocks run in order)
         int b = w.blk, lt = 0, nt = fwd_block_tiles(args.sk[b]);
@@ -353,7 +365,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       bool ok = true;
       int kslot = 0, units = 0;
       uint32_t kph = 0, jg = 0;
-      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+      for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u = fwd_unit_index<kPersist>(++units)) {
         const FwdUnit w = fwd_unit(args, u);
         const int n_kv = w.n_kv;
         ok = mbar_wait(bb.q_full, units & 1, kSiteQFull);
@@ -418,7 +430,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     bool ok = true;
     uint32_t jg = 0;                                  // this CTA's tile count
     int units = 0;
-    for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u += u_step, ++units) {
+    for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u = fwd_unit_index<kPersist>(++units)) {
       const FwdUnit w = fwd_unit(args, u);
       const int n_kv = w.n_kv, sk = w.sk, bh = w.bh;
       const int row = w.q_row0 + tile * kBlockM + r;

@@ -95,11 +95,13 @@ int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
-// Units of 256 query rows x one KV block.  Short units (few KV tiles, no mask)
-// go to the persistent kernel, one CTA per SM, which overlaps each unit's
-// epilogue and the next unit's Q load with the running MMAs; long or causal
-// units go one CTA per unit, ordered heaviest first, and the hardware
-// scheduler balances them.
+// Units of 256 query rows x one KV block.  Short units (on average at most 8
+// KV tiles: up to 8 without a mask, up to 16 under a causal mask, whose units
+// average half the longest) go to the persistent kernel, one CTA per SM, which
+// overlaps each unit's epilogue and the next unit's Q load with the running
+// MMAs and deals the heaviest-first unit list out in snake order; long units
+// go one CTA per unit, ordered heaviest first, and the hardware scheduler
+// balances them.
 constexpr int kPersistMaxKvTiles = 8;
 
 template <bool kFp8, bool kPartial>
@@ -110,7 +112,8 @@ int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, int max_sk, cudaStream_
   if (sms <= 0) return HATTN_EDEVICE;
   FwdArgs args = a;
   args.total_units = (int)units;
-  const bool persist = !a.causal && (max_sk + kBlockN - 1) / kBlockN <= kPersistMaxKvTiles && units > sms;
+  const int max_tiles = (max_sk + kBlockN - 1) / kBlockN;
+  const bool persist = max_tiles <= (a.causal ? 2 : 1) * kPersistMaxKvTiles && units > sms;
   if (persist) return launch_fwd_grid<kFp8, kPartial, true>(args, sms, st);
   return launch_fwd_grid<kFp8, kPartial, false>(args, (int)units, st);
 }
