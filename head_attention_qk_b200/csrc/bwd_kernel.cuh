@@ -61,19 +61,39 @@ enum : int {
 };
 
 // ---------------------------------------------------------------------------- Delta
+// Delta_r = sum_d dO_rd O_rd.  16 threads share a row (8 values each, one
+// 16-byte load of O and of dO), so a warp reads two whole rows per load; each
+// thread has four rows in flight.  The 16 partial sums meet by a xor
+// butterfly in a fixed order: the result does not depend on the grid.
+constexpr int kDeltaRowsPerCta = 64;
+
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                         float* __restrict__ delta, long long rows) {
-  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
-  const int lane = threadIdx.x & 31;
-  const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + r * kHeadDim) + lane);
-  const uint2 g = __ldg(reinterpret_cast<const uint2*>(dout + r * kHeadDim) + lane);
+  const int sub = threadIdx.x & 15;
+  const long long r0 = (long long)blockIdx.x * kDeltaRowsPerCta + (threadIdx.x >> 4);
+  const uint4* o4 = reinterpret_cast<const uint4*>(o) + sub;
+  const uint4* g4 = reinterpret_cast<const uint4*>(dout) + sub;
+  uint4 a[4], g[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const long long r = r0 + 16 * k;
+    const bool in = r < rows;
+    a[k] = in ? __ldg(o4 + r * 16) : make_uint4(0u, 0u, 0u, 0u);
+    g[k] = in ? __ldg(g4 + r * 16) : make_uint4(0u, 0u, 0u, 0u);
+  }
   auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
   auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
-  float s = lo(a.x) * lo(g.x) + hi(a.x) * hi(g.x) + lo(a.y) * lo(g.y) + hi(a.y) * hi(g.y);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) delta[r] = s;
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, gw[4] = {g[k].x, g[k].y, g[k].z, g[k].w};
+    float s = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) s += lo(aw[t]) * lo(gw[t]) + hi(aw[t]) * hi(gw[t]);
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    const long long r = r0 + 16 * k;
+    if (sub == 0 && r < rows) delta[r] = s;
+  }
 }
 
 // Shared helpers --------------------------------------------------------------
@@ -784,8 +804,8 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
   const long long rows = (long long)B * Hq * Sq;
-  bwd_delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(reinterpret_cast<const uint16_t*>(out),
-                                                                reinterpret_cast<const uint16_t*>(dout), delta, rows);
+  bwd_delta_kernel<<<(unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta), 256, 0, st>>>(
+      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows);
   bwd_dkdv_kernel<<<dim3(B * Hkv, (Sk + kTile - 1) / kTile), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
   const long long dq_units = (long long)((Sq + kTile - 1) / kTile) * B * Hq;
   const int dq_grid = (int)std::min<long long>(dq_units, n_sm);
