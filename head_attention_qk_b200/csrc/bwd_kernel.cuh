@@ -728,24 +728,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         }
         const int kbase = jj * kTile + hc * 64;
         const bool need_mask = kbase + 63 > kv_limit;
+        const float2 c2 = make_float2(c, c), nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          float x = ex2_approx(fmaf(p[e], c, -lse2));
-          if (need_mask && kbase + e > kv_limit) x = 0.f;
-          p[e] = x;
+        for (int e = 0; e < 64; e += 2) {
+          const float2 t = __ffma2_rn(make_float2(p[e], p[e + 1]), c2, nl2);
+          float x0 = ex2_approx(t.x), x1 = ex2_approx(t.y);
+          if (need_mask) {
+            x0 = kbase + e > kv_limit ? 0.f : x0;
+            x1 = kbase + e + 1 > kv_limit ? 0.f : x1;
+          }
+          p[e] = x0;
+          p[e + 1] = x1;
         }
         __syncwarp();
         ok = warp_wait(dp_full, g & 1, kSiteBwdDP);
         if (!ok) break;
         tc_fence_after();
         {
-          uint32_t uu[32];
+          uint32_t uu[64];
+          tmem_ld32(tmem + lane_base + 128 + hc * 64, *reinterpret_cast<uint32_t(*)[32]>(&uu[0]));
+          tmem_ld32(tmem + lane_base + 128 + hc * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&uu[32]));
+          tmem_wait_ld();
+          const float2 nd2 = make_float2(-dlt, -dlt);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            tmem_ld32(tmem + lane_base + 128 + hc * 64 + q * 32, uu);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) p[q * 32 + e] *= __uint_as_float(uu[e]) - dlt;
+          for (int e = 0; e < 64; e += 2) {
+            const float2 d = __fadd2_rn(make_float2(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1])), nd2);
+            const float2 r = __fmul2_rn(make_float2(p[e], p[e + 1]), d);
+            p[e] = r.x;
+            p[e + 1] = r.y;
           }
         }
         {
