@@ -54,3 +54,41 @@ def test_weak_scaling_aggregation_two_ranks():
     assert s0 == s1 == 2.5                          # max over ranks
     assert v0 == v1 == pytest.approx(2 * 1e12 * 10 / 2.5 / 1e12)
     assert g0 == g1 and g0[0] != g0[1]              # distinct units per rank
+
+
+def _cp_worker(rank, world, port, out):
+    import datetime
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from head_attention_qk_b200.context_parallel import gather_kv_shards
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r's shard holds the value 100 r + position, so the gathered order is visible
+        k = (torch.arange(2 * 3 * 5 * 4, dtype=torch.float32).view(2, 3, 5, 4) + 100 * rank)
+        v = -k
+        kg, vg = gather_kv_shards(k, v)
+        ok = kg.shape == (world, 2, 3, 5, 4) and all(
+            torch.equal(kg[r], k - 100 * rank + 100 * r) and torch.equal(vg[r], -kg[r]) for r in range(world))
+        # shards of different lengths are refused on every rank (no rank is left waiting)
+        k2 = torch.zeros(1, 1, 3 + rank, 4)
+        try:
+            gather_kv_shards(k2, k2)
+            refused = False
+        except ValueError:
+            refused = True
+        out[rank] = (ok, refused)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_gather_order_two_ranks():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    mp.start_processes(_cp_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert out[0] == (True, True) and out[1] == (True, True)
