@@ -83,6 +83,23 @@ def test_persistent_short_kv(h, B, Hq, Hkv, Sq, Sk):
     check_bf16(h, Workload("persist", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, seed=500 + Sq + Sk))
 
 
+def test_persistent_causal_ragged(h):
+    # causal with at most 16 KV tiles and more units than SMs: persistent, units
+    # of unequal length dealt in snake order; ragged tails, Sq < Sk, 5 query heads per KV head
+    check_bf16(h, Workload("persist_causal", B=2, Hq=40, Hkv=8, Sq=1000, Sk=1100, causal=True, seed=611))
+
+
+def test_persistent_causal_matches_one_cta_per_unit_bitwise(h):
+    # 320 units run persistently; one batch row of two heads (8 units) runs one CTA per unit
+    w = Workload("persist_causal_bits", B=2, Hq=40, Hkv=8, Sq=1000, Sk=1100, causal=True, seed=612)
+    x = cuda(make_fwd_inputs(w))
+    o, l = run_fwd(h, x, True)
+    xs = {"q": x["q"][1:, 5:7].contiguous(), "k": x["k"][1:, 1:2].contiguous(), "v": x["v"][1:, 1:2].contiguous()}
+    o2, l2 = run_fwd(h, xs, True)
+    assert torch.equal(o2.view(torch.int16), o[1:, 5:7].view(torch.int16))
+    assert torch.equal(l2, l[1:, 5:7])
+
+
 def test_persistent_matches_one_cta_per_unit_bitwise(h):
     # 280 units run persistently; three heads alone (21 units) run one CTA per unit
     w = Workload("persist_bits", B=1, Hq=40, Hkv=40, Sq=1560, Sk=512, seed=77)
