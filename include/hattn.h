@@ -149,7 +149,8 @@ HATTN_API int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, cons
                       const float* q_descale, const float* k_descale, const float* v_descale,
                       void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of workspace attn_fwd_kvblocks needs: n_blocks * B*Hq*Sq * (D + 1) * 4. */
+/* Bytes of workspace attn_fwd_kvblocks needs: 0 for up to 32 blocks (folded
+ * in one launch), else n_blocks * B*Hq*Sq * (D + 1) * 4 (per-block partials). */
 HATTN_API size_t attn_fwd_kvblocks_workspace_size(int B, int Hq, int Sq, int D, int n_blocks);
 
 /*
