@@ -157,6 +157,23 @@ def test_fp8_persistent_short_kv(h):
     check_fp8(h, Workload("f8p", B=1, Hq=40, Hkv=20, Sq=1200, Sk=640, dtype="e4m3", seed=41))
 
 
+def test_fp8_persistent_causal_ragged(h):
+    # the persistent causal path (more units than SMs, at most 16 KV tiles) with e4m3 inputs
+    check_fp8(h, Workload("f8pc", B=2, Hq=40, Hkv=8, Sq=1000, Sk=1100, causal=True, dtype="e4m3", seed=42))
+
+
+def test_fp8_at_video_shape_sampled_rows(h):
+    # the e4m3 bench line at the 32760-token video shape (Q, K RMS-normalised)
+    w = workloads.get("fp8_32760")
+    check_fp8(h, w, rows=sample_rows(w.Sq, 16, seed=w.seed))
+
+
+def test_bf16_at_fp8_shape_sampled_rows(h):
+    # the bf16 bench line at the 75600-token shape
+    w = workloads.get("bf16_75600")
+    check_bf16(h, w, rows=sample_rows(w.Sq, 32, seed=w.seed))
+
+
 def test_fp8_entry_points_agree_bitwise(h):
     # attn_fwd takes its fp16 scratch for V from the stream-ordered pool,
     # attn_fwd_ws (the binding's path) from the caller: same kernels, same bits
