@@ -102,6 +102,37 @@ def test_cuda_graph_capture_fp8_stream_ordered_scratch(h):
     del g
 
 
+def test_cuda_graph_capture_prologue_then_fp8(h):
+    # the e4m3 prologue (memset + two kernels) and the e4m3 forward on its
+    # codes, captured in one graph; replays equal the eager calls bit for bit
+    g0 = torch.Generator().manual_seed(80)
+    q, k, v = (torch.randn(1, 3, S, 128, generator=g0).to(torch.bfloat16).cuda() for S in (250, 270, 270))
+    ws = torch.empty(h.fwd_workspace_size(1, 3, 270, 128, h.E4M3), dtype=torch.uint8, device="cuda")
+
+    def run(stream):
+        qc, qd = h.quantize_e4m3(q, rmsnorm=True, stream=stream)
+        kc, kd = h.quantize_e4m3(k, rmsnorm=True, stream=stream)
+        vc, vd = h.quantize_e4m3(v, rmsnorm=False, stream=stream)
+        out, lse = h.attn_fwd(qc, kc, vc, q_descale=qd, k_descale=kd, v_descale=vd, workspace=ws, stream=stream)
+        return qc, qd, out, lse
+
+    eager = run(None)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            graphed = run(s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    for a, b in zip(graphed, eager):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    del g
+
+
 def test_fail_closed_on_device(h):
     q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")     # head dim 64 is not offered
     with pytest.raises(h.HattnError) as ei:
