@@ -4,6 +4,8 @@ its bitwise properties (repeat runs, batch composition, head slicing).
 Bar (the pages give none for gradients): for each of dQ, dK, dV,
 max abs <= 2e-2 * max(1, max |ref|) and normalised RMS <= 1e-2.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -104,3 +106,21 @@ def test_bwd_single_key_closed_form(h):
     assert dq.float().abs().max() < 1e-3 and dk.float().abs().max() < 1e-2
     ref = do.double().sum(dim=2)
     assert np.allclose(dv[:, :, 0].double().cpu().numpy(), ref.cpu().numpy(), atol=2e-2 * max(1, ref.abs().max().item()))
+
+
+def test_bwd_llm_config_sums_over_keys(h):
+    # the bench's backward (B=2, Hq=32, Hkv=8, S=2048, causal) at full size,
+    # checked by properties that hold at any size: rows of dS sum to zero, so
+    # dK summed over keys vanishes; rows of P sum to one, so dV summed over
+    # keys equals dO summed over the rows of the KV head's query heads.  With
+    # bf16 P, dS and outputs the identities hold to a small fraction of each
+    # sum's absolute mass; a wrong or missing term breaks them at order one.
+    w = workloads.get("llm_gqa")
+    x = {k: v.cuda() for k, v in make_bwd_inputs(w).items()}
+    _, _, dq, dk, dv = fwd_bwd(h, x, True)
+    G = w.Hq // w.Hkv
+    dk_err = dk.double().sum(dim=2).abs() / dk.double().abs().sum(dim=2)
+    want = x["dout"].double().view(w.B, w.Hkv, G, w.Sq, w.D).sum(dim=(2, 3))
+    dv_err = (dv.double().sum(dim=2) - want).abs() / dv.double().abs().sum(dim=2)
+    print("max relative sums: dK %.3e, dV %.3e" % (dk_err.max().item(), dv_err.max().item()))
+    assert dk_err.max().item() <= 1e-2 and dv_err.max().item() <= 1e-2
