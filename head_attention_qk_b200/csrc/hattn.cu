@@ -139,6 +139,17 @@ bool sizes_fit(long long B, long long H, long long S) {
   return B * H <= 65535LL * 1024 && B * H * S < (1LL << 40) && S < (1LL << 30);
 }
 
+// The backward's launch sizes: the persistent dQ kernel counts its units
+// (B*Hq*ceil(Sq/128)) in an int, the Delta kernel takes one CTA per 64 rows in
+// grid x, and dK/dV puts B*Hkv in grid x and the key tiles in grid y.
+bool bwd_sizes_ok(int B, int Hq, int Hkv, int Sq, int Sk) {
+  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk)) return false;
+  const long long rows = (long long)B * Hq * Sq;
+  if ((long long)B * Hq * ((Sq + kTile - 1) / kTile) > INT_MAX) return false;
+  if ((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta > INT_MAX) return false;
+  return (Sk + kTile - 1) / kTile <= 65535;
+}
+
 }  // namespace
 
 // 3-D view (D, S, heads) of a [.., heads, S, D] tensor, box (box_x, 128 rows, 1 head),
@@ -419,8 +430,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (rc) return rc;
   if (Sk <= 0) return HATTN_EINVAL;
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
-  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
-  if ((Sk + kTile - 1) / kTile > 65535) return HATTN_EUNSUPPORTED;   // key tiles index the grid's y dimension
+  if (!bwd_sizes_ok(B, Hq, Hkv, Sq, Sk)) return HATTN_EUNSUPPORTED;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
   for (const void* p : ptrs)
     if (!aligned16(p)) return HATTN_EALIGN;
@@ -466,8 +476,7 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   if (rc) return rc;
   if (Sk <= 0) return HATTN_EINVAL;
   if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
-  if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk) || B * Hq > 65535) return HATTN_EUNSUPPORTED;
-  if ((Sk + kTile - 1) / kTile > 65535) return HATTN_EUNSUPPORTED;   // key tiles index the grid's y dimension
+  if (!bwd_sizes_ok(B, Hq, Hkv, Sq, Sk)) return HATTN_EUNSUPPORTED;
   if ((long long)B * Hq * Sq > (long long)HATTN_NOALLOC_MAX_ROWS) return HATTN_EWORKSPACE;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
   for (const void* p : ptrs)

@@ -124,3 +124,24 @@ def test_bwd_llm_config_sums_over_keys(h):
     dv_err = (dv.double().sum(dim=2) - want).abs() / dv.double().abs().sum(dim=2)
     print("max relative sums: dK %.3e, dV %.3e" % (dk_err.max().item(), dv_err.max().item()))
     assert dk_err.max().item() <= 1e-2 and dv_err.max().item() <= 1e-2
+
+
+def test_bwd_more_than_65535_heads(h):
+    # B*Hq = 65600 query heads (more than a grid's y dimension holds): rows of
+    # the batch agree bit for bit with the same rows run alone, and one row
+    # with the oracle
+    w = Workload("manyheads", B=4100, Hq=16, Hkv=8, Sq=5, Sk=7, causal=False, seed=71)
+    x_cpu = make_bwd_inputs(w)
+    x = {k: v.cuda() for k, v in x_cpu.items()}
+    _, _, dq, dk, dv = fwd_bwd(h, x, False)
+    for rows in (slice(0, 2), slice(4098, 4100)):
+        xs = {k: v[rows].contiguous() for k, v in x.items()}
+        _, _, dqs, dks, dvs = fwd_bwd(h, xs, False)
+        assert torch.equal(dqs.view(torch.int16), dq[rows].view(torch.int16))
+        assert torch.equal(dks.view(torch.int16), dk[rows].view(torch.int16))
+        assert torch.equal(dvs.view(torch.int16), dv[rows].view(torch.int16))
+    b = 4099
+    rdq, rdk, rdv, _, _ = oracle.attn_bwd(*(np_bits(x_cpu[n][b:b + 1]) for n in ("q", "k", "v", "dout")), w.scale)
+    for n, g, r in (("dq", dq[b:b + 1], rdq), ("dk", dk[b:b + 1], rdk), ("dv", dv[b:b + 1], rdv)):
+        e = grad_errors(g, r)
+        assert grad_ok(e), (n, e)
