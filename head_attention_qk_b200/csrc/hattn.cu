@@ -318,16 +318,16 @@ int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H,
   const float eps32 = (float)eps;                  // the normalisation runs in fp32
   if (rmsnorm && !(eps32 > 0.f && eps32 < 3.0e38f)) return HATTN_EINVAL;
   if (D != kPrepD) return HATTN_EUNSUPPORTED;
-  if ((long long)B * H > 65535 || !sizes_fit(B, H, S)) return HATTN_EUNSUPPORTED;
+  if (!sizes_fit(B, H, S) || (S + kPrepRowsPerCta - 1) / kPrepRowsPerCta > INT_MAX) return HATTN_EUNSUPPORTED;
   if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(descale) & 3u)) return HATTN_EALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int bh = B * H;
-  const dim3 grid((S + kPrepRowsPerCta - 1) / kPrepRowsPerCta, bh);
+  const dim3 grid((S + kPrepRowsPerCta - 1) / kPrepRowsPerCta, bh < 65535 ? bh : 65535);   // heads strided over y
   if (cudaMemsetAsync(descale, 0, (size_t)bh * sizeof(float), st) != cudaSuccess) return HATTN_ELAUNCH;
   prep_amax_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
-                                                   reinterpret_cast<unsigned int*>(descale), S, rmsnorm ? 1 : 0, eps32);
+                                                   reinterpret_cast<unsigned int*>(descale), S, bh, rmsnorm ? 1 : 0, eps32);
   prep_quantize_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
-                                                       reinterpret_cast<uint8_t*>(codes), descale, S,
+                                                       reinterpret_cast<uint8_t*>(codes), descale, S, bh,
                                                        rmsnorm ? 1 : 0, eps32);
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }

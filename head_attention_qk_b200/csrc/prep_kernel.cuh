@@ -62,14 +62,15 @@ __device__ __forceinline__ float prep_row_factor(const PrepVals& p, int rmsnorm,
   return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fmul_rn(s, 0.0078125f), eps)));
 }
 
-// grid (ceil(S / 64), B*H): the largest |y| of each head, stored negated into
+// grid (ceil(S / 64), min(B*H, 65535)), heads strided over grid y: the largest |y| of each head, stored negated into
 // amax_bits (zeroed): the bit patterns of non-positive floats order like
 // unsigned integers by magnitude, so atomicMax keeps the largest, and the
 // sign bit tells this value apart from a finished descale.
 __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
                                                                    unsigned int* __restrict__ amax_bits, int S,
-                                                                   int rmsnorm, float eps) {
-  const int bh = blockIdx.y;
+                                                                   int n_bh, int rmsnorm, float eps) {
+  __shared__ float wmax[kPrepThreads / 32];
+  for (int bh = blockIdx.y; bh < n_bh; bh += gridDim.y) {
   const int sub = threadIdx.x & 15;               // which 8 values of the row
   const int r0 = blockIdx.x * kPrepRowsPerCta + (threadIdx.x >> 4);
   const uint4* base = reinterpret_cast<const uint4*>(x) + (long long)bh * S * 16 + sub;
@@ -89,7 +90,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t*
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  __shared__ float wmax[kPrepThreads / 32];
   if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t*
 #pragma unroll
     for (int i = 1; i < kPrepThreads / 32; ++i) bm = fmaxf(bm, wmax[i]);
     atomicMax(&amax_bits[bh], __float_as_uint(-bm));
+  }
+  __syncthreads();                                // wmax is rewritten for the next head
   }
 }
 
@@ -130,14 +132,15 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   return r;
 }
 
-// grid (ceil(S / 64), B*H): the codes of each row, and the descale of each
+// grid (ceil(S / 64), min(B*H, 65535)), heads strided over grid y: the codes of each row, and the descale of each
 // head in place of its maximum.  CTAs walk the rows in the reverse of the
 // maxima kernel's order, so the rows it read last, still in L2, come first.
 __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
                                                                        uint8_t* __restrict__ codes,
                                                                        float* __restrict__ descale, int S,
-                                                                       int rmsnorm, float eps) {
-  const int bh = gridDim.y - 1 - blockIdx.y;
+                                                                       int n_bh, int rmsnorm, float eps) {
+  for (int bi = blockIdx.y; bi < n_bh; bi += gridDim.y) {
+  const int bh = n_bh - 1 - bi;
   const int tile = gridDim.x - 1 - blockIdx.x;
   const int sub = threadIdx.x & 15;
   const int r0 = tile * kPrepRowsPerCta + (threadIdx.x >> 4);
@@ -168,6 +171,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint1
     const int s = r0 + 16 * k;
     if (s < S)
       dst[(long long)s * 16] = make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
+  }
   }
 }
 

@@ -67,6 +67,14 @@ def test_prologue_extreme_magnitudes(h):
         check_exact(h, x.to(torch.bfloat16), rms)
 
 
+def test_prologue_more_than_65535_heads(h):
+    # 70000 heads: more than a grid's y dimension holds, so CTAs stride over heads
+    g = torch.Generator().manual_seed(33)
+    x = (torch.randn(2, 35000, 3, 128, generator=g) * 1.3).to(torch.bfloat16)
+    check_exact(h, x, True)
+    check_exact(h, x, False)
+
+
 def test_prologue_fp8_config_q_bit_exact(h):
     w = workloads.get("fp8")
     g = torch.Generator().manual_seed(w.seed)
