@@ -324,11 +324,17 @@ int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H,
   const int bh = B * H;
   const dim3 grid((S + kPrepRowsPerCta - 1) / kPrepRowsPerCta, bh < 65535 ? bh : 65535);   // heads strided over y
   if (cudaMemsetAsync(descale, 0, (size_t)bh * sizeof(float), st) != cudaSuccess) return HATTN_ELAUNCH;
-  prep_amax_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
-                                                   reinterpret_cast<unsigned int*>(descale), S, bh, rmsnorm ? 1 : 0, eps32);
-  prep_quantize_kernel<<<grid, kPrepThreads, 0, st>>>(reinterpret_cast<const uint16_t*>(x),
-                                                       reinterpret_cast<uint8_t*>(codes), descale, S, bh,
-                                                       rmsnorm ? 1 : 0, eps32);
+  const uint16_t* xs = reinterpret_cast<const uint16_t*>(x);
+  unsigned int* amax = reinterpret_cast<unsigned int*>(descale);
+  uint8_t* cs = reinterpret_cast<uint8_t*>(codes);
+  const int rms = rmsnorm ? 1 : 0;
+  if (bh <= 65535) {
+    prep_amax_kernel<false><<<grid, kPrepThreads, 0, st>>>(xs, amax, S, bh, rms, eps32);
+    prep_quantize_kernel<false><<<grid, kPrepThreads, 0, st>>>(xs, cs, descale, S, bh, rms, eps32);
+  } else {
+    prep_amax_kernel<true><<<grid, kPrepThreads, 0, st>>>(xs, amax, S, bh, rms, eps32);
+    prep_quantize_kernel<true><<<grid, kPrepThreads, 0, st>>>(xs, cs, descale, S, bh, rms, eps32);
+  }
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 

@@ -62,15 +62,13 @@ __device__ __forceinline__ float prep_row_factor(const PrepVals& p, int rmsnorm,
   return __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fmul_rn(s, 0.0078125f), eps)));
 }
 
-// grid (ceil(S / 64), min(B*H, 65535)), heads strided over grid y: the largest |y| of each head, stored negated into
+// grid (ceil(S / 64), min(B*H, 65535)); kStride: heads strided over grid y
+// (more than 65535 of them), else head = blockIdx.y.  The largest |y| of each head, stored negated into
 // amax_bits (zeroed): the bit patterns of non-positive floats order like
 // unsigned integers by magnitude, so atomicMax keeps the largest, and the
 // sign bit tells this value apart from a finished descale.
-__global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
-                                                                   unsigned int* __restrict__ amax_bits, int S,
-                                                                   int n_bh, int rmsnorm, float eps) {
-  __shared__ float wmax[kPrepThreads / 32];
-  for (int bh = blockIdx.y; bh < n_bh; bh += gridDim.y) {
+__device__ __forceinline__ void prep_amax_head(const uint16_t* __restrict__ x, unsigned int* __restrict__ amax_bits,
+                                               int S, int bh, int rmsnorm, float eps, float* wmax) {
   const int sub = threadIdx.x & 15;               // which 8 values of the row
   const int r0 = blockIdx.x * kPrepRowsPerCta + (threadIdx.x >> 4);
   const uint4* base = reinterpret_cast<const uint4*>(x) + (long long)bh * S * 16 + sub;
@@ -98,7 +96,20 @@ __global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t*
     for (int i = 1; i < kPrepThreads / 32; ++i) bm = fmaxf(bm, wmax[i]);
     atomicMax(&amax_bits[bh], __float_as_uint(-bm));
   }
-  __syncthreads();                                // wmax is rewritten for the next head
+}
+
+template <bool kStride>
+__global__ void __launch_bounds__(kPrepThreads) prep_amax_kernel(const uint16_t* __restrict__ x,
+                                                                   unsigned int* __restrict__ amax_bits, int S,
+                                                                   int n_bh, int rmsnorm, float eps) {
+  __shared__ float wmax[kPrepThreads / 32];
+  if constexpr (!kStride) {
+    prep_amax_head(x, amax_bits, S, blockIdx.y, rmsnorm, eps, wmax);
+  } else {
+    for (int bh = blockIdx.y; bh < n_bh; bh += gridDim.y) {
+      prep_amax_head(x, amax_bits, S, bh, rmsnorm, eps, wmax);
+      __syncthreads();                            // wmax is rewritten for the next head
+    }
   }
 }
 
@@ -132,15 +143,12 @@ __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
   return r;
 }
 
-// grid (ceil(S / 64), min(B*H, 65535)), heads strided over grid y: the codes of each row, and the descale of each
+// grid (ceil(S / 64), min(B*H, 65535)), heads strided over grid y with kStride: the codes of each row, and the descale of each
 // head in place of its maximum.  CTAs walk the rows in the reverse of the
 // maxima kernel's order, so the rows it read last, still in L2, come first.
-__global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
-                                                                       uint8_t* __restrict__ codes,
-                                                                       float* __restrict__ descale, int S,
-                                                                       int n_bh, int rmsnorm, float eps) {
-  for (int bi = blockIdx.y; bi < n_bh; bi += gridDim.y) {
-  const int bh = n_bh - 1 - bi;
+__device__ __forceinline__ void prep_quantize_head(const uint16_t* __restrict__ x, uint8_t* __restrict__ codes,
+                                                   float* __restrict__ descale, int S, int bh, int rmsnorm,
+                                                   float eps) {
   const int tile = gridDim.x - 1 - blockIdx.x;
   const int sub = threadIdx.x & 15;
   const int r0 = tile * kPrepRowsPerCta + (threadIdx.x >> 4);
@@ -172,6 +180,18 @@ __global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint1
     if (s < S)
       dst[(long long)s * 16] = make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));
   }
+}
+
+template <bool kStride>
+__global__ void __launch_bounds__(kPrepThreads) prep_quantize_kernel(const uint16_t* __restrict__ x,
+                                                                       uint8_t* __restrict__ codes,
+                                                                       float* __restrict__ descale, int S,
+                                                                       int n_bh, int rmsnorm, float eps) {
+  if constexpr (!kStride) {
+    prep_quantize_head(x, codes, descale, S, gridDim.y - 1 - blockIdx.y, rmsnorm, eps);
+  } else {
+    for (int bi = blockIdx.y; bi < n_bh; bi += gridDim.y)
+      prep_quantize_head(x, codes, descale, S, n_bh - 1 - bi, rmsnorm, eps);
   }
 }
 
