@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <cfloat>
 #include <climits>
 #include <mutex>
 
@@ -105,14 +106,13 @@ int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
 constexpr int kPersistMaxKvTiles = 8;
 
 template <bool kFp8, bool kPartial>
-int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, int max_sk, cudaStream_t st) {
+int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, long long max_tiles, cudaStream_t st) {
   const long long units = (long long)a.n_qpairs * a.B * a.Hq * n_blocks_in_launch;
   if (units <= 0 || units > INT_MAX) return HATTN_EUNSUPPORTED;
   const int sms = device_sm_count();
-  if (sms <= 0) return HATTN_EDEVICE;
+  if (sms <= 0) return HATTN_ELAUNCH;
   FwdArgs args = a;
   args.total_units = (int)units;
-  const int max_tiles = (max_sk + kBlockN - 1) / kBlockN;
   const bool persist = max_tiles <= (a.causal ? 2 : 1) * kPersistMaxKvTiles && units > sms;
   if (persist) return launch_fwd_grid<kFp8, kPartial, true>(args, sms, st);
   return launch_fwd_grid<kFp8, kPartial, false>(args, (int)units, st);
@@ -121,7 +121,7 @@ int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, int max_sk, cudaStream_
 int check_common(int B, int Hq, int Hkv, int Sq, int D, float scale) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || D <= 0) return HATTN_EINVAL;
   if (Hq % Hkv != 0) return HATTN_EINVAL;
-  if (!(scale > 0.f) || scale != scale) return HATTN_EINVAL;
+  if (!(scale > 0.f && scale <= FLT_MAX)) return HATTN_EINVAL;   // also refuses NaN and +inf
   if (D != kHeadDim) return HATTN_EUNSUPPORTED;
   return HATTN_OK;
 }
@@ -201,7 +201,7 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
     // V widened to fp16 once (exact), read by the attention kernel's P V MMAs
     const long long n16 = (long long)B * Hkv * Sk * kHeadDim / 16;
     const int sms = device_sm_count();
-    if (sms <= 0) return HATTN_EDEVICE;
+    if (sms <= 0) return HATTN_ELAUNCH;
     const long long want = (n16 + 255) / 256;
     const int grid = (int)(want < 8LL * sms ? want : 8LL * sms);
     widen_e4m3_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(v), reinterpret_cast<uint4*>(v16), n16);
@@ -220,7 +220,8 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
   a.lse = lse;
   a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
   a.block_offset = 0;
-  return fp8 ? launch_fwd<true, false>(a, 1, Sk, st) : launch_fwd<false, false>(a, 1, Sk, st);
+  const long long kv_tiles = (Sk + kBlockN - 1) / kBlockN;
+  return fp8 ? launch_fwd<true, false>(a, 1, kv_tiles, st) : launch_fwd<false, false>(a, 1, kv_tiles, st);
 }
 
 // Stream-ordered scratch for attn_fwd callers that pass no workspace.  Outside
@@ -233,12 +234,12 @@ constexpr uint64_t kPoolKeepBytes = 256ull << 20;
 int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return HATTN_ELAUNCH;
-  if (cs != cudaStreamCaptureStatusNone) return cudaMallocAsync(p, bytes, st) == cudaSuccess ? HATTN_OK : HATTN_EDEVICE;
+  if (cs != cudaStreamCaptureStatusNone) return cudaMallocAsync(p, bytes, st) == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static cudaMemPool_t pools[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HATTN_EDEVICE;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HATTN_ELAUNCH;
   cudaMemPool_t pool;
   {
     std::lock_guard<std::mutex> g(mu);
@@ -248,14 +249,14 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
       props.location.type = cudaMemLocationTypeDevice;
       props.location.id = dev;
       cudaMemPool_t np;
-      if (cudaMemPoolCreate(&np, &props) != cudaSuccess) return HATTN_EDEVICE;
+      if (cudaMemPoolCreate(&np, &props) != cudaSuccess) return HATTN_ELAUNCH;
       uint64_t keep = kPoolKeepBytes;
       cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep);
       pools[dev] = np;
     }
     pool = pools[dev];
   }
-  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? HATTN_OK : HATTN_EDEVICE;
+  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
 int check_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
@@ -307,7 +308,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
   if ((rc = scratch_alloc(&v16, need, st))) return rc;
   rc = attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale, v_descale,
                      v16, st);
-  if (cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_EDEVICE;
+  if (cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_ELAUNCH;
   return rc;
 }
 
@@ -374,7 +375,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     // partials are written and no merge pass is needed.
     memset(&a, 0, sizeof(a));
     if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
-    int tiles = 0;
+    long long tiles = 0;
     for (int i = 0; i < n_blocks; ++i) {
       if (!encode_rows(&a.tm_k[i], k_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
       if (!encode_rows(&a.tm_v[i], v_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
@@ -388,9 +389,9 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     a.out = out;
     a.lse = lse;
     a.fused_blocks = n_blocks;
-    a.fused_tiles = tiles;
+    a.fused_tiles = (int)tiles;   // < 32 * 2^23
     if (n_blocks == 1) a.fused_blocks = 0;   // a single block is a plain forward
-    return launch_fwd<false, false>(a, 1, tiles * kBlockN, st);
+    return launch_fwd<false, false>(a, 1, tiles, st);
   }
 
   const long long rows = (long long)B * Hq * Sq;
@@ -416,7 +417,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     a.out = o_parts;
     a.lse = lse_parts;
     a.block_offset = first;
-    if ((rc = launch_fwd<false, true>(a, cnt, max_len, st))) return rc;
+    if ((rc = launch_fwd<false, true>(a, cnt, (max_len + kBlockN - 1) / kBlockN, st))) return rc;
   }
   const unsigned grid = (unsigned)((rows + 7) / 8);
   lse_merge_kernel<<<grid, 256, 0, st>>>(o_parts, lse_parts, n_blocks, rows, reinterpret_cast<uint16_t*>(out), lse);
@@ -442,7 +443,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
     if (!aligned16(p)) return HATTN_EALIGN;
   if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq)) return HATTN_EWORKSPACE;
   const int sms = device_sm_count();
-  if (sms <= 0) return HATTN_EDEVICE;
+  if (sms <= 0) return HATTN_ELAUNCH;
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
                     reinterpret_cast<float*>(workspace), sms, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -492,7 +493,7 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   // Delta is fully rewritten for every row this call reads, so the array needs
   // no clearing between calls.
   const int sms = device_sm_count();
-  if (sms <= 0) return HATTN_EDEVICE;
+  if (sms <= 0) return HATTN_ELAUNCH;
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta, sms,
                     reinterpret_cast<cudaStream_t>(stream));
 }

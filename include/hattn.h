@@ -51,12 +51,14 @@ typedef enum { HATTN_BF16 = 0, HATTN_E4M3 = 1 } hattn_dtype;
 
 enum {
   HATTN_OK = 0,
-  HATTN_EINVAL = -1,        /* null pointer, size <= 0, Hq % Hkv != 0, scale <= 0,
-                               descales given for bf16 or missing for e4m3 */
+  HATTN_EINVAL = -1,        /* null pointer, size <= 0, Hq % Hkv != 0, scale not a
+                               finite positive number, descales given for bf16 or
+                               missing for e4m3 */
   HATTN_EUNSUPPORTED = -2,  /* D != 128, causal with Sq > Sk, fp8 backward, a zero-length block */
   HATTN_EALIGN = -3,        /* a device pointer is not 16-byte aligned */
   HATTN_EWORKSPACE = -4,    /* workspace smaller than the matching *_workspace_size() */
-  HATTN_ELAUNCH = -5,       /* CUDA reported an error when encoding or launching */
+  HATTN_ELAUNCH = -5,       /* CUDA reported an error: no usable device, scratch
+                               allocation, descriptor encoding or kernel launch */
   HATTN_EDEVICE = -6        /* a kernel gave up on a bounded wait (see attn_get_device_error) */
 };
 
@@ -66,7 +68,7 @@ enum {
  *   k, v [B, Hkv, Sk, D]  same element type as q
  *   out  [B, Hq,  Sq, D]  bf16, written
  *   lse  [B, Hq,  Sq]     fp32, written
- *   scale: softmax scale (> 0), e.g. 1/sqrt(D).
+ *   scale: softmax scale (finite, > 0), e.g. 1/sqrt(D).
  *   q_descale [B*Hq], k_descale [B*Hkv], v_descale [B*Hkv]: fp32 device arrays
  *     for e4m3 (the real value of a code x of head (b, h) is x * descale[b*H + h];
  *     one value per tensor is the case where all entries are equal); all three

@@ -60,6 +60,7 @@ def fwd(h, q=A, k=A, v=A, out=A, lse=A, B=1, Hq=2, Hkv=2, Sq=128, Sk=128, D=128,
 @pytest.mark.parametrize("kw,code", [
     (dict(q=None), -1), (dict(lse=None), -1), (dict(B=0), -1), (dict(Sq=0), -1), (dict(Sk=-1), -1),
     (dict(Hq=3, Hkv=2), -1), (dict(scale=0.0), -1), (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1),
+    (dict(scale=float("inf")), -1),
     (dict(qd=A, kd=A, vd=A), -1),               # descales with bf16
     (dict(dtype=1), -1),                        # e4m3 without descales
     (dict(dtype=1, qd=A, kd=A, vd=None), -1),
