@@ -71,10 +71,58 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+# Argument checks.  The library sees only pointers and the sizes passed with
+# them, so every tensor's shape and dtype are checked against those sizes here
+# (a buffer smaller than the sizes say would be read or written out of
+# bounds).  Shapes and dtypes are checked first, then that every tensor is a
+# contiguous CUDA tensor on one device; the call runs with that device current
+# and, by default, on its current stream.
+
+def _shape(t, name, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _dtype(t, name, *dtypes):
+    if t.dtype not in dtypes:
+        raise TypeError("%s must be %s, got %s" % (name, " or ".join(str(d) for d in dtypes), t.dtype))
+
+
+def _dims4(t, name):
+    if not isinstance(t, torch.Tensor) or t.dim() != 4:
+        raise ValueError("%s must be a 4-d [B, H, S, D] tensor" % name)
+    return tuple(int(x) for x in t.shape)
+
+
+def _device(named):
+    """The one CUDA device of the (name, tensor) pairs (None entries skipped)."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be a CUDA tensor" % name)
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("%s is on %s, the other tensors on %s" % (name, t.device, dev))
+    return dev
+
+
+def _stream(stream, dev=None):
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and stream.device != dev:
+        raise ValueError("stream is on %s, the tensors on %s" % (stream.device, dev))
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -85,11 +133,19 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError("inputs must be bfloat16 or float8_e4m3fn, got %s" % t.dtype)
 
 
-def _require(t: torch.Tensor, name: str):
-    if not t.is_cuda:
-        raise ValueError("%s must be a CUDA tensor" % name)
-    if not t.is_contiguous():
-        raise ValueError("%s must be contiguous" % name)
+def _descales(dt, B, Hq, Hkv, q_descale, k_descale, v_descale):
+    given = [d is not None for d in (q_descale, k_descale, v_descale)]
+    if dt == BF16:
+        if any(given):
+            raise ValueError("descales are for e4m3 inputs only")
+        return
+    if not all(given):
+        raise ValueError("e4m3 inputs need q_descale, k_descale and v_descale")
+    for d, name, n in ((q_descale, "q_descale", B * Hq), (k_descale, "k_descale", B * Hkv),
+                       (v_descale, "v_descale", B * Hkv)):
+        _dtype(d, name, torch.float32)
+        if d.numel() != n:
+            raise ValueError("%s must hold %d values (one per batch and head), got %d" % (name, n, d.numel()))
 
 
 def fwd_workspace_size(B, Hkv, Sk, D, dtype) -> int:
@@ -104,25 +160,34 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
     tensor of at least fwd_workspace_size() bytes), else one from torch's
     allocator; the library itself then allocates nothing.
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, n)
-    B, Hq, Sq, D = q.shape
-    _, Hkv, Sk, _ = k.shape
+    B, Hq, Sq, D = _dims4(q, "q")
+    _, Hkv, Sk, _ = _dims4(k, "k")
+    _shape(k, "k", (B, Hkv, Sk, D))
+    _shape(v, "v", (B, Hkv, Sk, D))
     dt = _dtype_code(q)
+    _dtype(k, "k", q.dtype)
+    _dtype(v, "v", q.dtype)
+    _descales(dt, B, Hq, Hkv, q_descale, k_descale, v_descale)
+    if out is not None:
+        _shape(out, "out", (B, Hq, Sq, D))
+        _dtype(out, "out", torch.bfloat16)
+    if lse is not None:
+        _shape(lse, "lse", (B, Hq, Sq))
+        _dtype(lse, "lse", torch.float32)
+    dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("q_descale", q_descale),
+                   ("k_descale", k_descale), ("v_descale", v_descale), ("workspace", workspace)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
     if lse is None:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
     ws_bytes = fwd_workspace_size(B, Hkv, Sk, D, dt)
     if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    if workspace is not None:
-        _require(workspace, "workspace")
-    rc = lib.attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
-                         int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
-                         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
-                         _stream(stream))
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+                             int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
+                             _ptr(workspace), _nbytes(workspace), _stream(stream, dev))
     _check(rc, "attn_fwd")
     return out, lse
 
@@ -130,16 +195,23 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
 def quantize_e4m3(x, rmsnorm=False, eps=1e-6, codes=None, descale=None, stream=None):
     """bf16 x [B,H,S,D] -> (e4m3fn codes [B,H,S,D], fp32 descale [B,H]) with an
     optional per-row RMS normalisation first (see attn_quantize_e4m3 in hattn.h)."""
-    _require(x, "x")
-    if x.dtype != torch.bfloat16 or x.dim() != 4:
-        raise TypeError("quantize_e4m3 takes a [B,H,S,D] bfloat16 tensor")
-    B, H, S, D = x.shape
+    B, H, S, D = _dims4(x, "x")
+    _dtype(x, "x", torch.bfloat16)
+    if codes is not None:
+        _shape(codes, "codes", (B, H, S, D))
+        _dtype(codes, "codes", torch.float8_e4m3fn)
+    if descale is not None:
+        _dtype(descale, "descale", torch.float32)
+        if descale.numel() != B * H:
+            raise ValueError("descale must hold %d values (one per batch and head)" % (B * H))
+    dev = _device([("x", x), ("codes", codes), ("descale", descale)])
     if codes is None:
-        codes = torch.empty((B, H, S, D), dtype=torch.float8_e4m3fn, device=x.device)
+        codes = torch.empty((B, H, S, D), dtype=torch.float8_e4m3fn, device=dev)
     if descale is None:
-        descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
-    rc = lib.attn_quantize_e4m3(_ptr(x), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)), float(eps),
-                                _stream(stream))
+        descale = torch.empty((B, H), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.attn_quantize_e4m3(_ptr(x), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)),
+                                    float(eps), _stream(stream, dev))
     _check(rc, "attn_quantize_e4m3")
     return codes, descale
 
@@ -149,31 +221,46 @@ def kvblocks_workspace_size(B, Hq, Sq, D, n_blocks) -> int:
 
 
 def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=None, lse=None, stream=None):
-    """Unmasked attention of q to the concatenation of the KV blocks, per block + fixed-order LSE merge."""
-    _require(q, "q")
+    """Unmasked attention of q to the concatenation of the KV blocks, folded in block order."""
+    B, Hq, Sq, D = _dims4(q, "q")
     n = len(k_blocks)
     if n != len(v_blocks) or n == 0:
         raise ValueError("need the same non-zero number of K and V blocks")
-    for t in list(k_blocks) + list(v_blocks):
-        _require(t, "kv block")
-    B, Hq, Sq, D = q.shape
-    Hkv = k_blocks[0].shape[1]
+    dt = _dtype_code(q)
+    Hkv = _dims4(k_blocks[0], "k_blocks[0]")[1]
+    lens = []
+    for i, (kb, vb) in enumerate(zip(k_blocks, v_blocks)):
+        L = _dims4(kb, "k_blocks[%d]" % i)[2]
+        _shape(kb, "k_blocks[%d]" % i, (B, Hkv, L, D))
+        _shape(vb, "v_blocks[%d]" % i, (B, Hkv, L, D))
+        _dtype(kb, "k_blocks[%d]" % i, q.dtype)
+        _dtype(vb, "v_blocks[%d]" % i, q.dtype)
+        lens.append(L)
+    if out is not None:
+        _shape(out, "out", (B, Hq, Sq, D))
+        _dtype(out, "out", torch.bfloat16)
+    if lse is not None:
+        _shape(lse, "lse", (B, Hq, Sq))
+        _dtype(lse, "lse", torch.float32)
+    dev = _device([("q", q), ("out", out), ("lse", lse), ("workspace", workspace)]
+                  + [("k_blocks[%d]" % i, t) for i, t in enumerate(k_blocks)]
+                  + [("v_blocks[%d]" % i, t) for i, t in enumerate(v_blocks)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     kp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in k_blocks])
     vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in v_blocks])
-    lens = (ctypes.c_int * n)(*[int(t.shape[2]) for t in k_blocks])
+    ln = (ctypes.c_int * n)(*lens)
     ws_bytes = kvblocks_workspace_size(B, Hq, Sq, D, n)
     if workspace is None and ws_bytes:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
     if lse is None:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    rc = lib.attn_fwd_kvblocks(_ptr(q), ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
-                               ctypes.cast(lens, ctypes.c_void_p), n, _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, D,
-                               scale, _dtype_code(q), None, None, None, _ptr(workspace),
-                               0 if workspace is None else workspace.numel() * workspace.element_size(),
-                               _stream(stream))
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_kvblocks(_ptr(q), ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
+                                   ctypes.cast(ln, ctypes.c_void_p), n, _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, D,
+                                   scale, dt, None, None, None, _ptr(workspace), _nbytes(workspace),
+                                   _stream(stream, dev))
     _check(rc, "attn_fwd_kvblocks")
     return out, lse
 
@@ -182,22 +269,38 @@ def bwd_workspace_size(B, Hq, Sq) -> int:
     return lib.attn_bwd_workspace_size(B, Hq, Sq)
 
 
+def _bwd_args(q, k, v, out, lse, dout, dq, dk, dv):
+    """Sizes of a backward call after checking every tensor against them."""
+    B, Hq, Sq, D = _dims4(q, "q")
+    _, Hkv, Sk, _ = _dims4(k, "k")
+    for t, name, shape in ((k, "k", (B, Hkv, Sk, D)), (v, "v", (B, Hkv, Sk, D)), (out, "out", (B, Hq, Sq, D)),
+                           (dout, "dout", (B, Hq, Sq, D)), (dq, "dq", (B, Hq, Sq, D)), (dk, "dk", (B, Hkv, Sk, D)),
+                           (dv, "dv", (B, Hkv, Sk, D))):
+        if t is not None:
+            _shape(t, name, shape)
+            _dtype(t, name, torch.bfloat16)
+    _dtype(q, "q", torch.bfloat16)
+    _shape(lse, "lse", (B, Hq, Sq))
+    _dtype(lse, "lse", torch.float32)
+    return B, Hq, Hkv, Sq, Sk, D
+
+
 def attn_bwd(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, dq=None, dk=None, dv=None,
              stream=None):
     """dQ, dK, dV (bf16) of attention for upstream gradient dout."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (lse, "lse"), (dout, "dout")):
-        _require(t, n)
-    B, Hq, Sq, D = q.shape
-    _, Hkv, Sk, _ = k.shape
+    B, Hq, Hkv, Sq, Sk, D = _bwd_args(q, k, v, out, lse, dout, dq, dk, dv)
+    dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout), ("dq", dq),
+                   ("dk", dk), ("dv", dv), ("workspace", workspace)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if workspace is None:
-        workspace = torch.empty(bwd_workspace_size(B, Hq, Sq), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(bwd_workspace_size(B, Hq, Sq), dtype=torch.uint8, device=dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    rc = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                      B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
-                      workspace.numel() * workspace.element_size(), _stream(stream))
+    with torch.cuda.device(dev):
+        rc = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                          _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
+                          _nbytes(workspace), _stream(stream, dev))
     _check(rc, "attn_bwd")
     return dq, dk, dv
 
@@ -205,16 +308,17 @@ def attn_bwd(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, 
 def attn_bwd_noalloc(q, k, v, out, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, stream=None):
     """attn_bwd without a workspace, for callers that may not allocate device
     scratch; the library's static 16 MiB array holds Delta (B*Hq*Sq <= 2^22)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (lse, "lse"), (dout, "dout")):
-        _require(t, n)
-    B, Hq, Sq, D = q.shape
-    _, Hkv, Sk, _ = k.shape
+    B, Hq, Hkv, Sq, Sk, D = _bwd_args(q, k, v, out, lse, dout, dq, dk, dv)
+    dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout), ("dq", dq),
+                   ("dk", dk), ("dv", dv)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    rc = lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
-                              _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _stream(stream))
+    with torch.cuda.device(dev):
+        rc = lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)),
+                                  _stream(stream, dev))
     _check(rc, "attn_bwd_noalloc")
     return dq, dk, dv
 
