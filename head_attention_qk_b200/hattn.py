@@ -133,16 +133,13 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError("inputs must be bfloat16 or float8_e4m3fn, got %s" % t.dtype)
 
 
-def _descales(dt, B, Hq, Hkv, q_descale, k_descale, v_descale):
-    given = [d is not None for d in (q_descale, k_descale, v_descale)]
-    if dt == BF16:
-        if any(given):
-            raise ValueError("descales are for e4m3 inputs only")
-        return
-    if not all(given):
-        raise ValueError("e4m3 inputs need q_descale, k_descale and v_descale")
+def _descales(B, Hq, Hkv, q_descale, k_descale, v_descale):
+    """Size and type of each descale given; which ones must be given (all three
+    for e4m3, none for bf16) is the library's check (HATTN_EINVAL)."""
     for d, name, n in ((q_descale, "q_descale", B * Hq), (k_descale, "k_descale", B * Hkv),
                        (v_descale, "v_descale", B * Hkv)):
+        if d is None:
+            continue
         _dtype(d, name, torch.float32)
         if d.numel() != n:
             raise ValueError("%s must hold %d values (one per batch and head), got %d" % (name, n, d.numel()))
@@ -167,7 +164,7 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
     dt = _dtype_code(q)
     _dtype(k, "k", q.dtype)
     _dtype(v, "v", q.dtype)
-    _descales(dt, B, Hq, Hkv, q_descale, k_descale, v_descale)
+    _descales(B, Hq, Hkv, q_descale, k_descale, v_descale)
     if out is not None:
         _shape(out, "out", (B, Hq, Sq, D))
         _dtype(out, "out", torch.bfloat16)

@@ -41,7 +41,6 @@ def fwd_args(**kw):
     (dict(out=t(1, 4, 64, 128, dtype=f32)), TypeError),
     (dict(lse=t(1, 4, 64, dtype=bf)), TypeError),
     (dict(lse=t(1, 4, 32, dtype=f32)), ValueError),
-    (dict(q_descale=t(1, 4, dtype=f32)), ValueError),    # descales with bf16
 ])
 def test_fwd_argument_checks(h, kw, exc):
     with pytest.raises(exc):
@@ -51,8 +50,7 @@ def test_fwd_argument_checks(h, kw, exc):
 def test_fwd_e4m3_descale_checks(h):
     q, k, v = t(1, 4, 64, 128, dtype=e4), t(1, 2, 96, 128, dtype=e4), t(1, 2, 96, 128, dtype=e4)
     good = dict(q_descale=t(1, 4, dtype=f32), k_descale=t(1, 2, dtype=f32), v_descale=t(1, 2, dtype=f32))
-    with pytest.raises(ValueError):                      # missing descales
-        h.attn_fwd(q, k, v)
+    # which descales must be given is the library's check (HATTN_EINVAL, see test_abi.py)
     with pytest.raises(ValueError):                      # one value per tensor is not enough
         h.attn_fwd(q, k, v, **dict(good, k_descale=t(1, dtype=f32)))
     with pytest.raises(TypeError):

@@ -1,0 +1,94 @@
+"""GPU parity on scores that rise or fall steadily along the keys.
+
+With random inputs the running row maximum of the online softmax seldom moves
+by much after the first key tile, so the rescale of O and l (and the lazy
+skip of that rescale while the maximum has risen by at most 8 in log2 units)
+is barely exercised.  Here every query row i has its own slope: q_i is about
+c_i times the all-ones vector and key j about (j / 128) times it, so the
+scores of row i change by about sqrt(128) c_i per 128 keys (c_i from -1 to
+1.5: a fall of up to 16 and a rise of up to 24 in log2 units per key tile).
+Rows with a rise below 8 per tile take the lazy path with probabilities up to
+2^8 before the next rescale, rows above it rescale at every tile, and falling
+rows never do.  The softmax is nearly one-hot at one end of the range and
+flat in the middle.
+
+Bars as for the other parity tests: bf16 max |dO| <= 2e-2 and max |dLSE| <=
+1e-3; e4m3 normalised RMS of O <= 1e-2 against the oracle on the dequantized
+inputs; gradients max abs <= 2e-2 * max(1, max |ref|) and normalised RMS <=
+1e-2.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, fwd_errors, grad_errors, grad_ok, np_bits, oracle_fwd
+from workloads.gen import quantize_e4m3_per_head
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module")
+def h():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import head_attention_qk_b200 as pkg
+
+    return pkg
+
+
+def ramp_inputs(B, Hq, Hkv, Sq, Sk, seed):
+    g = torch.Generator().manual_seed(seed)
+    c = torch.linspace(-1.0, 1.5, Sq)
+    q = c[None, None, :, None] + 0.1 * torch.randn(B, Hq, Sq, 128, generator=g)
+    t = torch.arange(Sk, dtype=torch.float32) / 128.0
+    k = t[None, None, :, None] + 0.05 * torch.randn(B, Hkv, Sk, 128, generator=g)
+    v = torch.randn(B, Hkv, Sk, 128, generator=g)
+    do = torch.randn(B, Hq, Sq, 128, generator=g)
+    return [x.to(torch.bfloat16) for x in (q, k, v, do)]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
+    (1, 4, 2, 300, 1000, False),
+    (2, 2, 1, 700, 700, True),
+    (1, 2, 2, 129, 1500, True),
+])
+def test_fwd_rising_and_falling_scores(h, B, Hq, Hkv, Sq, Sk, causal):
+    q, k, v, _ = ramp_inputs(B, Hq, Hkv, Sq, Sk, 7 + Sq)
+    out, lse = h.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    assert h.get_device_error() == 0
+    o_ref, lse_ref = oracle_fwd(q, k, v, SCALE, causal)
+    assert float(np.max(lse_ref)) > 60.0                  # the steep rows reach large scores
+    e = fwd_errors(out, lse, o_ref, lse_ref)
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+
+
+def test_fp8_rising_and_falling_scores(h):
+    q, k, v, _ = ramp_inputs(1, 4, 2, 300, 1000, 31)
+    (qc, qd), (kc, kd), (vc, vd) = (quantize_e4m3_per_head(x) for x in (q, k, v))
+    out, lse = h.attn_fwd(qc.cuda(), kc.cuda(), vc.cuda(), q_descale=qd.cuda(), k_descale=kd.cuda(),
+                          v_descale=vd.cuda())
+    assert h.get_device_error() == 0
+    o_ref, lse_ref = oracle_fwd(qc, kc, vc, SCALE, descales=(qd, kd, vd))
+    e = fwd_errors(out, lse, o_ref, lse_ref)
+    assert e["o_nrms"] <= FP8_NRMS, e
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
+    (1, 4, 2, 300, 600, True),
+    (1, 2, 1, 260, 900, False),
+])
+def test_bwd_rising_and_falling_scores(h, B, Hq, Hkv, Sq, Sk, causal):
+    q, k, v, do = ramp_inputs(B, Hq, Hkv, Sq, Sk, 53 + Sk)
+    qc, kc, vc, doc = (x.cuda() for x in (q, k, v, do))
+    out, lse = h.attn_fwd(qc, kc, vc, causal=causal)
+    dq, dk, dv = h.attn_bwd(qc, kc, vc, out, lse, doc, causal=causal)
+    assert h.get_device_error() == 0
+    rdq, rdk, rdv, _, _ = oracle.attn_bwd(*(np_bits(x) for x in (q, k, v, do)), SCALE, causal=causal)
+    errs = {n: grad_errors(g, r) for n, g, r in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv))}
+    for n, e in errs.items():
+        assert grad_ok(e), (n, errs)
