@@ -41,12 +41,12 @@ def h():
     return pkg
 
 
-def ramp_inputs(B, Hq, Hkv, Sq, Sk, seed):
+def ramp_inputs(B, Hq, Hkv, Sq, Sk, seed, c_lo=-1.0, c_hi=1.5, tau=1.0, k_noise=0.05):
     g = torch.Generator().manual_seed(seed)
-    c = torch.linspace(-1.0, 1.5, Sq)
+    c = torch.linspace(c_lo, c_hi, Sq)
     q = c[None, None, :, None] + 0.1 * torch.randn(B, Hq, Sq, 128, generator=g)
-    t = torch.arange(Sk, dtype=torch.float32) / 128.0
-    k = t[None, None, :, None] + 0.05 * torch.randn(B, Hkv, Sk, 128, generator=g)
+    t = torch.arange(Sk, dtype=torch.float32) / 128.0 * tau
+    k = t[None, None, :, None] + k_noise * torch.randn(B, Hkv, Sk, 128, generator=g)
     v = torch.randn(B, Hkv, Sk, 128, generator=g)
     do = torch.randn(B, Hq, Sq, 128, generator=g)
     return [x.to(torch.bfloat16) for x in (q, k, v, do)]
@@ -78,17 +78,26 @@ def test_fp8_rising_and_falling_scores(h):
     assert e["o_nrms"] <= FP8_NRMS, e
 
 
+# The backward takes the slope from q (c from -4 to 6) over a smaller key ramp
+# (tau = 1/4) with unit key noise.  With the forward's inputs the keys share a
+# large common component w, and dQ_i = scale sum_j dS_ij k_j then carries
+# scale (Delta_i error) sum_j P_ij w: Delta comes from the bf16 O, whose
+# rounding alone (computed in fp64 on the CPU: round O to bf16, form Delta and
+# dS from it, round dS to bf16) puts dQ 4-9 % (normalised RMS) from the exact
+# gradient on those inputs, for any bf16 implementation of the method.  Here
+# the same computation gives 0.3-0.4 %, and LSE still reaches 75-96.
 @pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
     (1, 4, 2, 300, 600, True),
-    (1, 2, 1, 260, 900, False),
+    (1, 2, 1, 260, 500, False),
 ])
 def test_bwd_rising_and_falling_scores(h, B, Hq, Hkv, Sq, Sk, causal):
-    q, k, v, do = ramp_inputs(B, Hq, Hkv, Sq, Sk, 53 + Sk)
+    q, k, v, do = ramp_inputs(B, Hq, Hkv, Sq, Sk, 53 + Sk, c_lo=-4.0, c_hi=6.0, tau=0.25, k_noise=1.0)
     qc, kc, vc, doc = (x.cuda() for x in (q, k, v, do))
     out, lse = h.attn_fwd(qc, kc, vc, causal=causal)
     dq, dk, dv = h.attn_bwd(qc, kc, vc, out, lse, doc, causal=causal)
     assert h.get_device_error() == 0
-    rdq, rdk, rdv, _, _ = oracle.attn_bwd(*(np_bits(x) for x in (q, k, v, do)), SCALE, causal=causal)
+    rdq, rdk, rdv, _, lse_ref = oracle.attn_bwd(*(np_bits(x) for x in (q, k, v, do)), SCALE, causal=causal)
+    assert float(np.max(lse_ref)) > 60.0
     errs = {n: grad_errors(g, r) for n, g, r in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv))}
     for n, e in errs.items():
         assert grad_ok(e), (n, errs)
