@@ -46,13 +46,23 @@
 #include <omp.h>
 #endif
 
+/* Planted mistakes for the pin suite's own test (tests/test_oracle_mutants.py):
+ * built with -DORACLE_MUTANT=n (n > 0), MUT(n) is true at one site and the
+ * oracle computes something plausible but wrong there; every pin run against
+ * such a build must fail.  The normal build has ORACLE_MUTANT 0, where every
+ * MUT() is the constant 0 and the code is the definition. */
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+#define MUT(n) (ORACLE_MUTANT == (n))
+
 /* Storage kinds of the input arrays.  The oracle reads the same bytes the GPU
  * reads and widens them exactly to double. */
 enum { ORACLE_F64 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
 
 /* bfloat16: the upper 16 bits of an IEEE-754 binary32.  Widening is exact. */
 static double bf16_to_double(uint16_t bits) {
-    uint32_t u = ((uint32_t)bits) << 16;
+    uint32_t u = ((uint32_t)bits) << (MUT(19) ? 15 : 16);
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
@@ -69,7 +79,7 @@ double oracle_e4m3_to_double(uint8_t code) {
     double mag;
     if (e == 0xF && m == 0x7) return NAN;
     if (e == 0)
-        mag = ldexp((double)m / 8.0, -6);
+        mag = ldexp((double)m / 8.0, MUT(18) ? -7 : -6);
     else
         mag = ldexp(1.0 + (double)m / 8.0, e - 7);
     return s ? -mag : mag;
@@ -95,7 +105,7 @@ static int check_shape(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
 /* Last key index visible to query row i (inclusive); Sk - 1 without a mask. */
 static int64_t last_visible_key(int64_t i, int Sq, int Sk, int causal) {
     if (!causal) return (int64_t)Sk - 1;
-    int64_t last = i + ((int64_t)Sk - (int64_t)Sq);
+    int64_t last = MUT(2) ? i : i + ((int64_t)Sk - (int64_t)Sq);
     if (last > (int64_t)Sk - 1) last = (int64_t)Sk - 1;
     return last;   /* may be negative: no key visible */
 }
@@ -142,11 +152,11 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 const int r = (int)(u % n_rows);
                 const int h = (int)((u / n_rows) % Hq);
                 const int b = (int)(u / ((int64_t)n_rows * Hq));
-                const int kh = h / G;
+                const int kh = MUT(3) ? h % Hkv : h / G;
                 const int64_t i = rows ? rows[r] : r;
                 const double dq = kind == ORACLE_E4M3 ? q_descale[(int64_t)b * Hq + h] : 1.0;
                 const double dk = kind == ORACLE_E4M3 ? k_descale[(int64_t)b * Hkv + kh] : 1.0;
-                const double dv = kind == ORACLE_E4M3 ? v_descale[(int64_t)b * Hkv + kh] : 1.0;
+                const double dv = kind == ORACLE_E4M3 && !MUT(7) ? v_descale[(int64_t)b * Hkv + kh] : 1.0;
                 const int64_t qbase = (((int64_t)b * Hq + h) * Sq + i) * D;
                 const int64_t kvbase = ((int64_t)b * Hkv + kh) * (int64_t)Sk * D;
                 double* orow = o + u * D;
@@ -157,8 +167,8 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 for (int64_t j = 0; j <= last; ++j) {
                     double acc = 0.0;
                     for (int d = 0; d < D; ++d)
-                        acc += qrow[d] * load_elem(kind, k, kvbase + j * D + d, dk);
-                    s[j] = scale * acc;
+                        acc += qrow[d] * load_elem(kind, k, kvbase + (MUT(6) ? d * (int64_t)Sk + j : j * D + d), dk);
+                    s[j] = MUT(1) ? acc : scale * acc;
                     if (s[j] > m) m = s[j];
                 }
                 for (int d = 0; d < D; ++d) orow[d] = 0.0;
@@ -168,10 +178,10 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 }
                 double sum = 0.0;
                 for (int64_t j = 0; j <= last; ++j) sum += exp(s[j] - m);
-                const double L = m + log(sum);
+                const double L = MUT(4) ? log(sum) : m + log(sum);
                 lse[u] = L;
                 for (int64_t j = 0; j <= last; ++j) {
-                    const double p = exp(s[j] - L);
+                    const double p = exp(s[j] - (MUT(5) ? m : L));
                     for (int d = 0; d < D; ++d)
                         orow[d] += p * load_elem(kind, v, kvbase + j * D + d, dv);
                 }
@@ -212,10 +222,10 @@ int oracle_lse_merge(const double* o_parts, const double* lse_parts,
             const double* ob = o_parts + ((int64_t)bl * rows + r) * D;
             const double M = L > Lb ? L : Lb;
             const double w = exp(L - M);      /* 0 when L = -inf */
-            const double wb = exp(Lb - M);
+            const double wb = exp((MUT(8) ? L : Lb) - M);
             const double den = w + wb;
             for (int d = 0; d < D; ++d) orow[d] = (w * orow[d] + wb * ob[d]) / den;
-            L = M + log(den);
+            L = MUT(9) ? log(den) : M + log(den);
         }
         lse[r] = L;
     }
@@ -271,7 +281,7 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                 double* dkh = dk + kvbase;
                 double* dvh = dv + kvbase;
                 for (int64_t e = 0; e < (int64_t)Sk * D; ++e) { dkh[e] = 0.0; dvh[e] = 0.0; }
-                for (int g = 0; g < G; ++g) {
+                for (int g = 0; g < (MUT(14) ? 1 : G); ++g) {
                     const int h = kh * G + g;
                     for (int64_t i = 0; i < Sq; ++i) {
                         const int64_t qoff = (((int64_t)b * Hq + h) * Sq + i) * D;
@@ -305,17 +315,17 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                                 orow[d] += s[j] * load_elem(kind, v, kvbase + j * D + d, 1.0);
                         }
                         double delta = 0.0;
-                        for (int d = 0; d < D; ++d) delta += dorow[d] * orow[d];
+                        for (int d = 0; d < D; ++d) delta += dorow[d] * (MUT(13) ? qrow[d] : orow[d]);
                         for (int64_t j = 0; j <= last; ++j) {
                             const double p = s[j];
                             double dp = 0.0;
                             for (int d = 0; d < D; ++d)
                                 dp += dorow[d] * load_elem(kind, v, kvbase + j * D + d, 1.0);
-                            const double ds = p * (dp - delta);
+                            const double ds = p * (MUT(10) ? delta - dp : dp - delta);
                             for (int d = 0; d < D; ++d) {
                                 dqrow[d] += scale * ds * load_elem(kind, k, kvbase + j * D + d, 1.0);
-                                dkh[j * D + d] += scale * ds * qrow[d];
-                                dvh[j * D + d] += p * dorow[d];
+                                dkh[j * D + d] += (MUT(11) ? 1.0 : scale) * ds * qrow[d];
+                                dvh[j * D + d] += (MUT(12) ? ds : p) * dorow[d];
                             }
                         }
                     }
@@ -376,7 +386,7 @@ uint8_t oracle_e4m3_rne(float v) {
         code = lo;
         if (e4m3_pos_value(code) < a) {        /* between code and code + 1 */
             const double dl = a - e4m3_pos_value(code), dh = e4m3_pos_value(code + 1) - a;
-            if (dh < dl || (dh == dl && ((code + 1) & 1) == 0)) code = code + 1;
+            if (dh < dl || (dh == dl && ((code + 1) & 1) == (MUT(16) ? 1 : 0))) code = code + 1;
         }
     }
     return (uint8_t)(code | (neg << 7));
@@ -411,7 +421,7 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
                 for (int width = 1; width < 16; width *= 2)
                     for (int k = 0; k < 16; k += 2 * width) part[k] = part[k] + part[k + width];
                 const float mean = part[0] * 0.0078125f;
-                const float den = sqrtf(mean + eps32);
+                const float den = sqrtf(mean + (MUT(17) ? 0.0f : eps32));
                 r = 1.0f / den;
             }
             for (int d = 0; d < D; ++d) {
@@ -421,7 +431,7 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
                 if (fabsf(yv) > amax) amax = fabsf(yv);
             }
         }
-        const float ds = amax > 0.f ? amax / 448.0f : 1.0f;
+        const float ds = amax > 0.f ? amax / (MUT(15) ? 447.0f : 448.0f) : 1.0f;
         descale[bh] = ds;
         uint8_t* ch = codes + bh * (int64_t)S * D;
         for (int64_t i = 0; i < (int64_t)S * D; ++i) ch[i] = oracle_e4m3_rne(y[i] / ds);

@@ -31,23 +31,37 @@ _lib = None
 F64, BF16, E4M3 = 0, 1, 2
 
 
+def _compile(out: str, mutant: int = 0) -> None:
+    tmp = out + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
+           "-Wall", "-shared", "-fPIC", "-DORACLE_MUTANT=%d" % mutant, "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+
+
 def build(force: bool = False) -> str:
     """Compile attn_oracle.c into liboracle.so next to it (gcc, OpenMP, no fast-math)."""
     if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
         return _LIB
-    tmp = _LIB + ".tmp.%d" % os.getpid()
-    cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
-           "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
+    _compile(_LIB)
     return _LIB
+
+
+def build_mutant(mutant: int, out: str) -> str:
+    """A build with planted mistake number `mutant` (> 0) at `out`, for the test
+    that checks the pins catch it; loaded instead of liboracle.so when the
+    environment variable ORACLE_LIB names it."""
+    if mutant <= 0:
+        raise ValueError("mutant numbers start at 1")
+    _compile(out, mutant)
+    return out
 
 
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            lib = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
             vp, dp, i64p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
             ci, cd = ctypes.c_int, ctypes.c_double
             lib.oracle_attn_fwd.argtypes = [ci, vp, vp, vp, dp, dp, dp, ci, ci, ci, ci, ci, ci,
