@@ -395,6 +395,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
   }
 
   const long long rows = (long long)B * Hq * Sq;
+  if ((rows + 7) / 8 > INT_MAX) return HATTN_EUNSUPPORTED;   // the merge takes 8 rows per CTA in grid x
   float* o_parts = reinterpret_cast<float*>(workspace);
   float* lse_parts = o_parts + (size_t)n_blocks * rows * kHeadDim;
   for (int first = 0; first < n_blocks; first += kMaxKvBlocks) {
