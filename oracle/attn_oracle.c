@@ -77,7 +77,7 @@ double oracle_e4m3_to_double(uint8_t code) {
     int e = (code >> 3) & 0xF;
     int m = code & 0x7;
     double mag;
-    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0xF && m == 0x7 && !MUT(29)) return NAN;
     if (e == 0)
         mag = ldexp((double)m / 8.0, MUT(18) ? -7 : -6);
     else
@@ -105,7 +105,7 @@ static int check_shape(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
 /* Last key index visible to query row i (inclusive); Sk - 1 without a mask. */
 static int64_t last_visible_key(int64_t i, int Sq, int Sk, int causal) {
     if (!causal) return (int64_t)Sk - 1;
-    int64_t last = MUT(2) ? i : i + ((int64_t)Sk - (int64_t)Sq);
+    int64_t last = MUT(2) ? i : i + ((int64_t)Sk - (int64_t)Sq) - (MUT(20) ? 1 : 0);
     if (last > (int64_t)Sk - 1) last = (int64_t)Sk - 1;
     return last;   /* may be negative: no key visible */
 }
@@ -294,7 +294,7 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                             orow[d] = 0.0;
                             dqrow[d] = 0.0;
                         }
-                        const int64_t last = last_visible_key(i, Sq, Sk, causal);
+                        const int64_t last = last_visible_key(i, Sq, Sk, MUT(25) ? 0 : causal);
                         if (last < 0) { lse[lidx] = -INFINITY; continue; }
                         double m = -INFINITY;
                         for (int64_t j = 0; j <= last; ++j) {
@@ -323,7 +323,7 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                                 dp += dorow[d] * load_elem(kind, v, kvbase + j * D + d, 1.0);
                             const double ds = p * (MUT(10) ? delta - dp : dp - delta);
                             for (int d = 0; d < D; ++d) {
-                                dqrow[d] += scale * ds * load_elem(kind, k, kvbase + j * D + d, 1.0);
+                                dqrow[d] += (MUT(27) ? 1.0 : scale) * ds * load_elem(kind, k, kvbase + j * D + d, 1.0);
                                 dkh[j * D + d] += (MUT(11) ? 1.0 : scale) * ds * qrow[d];
                                 dvh[j * D + d] += (MUT(12) ? ds : p) * dorow[d];
                             }
@@ -420,7 +420,7 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
                 }
                 for (int width = 1; width < 16; width *= 2)
                     for (int k = 0; k < 16; k += 2 * width) part[k] = part[k] + part[k + width];
-                const float mean = part[0] * 0.0078125f;
+                const float mean = part[0] * (MUT(22) ? 1.0f / 127.0f : 0.0078125f);
                 const float den = sqrtf(mean + (MUT(17) ? 0.0f : eps32));
                 r = 1.0f / den;
             }
@@ -428,7 +428,7 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
                 const float v = (float)bf16_to_double(xh[s * D + d]);
                 const float yv = rmsnorm ? v * r : v;
                 y[s * D + d] = yv;
-                if (fabsf(yv) > amax) amax = fabsf(yv);
+                if (fabsf(MUT(21) ? v : yv) > amax) amax = fabsf(MUT(21) ? v : yv);
             }
         }
         const float ds = amax > 0.f ? amax / (MUT(15) ? 447.0f : 448.0f) : 1.0f;

@@ -36,6 +36,12 @@ MUTANTS = {
     17: "RMS norm without eps",
     18: "e4m3 subnormals decoded at 2^-7 instead of 2^-6",
     19: "bf16 widened with a 15-bit shift",
+    20: "causal mask one key short (j < i + Sk - Sq)",
+    21: "head maximum taken before the RMS norm",
+    22: "RMS mean over 127 instead of 128",
+    25: "backward without the causal mask",
+    27: "dQ without the scale",
+    29: "e4m3 NaN code decoded as 480",
 }
 
 
