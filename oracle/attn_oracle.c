@@ -153,8 +153,8 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 const int h = (int)((u / n_rows) % Hq);
                 const int b = (int)(u / ((int64_t)n_rows * Hq));
                 const int kh = MUT(3) ? h % Hkv : h / G;
-                const int64_t i = rows ? rows[r] : r;
-                const double dq = kind == ORACLE_E4M3 ? q_descale[(int64_t)b * Hq + h] : 1.0;
+                const int64_t i = rows && !MUT(34) ? rows[r] : r;
+                const double dq = kind == ORACLE_E4M3 ? q_descale[MUT(30) ? (int64_t)b * Hkv + kh : (int64_t)b * Hq + h] : 1.0;
                 const double dk = kind == ORACLE_E4M3 ? k_descale[(int64_t)b * Hkv + kh] : 1.0;
                 const double dv = kind == ORACLE_E4M3 && !MUT(7) ? v_descale[(int64_t)b * Hkv + kh] : 1.0;
                 const int64_t qbase = (((int64_t)b * Hq + h) * Sq + i) * D;
@@ -224,7 +224,7 @@ int oracle_lse_merge(const double* o_parts, const double* lse_parts,
             const double w = exp(L - M);      /* 0 when L = -inf */
             const double wb = exp((MUT(8) ? L : Lb) - M);
             const double den = w + wb;
-            for (int d = 0; d < D; ++d) orow[d] = (w * orow[d] + wb * ob[d]) / den;
+            for (int d = 0; d < D; ++d) orow[d] = (w * orow[d] + wb * ob[d]) / (MUT(31) ? 1.0 : den);
             L = MUT(9) ? log(den) : M + log(den);
         }
         lse[r] = L;
@@ -371,7 +371,7 @@ static double e4m3_pos_value(int code) { return oracle_e4m3_to_double((uint8_t)c
 
 uint8_t oracle_e4m3_rne(float v) {
     if (isnan(v)) return 0x7F;
-    const int neg = signbit(v) ? 1 : 0;
+    const int neg = (MUT(32) ? v < 0.0f : signbit(v)) ? 1 : 0;
     const double a = fabs((double)v);
     int code;
     if (a >= 448.0) {

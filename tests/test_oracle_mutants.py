@@ -42,6 +42,10 @@ MUTANTS = {
     25: "backward without the causal mask",
     27: "dQ without the scale",
     29: "e4m3 NaN code decoded as 480",
+    30: "q_descale indexed by the KV head",
+    31: "merged O not divided by the sum of the weights",
+    32: "negative values that round to zero lose their sign bit",
+    34: "sampled query rows ignored (row r evaluated instead of rows[r])",
 }
 
 

@@ -282,10 +282,15 @@ def test_bf16_storage_is_exact_widening(oracle_mod):
     np.testing.assert_array_equal(lse, lse2)
 
 
-def test_e4m3_storage_applies_per_head_descale(oracle_mod):
-    g = torch.Generator().manual_seed(55)
-    x = [torch.randn(2, 3, 21, 16, generator=g).to(torch.bfloat16) for _ in range(3)]
+@pytest.mark.parametrize("Hq,Hkv", [(3, 3), (6, 2)])
+def test_e4m3_storage_applies_per_head_descale(oracle_mod, Hq, Hkv):
+    # heads of different magnitudes, so every (batch, head) has its own descale;
+    # with grouped heads the query descales are per query head, not per KV head
+    g = torch.Generator().manual_seed(55 + Hq)
+    mag = lambda H: torch.arange(1, 2 * H + 1, dtype=torch.float32).reshape(2, H, 1, 1)
+    x = [(torch.randn(2, H, 21, 16, generator=g) * mag(H)).to(torch.bfloat16) for H in (Hq, Hkv, Hkv)]
     (q8, dq), (k8, dk), (v8, dv) = (quantize_e4m3_per_head(t) for t in x)
+    assert len(set(dq.flatten().tolist())) == 2 * Hq
     o, lse = oracle_mod.attn_fwd(e4m3_bits(q8), e4m3_bits(k8), e4m3_bits(v8), 0.25,
                                  descales=(dq.numpy(), dk.numpy(), dv.numpy()))
     deq = [c.to(torch.float64) * d.double()[:, :, None, None] for c, d in ((q8, dq), (k8, dk), (v8, dv))]
