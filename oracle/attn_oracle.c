@@ -282,7 +282,7 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                 double* dvh = dv + kvbase;
                 for (int64_t e = 0; e < (int64_t)Sk * D; ++e) { dkh[e] = 0.0; dvh[e] = 0.0; }
                 for (int g = 0; g < (MUT(14) ? 1 : G); ++g) {
-                    const int h = kh * G + g;
+                    const int h = MUT(47) ? kh + g * Hkv : kh * G + g;
                     for (int64_t i = 0; i < Sq; ++i) {
                         const int64_t qoff = (((int64_t)b * Hq + h) * Sq + i) * D;
                         const int64_t lidx = ((int64_t)b * Hq + h) * Sq + i;
@@ -315,7 +315,7 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                                 orow[d] += s[j] * load_elem(kind, v, kvbase + j * D + d, 1.0);
                         }
                         double delta = 0.0;
-                        for (int d = 0; d < D; ++d) delta += dorow[d] * (MUT(13) ? qrow[d] : orow[d]);
+                        for (int d = 0; d < (MUT(36) ? D / 2 : D); ++d) delta += dorow[d] * (MUT(13) ? qrow[d] : orow[d]);
                         for (int64_t j = 0; j <= last; ++j) {
                             const double p = s[j];
                             double dp = 0.0;
@@ -422,13 +422,13 @@ int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int 
                     for (int k = 0; k < 16; k += 2 * width) part[k] = part[k] + part[k + width];
                 const float mean = part[0] * (MUT(22) ? 1.0f / 127.0f : 0.0078125f);
                 const float den = sqrtf(mean + (MUT(17) ? 0.0f : eps32));
-                r = 1.0f / den;
+                r = MUT(42) ? 1.0f / (sqrtf(mean) + eps32) : 1.0f / den;
             }
             for (int d = 0; d < D; ++d) {
                 const float v = (float)bf16_to_double(xh[s * D + d]);
                 const float yv = rmsnorm ? v * r : v;
                 y[s * D + d] = yv;
-                if (fabsf(MUT(21) ? v : yv) > amax) amax = fabsf(MUT(21) ? v : yv);
+                if (!(MUT(41) && s == S - 1) && fabsf(MUT(21) ? v : yv) > amax) amax = fabsf(MUT(21) ? v : yv);
             }
         }
         const float ds = amax > 0.f ? amax / (MUT(15) ? 447.0f : 448.0f) : 1.0f;

@@ -46,6 +46,10 @@ MUTANTS = {
     31: "merged O not divided by the sum of the weights",
     32: "negative values that round to zero lose their sign bit",
     34: "sampled query rows ignored (row r evaluated instead of rows[r])",
+    36: "Delta over the first half of the head dimension only",
+    41: "head maximum skips the last row",
+    42: "RMS factor 1 / (sqrt(mean) + eps) instead of 1 / sqrt(mean + eps)",
+    47: "backward groups query heads kv + g * Hkv instead of kv * G + g",
 }
 
 
