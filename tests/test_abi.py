@@ -38,6 +38,53 @@ def test_library_exports_every_declared_symbol(h):
         assert s in h.EXPORTED
 
 
+def declared_signatures():
+    """{name: [C parameter types]} of every HATTN_API function in hattn.h."""
+    txt = open(os.path.join(ROOT, "include", "hattn.h")).read()
+    txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)
+    out = {}
+    for m in re.finditer(r"HATTN_API\s+([\w\s\*]+?)\b(attn_\w+)\s*\(([^)]*)\)\s*;", txt):
+        params = [" ".join(p.split()) for p in m.group(3).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(2)] = (" ".join(m.group(1).split()), params)
+    return out
+
+
+def _ctype_of(decl):
+    """The ctypes type of a C declaration "type name" ("ptr" for any pointer)."""
+    import ctypes as C
+
+    if "*" in decl:
+        return "ptr"
+    base = " ".join(w for w in decl.split()[:-1] if w != "const")    # drop the name
+    table = {"int": C.c_int, "float": C.c_float, "double": C.c_double, "size_t": C.c_size_t,
+             "unsigned int": C.c_uint}
+    assert base in table, "unmapped C type: %r" % decl
+    return table[base]
+
+
+def test_binding_argtypes_match_the_header(h):
+    """Every ctypes prototype in the binding has the header's parameter count and
+    types (pointers as pointers, int/float/double/size_t/unsigned as such)."""
+    import ctypes as C
+
+    sigs = declared_signatures()
+    assert set(sigs) == set(h.EXPORTED)
+    for name, (ret, params) in sigs.items():
+        fn = getattr(h.lib, name)
+        assert len(fn.argtypes) == len(params), (name, fn.argtypes, params)
+        for c_decl, ct in zip(params, fn.argtypes):
+            want = _ctype_of(c_decl)
+            if want == "ptr":
+                assert ct in (C.c_void_p, C.c_char_p) or issubclass(ct, C._Pointer), (name, c_decl, ct)
+            else:
+                assert ct is want, (name, c_decl, ct)
+        r = _ctype_of(ret + " result")
+        if r == "ptr":
+            assert fn.restype in (C.c_void_p, C.c_char_p), (name, ret, fn.restype)
+        else:
+            assert fn.restype is r, (name, ret, fn.restype)
+
+
 def test_workspace_sizes(h):
     assert h.kvblocks_workspace_size(1, 40, 1560, 128, 21) == 0          # folded in one launch
     assert h.kvblocks_workspace_size(1, 40, 1560, 128, 40) == 40 * 40 * 1560 * 129 * 4
