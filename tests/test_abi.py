@@ -38,6 +38,23 @@ def test_library_exports_every_declared_symbol(h):
         assert s in h.EXPORTED
 
 
+def test_library_exports_nothing_undeclared(h):
+    """The attn_* entry points in the library's dynamic symbol table are exactly
+    those hattn.h declares (read with nm from the library built here)."""
+    import shutil
+    import subprocess
+
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    from head_attention_qk_b200 import hattn
+
+    out = subprocess.run([nm, "-D", "--defined-only", hattn.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted({line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("attn_")})
+    assert exported == declared_symbols()
+
+
 def declared_signatures():
     """{name: [C parameter types]} of every HATTN_API function in hattn.h."""
     txt = open(os.path.join(ROOT, "include", "hattn.h")).read()
