@@ -61,7 +61,7 @@ def _cp_worker(rank, world, port, out):
     import sys
 
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
-    from head_attention_qk_b200.context_parallel import gather_kv_shards
+    from head_attention_qk_b200.context_parallel import attn_fwd_context_parallel, gather_kv_shards
 
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -80,7 +80,16 @@ def _cp_worker(rank, world, port, out):
             refused = False
         except ValueError:
             refused = True
-        out[rank] = (ok, refused)
+        # the attention itself runs only in the CUDA library: CPU tensors are
+        # refused after the exchange (the same steps on every rank), never computed
+        q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+        kv = torch.zeros(1, 2, 6, 128, dtype=torch.bfloat16)
+        try:
+            attn_fwd_context_parallel(q, kv, kv)
+            no_fallback = False
+        except ValueError as e:
+            no_fallback = "CUDA" in str(e)
+        out[rank] = (ok, refused, no_fallback)
     finally:
         dist.destroy_process_group()
 
@@ -91,4 +100,4 @@ def test_context_parallel_gather_order_two_ranks():
     manager = ctx.Manager()
     out = manager.dict()
     mp.start_processes(_cp_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
-    assert out[0] == (True, True) and out[1] == (True, True)
+    assert out[0] == (True, True, True) and out[1] == (True, True, True)
