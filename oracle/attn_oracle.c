@@ -7,12 +7,10 @@
  * code, header, table or constant with the CUDA library under
  * head_attention_qk_b200/csrc, and it never includes or links it.
  *
- * Everything is computed in double precision with plain loops (no blocking, no
- * fusion, no reordering beyond the definition), except the e4m3 prologue's
- * RMS norm, which takes the kernel's fp32 steps in a stated order because its
- * values decide integer codes (see oracle_quantize_e4m3).  OpenMP splits independent
- * (batch, head, query-row) units across host threads; each unit is summed in a
- * fixed ascending order, so results do not depend on the thread count.
+ * Everything is computed in double precision with plain loops: no blocking,
+ * no fusion, no reordering beyond the definition.  OpenMP splits independent
+ * (batch, head, query-row) units across host threads; each unit is summed in
+ * a fixed ascending order, so results do not depend on the thread count.
  *
  * Sources (web pages of the subject, cited by title and section):
  *  - AITER PR #2911 "F8 fmha ASM gfx950", Test Result: the operation is
@@ -26,7 +24,7 @@
  *    Qwen3-8B heads Hq=32, Hkv=8, D=128 (ROCm Validation table).
  *  - FlashDreams PR #486 "flashdreams.accelerated API v0", section 1.2
  *    Optimized MHA: streaming self-attention over a block KV cache and static
- *    cross-attention.
+ *    cross-attention; sections 1.1-1.2 for the e4m3 prologue.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - layout is [B, H, S, D] contiguous; LSE is [B, Hq, Sq] in natural log;
@@ -36,6 +34,11 @@
  *  - a row that sees no key has O = 0 and LSE = -inf;
  *  - fp8 inputs are OCP e4m3fn codes; the dequantized value is
  *    decode(code) * descale[b, h], with one descale per (batch, head).
+ *
+ * The pin suite checks this file against closed forms, brute force, library
+ * routines and invariants, and checks that the pins catch plausible mistakes
+ * by applying text patches to a copy of this source (tests/oracle_mutants.py);
+ * nothing of that machinery lives here.
  */
 #include <math.h>
 #include <stdint.h>
@@ -46,23 +49,13 @@
 #include <omp.h>
 #endif
 
-/* Planted mistakes for the pin suite's own test (tests/test_oracle_mutants.py):
- * built with -DORACLE_MUTANT=n (n > 0), MUT(n) is true at one site and the
- * oracle computes something plausible but wrong there; every pin run against
- * such a build must fail.  The normal build has ORACLE_MUTANT 0, where every
- * MUT() is the constant 0 and the code is the definition. */
-#ifndef ORACLE_MUTANT
-#define ORACLE_MUTANT 0
-#endif
-#define MUT(n) (ORACLE_MUTANT == (n))
-
 /* Storage kinds of the input arrays.  The oracle reads the same bytes the GPU
  * reads and widens them exactly to double. */
 enum { ORACLE_F64 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
 
 /* bfloat16: the upper 16 bits of an IEEE-754 binary32.  Widening is exact. */
 static double bf16_to_double(uint16_t bits) {
-    uint32_t u = ((uint32_t)bits) << (MUT(19) ? 15 : 16);
+    uint32_t u = ((uint32_t)bits) << 16;
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
@@ -77,9 +70,9 @@ double oracle_e4m3_to_double(uint8_t code) {
     int e = (code >> 3) & 0xF;
     int m = code & 0x7;
     double mag;
-    if (e == 0xF && m == 0x7 && !MUT(29)) return NAN;
+    if (e == 0xF && m == 0x7) return NAN;
     if (e == 0)
-        mag = ldexp((double)m / 8.0, MUT(18) ? -7 : -6);
+        mag = ldexp((double)m / 8.0, -6);
     else
         mag = ldexp(1.0 + (double)m / 8.0, e - 7);
     return s ? -mag : mag;
@@ -105,7 +98,7 @@ static int check_shape(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
 /* Last key index visible to query row i (inclusive); Sk - 1 without a mask. */
 static int64_t last_visible_key(int64_t i, int Sq, int Sk, int causal) {
     if (!causal) return (int64_t)Sk - 1;
-    int64_t last = MUT(2) ? i : i + ((int64_t)Sk - (int64_t)Sq) - (MUT(20) ? 1 : 0);
+    int64_t last = i + ((int64_t)Sk - (int64_t)Sq);
     if (last > (int64_t)Sk - 1) last = (int64_t)Sk - 1;
     return last;   /* may be negative: no key visible */
 }
@@ -152,11 +145,11 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 const int r = (int)(u % n_rows);
                 const int h = (int)((u / n_rows) % Hq);
                 const int b = (int)(u / ((int64_t)n_rows * Hq));
-                const int kh = MUT(3) ? h % Hkv : h / G;
-                const int64_t i = rows && !MUT(34) ? rows[r] : r;
-                const double dq = kind == ORACLE_E4M3 ? q_descale[MUT(30) ? (int64_t)b * Hkv + kh : (int64_t)b * Hq + h] : 1.0;
+                const int kh = h / G;
+                const int64_t i = rows ? rows[r] : r;
+                const double dq = kind == ORACLE_E4M3 ? q_descale[(int64_t)b * Hq + h] : 1.0;
                 const double dk = kind == ORACLE_E4M3 ? k_descale[(int64_t)b * Hkv + kh] : 1.0;
-                const double dv = kind == ORACLE_E4M3 && !MUT(7) ? v_descale[(int64_t)b * Hkv + kh] : 1.0;
+                const double dv = kind == ORACLE_E4M3 ? v_descale[(int64_t)b * Hkv + kh] : 1.0;
                 const int64_t qbase = (((int64_t)b * Hq + h) * Sq + i) * D;
                 const int64_t kvbase = ((int64_t)b * Hkv + kh) * (int64_t)Sk * D;
                 double* orow = o + u * D;
@@ -167,8 +160,8 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 for (int64_t j = 0; j <= last; ++j) {
                     double acc = 0.0;
                     for (int d = 0; d < D; ++d)
-                        acc += qrow[d] * load_elem(kind, k, kvbase + (MUT(6) ? d * (int64_t)Sk + j : j * D + d), dk);
-                    s[j] = MUT(1) ? acc : scale * acc;
+                        acc += qrow[d] * load_elem(kind, k, kvbase + j * D + d, dk);
+                    s[j] = scale * acc;
                     if (s[j] > m) m = s[j];
                 }
                 for (int d = 0; d < D; ++d) orow[d] = 0.0;
@@ -178,10 +171,10 @@ int oracle_attn_fwd(int kind, const void* q, const void* k, const void* v,
                 }
                 double sum = 0.0;
                 for (int64_t j = 0; j <= last; ++j) sum += exp(s[j] - m);
-                const double L = MUT(4) ? log(sum) : m + log(sum);
+                const double L = m + log(sum);
                 lse[u] = L;
                 for (int64_t j = 0; j <= last; ++j) {
-                    const double p = exp(s[j] - (MUT(5) ? m : L));
+                    const double p = exp(s[j] - L);
                     for (int d = 0; d < D; ++d)
                         orow[d] += p * load_elem(kind, v, kvbase + j * D + d, dv);
                 }
@@ -222,10 +215,10 @@ int oracle_lse_merge(const double* o_parts, const double* lse_parts,
             const double* ob = o_parts + ((int64_t)bl * rows + r) * D;
             const double M = L > Lb ? L : Lb;
             const double w = exp(L - M);      /* 0 when L = -inf */
-            const double wb = exp((MUT(8) ? L : Lb) - M);
+            const double wb = exp(Lb - M);
             const double den = w + wb;
-            for (int d = 0; d < D; ++d) orow[d] = (w * orow[d] + wb * ob[d]) / (MUT(31) ? 1.0 : den);
-            L = MUT(9) ? log(den) : M + log(den);
+            for (int d = 0; d < D; ++d) orow[d] = (w * orow[d] + wb * ob[d]) / den;
+            L = M + log(den);
         }
         lse[r] = L;
     }
@@ -266,10 +259,10 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
 
 #pragma omp parallel
     {
-        double* s = (double*)malloc(sizeof(double) * (size_t)Sk);
+        double* p = (double*)malloc(sizeof(double) * (size_t)Sk);
         double* qrow = (double*)malloc(sizeof(double) * (size_t)D);
         double* dorow = (double*)malloc(sizeof(double) * (size_t)D);
-        if (!s || !qrow || !dorow) {
+        if (!p || !qrow || !dorow) {
 #pragma omp atomic write
             failed = 1;
         } else {
@@ -281,8 +274,8 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                 double* dkh = dk + kvbase;
                 double* dvh = dv + kvbase;
                 for (int64_t e = 0; e < (int64_t)Sk * D; ++e) { dkh[e] = 0.0; dvh[e] = 0.0; }
-                for (int g = 0; g < (MUT(14) ? 1 : G); ++g) {
-                    const int h = MUT(47) ? kh + g * Hkv : kh * G + g;
+                for (int g = 0; g < G; ++g) {
+                    const int h = kh * G + g;
                     for (int64_t i = 0; i < Sq; ++i) {
                         const int64_t qoff = (((int64_t)b * Hq + h) * Sq + i) * D;
                         const int64_t lidx = ((int64_t)b * Hq + h) * Sq + i;
@@ -294,45 +287,45 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
                             orow[d] = 0.0;
                             dqrow[d] = 0.0;
                         }
-                        const int64_t last = last_visible_key(i, Sq, Sk, MUT(25) ? 0 : causal);
+                        const int64_t last = last_visible_key(i, Sq, Sk, causal);
                         if (last < 0) { lse[lidx] = -INFINITY; continue; }
+                        /* scores, then LSE with the row maximum */
                         double m = -INFINITY;
                         for (int64_t j = 0; j <= last; ++j) {
-                            double acc = 0.0;
+                            double sij = 0.0;
                             for (int d = 0; d < D; ++d)
-                                acc += qrow[d] * load_elem(kind, k, kvbase + j * D + d, 1.0);
-                            s[j] = scale * acc;
-                            if (s[j] > m) m = s[j];
+                                sij += qrow[d] * load_elem(kind, k, kvbase + j * D + d, 1.0);
+                            p[j] = scale * sij;
+                            if (p[j] > m) m = p[j];
                         }
-                        double sum = 0.0;
-                        for (int64_t j = 0; j <= last; ++j) sum += exp(s[j] - m);
-                        const double L = m + log(sum);
-                        lse[lidx] = L;
-                        /* P_ij overwrites s_j; O_i = sum_j P_ij v_j */
+                        double z = 0.0;
+                        for (int64_t j = 0; j <= last; ++j) z += exp(p[j] - m);
+                        const double Lrow = m + log(z);
+                        lse[lidx] = Lrow;
+                        /* P_ij overwrites s_ij; O_i = sum_j P_ij v_j */
                         for (int64_t j = 0; j <= last; ++j) {
-                            s[j] = exp(s[j] - L);
+                            p[j] = exp(p[j] - Lrow);
                             for (int d = 0; d < D; ++d)
-                                orow[d] += s[j] * load_elem(kind, v, kvbase + j * D + d, 1.0);
+                                orow[d] += p[j] * load_elem(kind, v, kvbase + j * D + d, 1.0);
                         }
                         double delta = 0.0;
-                        for (int d = 0; d < (MUT(36) ? D / 2 : D); ++d) delta += dorow[d] * (MUT(13) ? qrow[d] : orow[d]);
+                        for (int d = 0; d < D; ++d) delta += dorow[d] * orow[d];
                         for (int64_t j = 0; j <= last; ++j) {
-                            const double p = s[j];
                             double dp = 0.0;
                             for (int d = 0; d < D; ++d)
                                 dp += dorow[d] * load_elem(kind, v, kvbase + j * D + d, 1.0);
-                            const double ds = p * (MUT(10) ? delta - dp : dp - delta);
+                            const double ds = p[j] * (dp - delta);
                             for (int d = 0; d < D; ++d) {
-                                dqrow[d] += (MUT(27) ? 1.0 : scale) * ds * load_elem(kind, k, kvbase + j * D + d, 1.0);
-                                dkh[j * D + d] += (MUT(11) ? 1.0 : scale) * ds * qrow[d];
-                                dvh[j * D + d] += (MUT(12) ? ds : p) * dorow[d];
+                                dqrow[d] += scale * ds * load_elem(kind, k, kvbase + j * D + d, 1.0);
+                                dkh[j * D + d] += scale * ds * qrow[d];
+                                dvh[j * D + d] += p[j] * dorow[d];
                             }
                         }
                     }
                 }
             }
         }
-        free(s);
+        free(p);
         free(qrow);
         free(dorow);
     }
@@ -347,32 +340,26 @@ int oracle_attn_bwd(int kind, const void* q, const void* k, const void* v,
  * clamp to the e4m3fn range +-448 as VeOmni PR #1363 describes its quantizers.
  * The pages give no formula; the readings (listed in the design notes) are:
  * the scale slice is one (batch, head); the optional normalisation is a plain
- * RMS over the head dimension with eps and no weight; and each step is fixed
- * in precision and order, so that every code is a function of the input:
- *   ss      = sum of the row's x_d^2 in fp32, each operation rounded to nearest:
- *             sixteen partial sums s_k over d = 8k .. 8k+7 (ascending d), then
- *             added pairwise, neighbours first: (s0 + s1), (s2 + s3), ...,
- *             ((s0 + s1) + (s2 + s3)), ... down to one value (D = 128)
- *   r       = 1 / sqrt(ss / 128 + eps)    (fp32: multiply by 2^-7, add the fp32
- *             eps, square root and division, each correctly rounded)
- *   y_d     = x_d * r rounded to fp32; y = x without the normalisation
- * (the norm's precision is the kernel's: the pages fix none, and these values
- * decide integer codes, so both sides take them in the same fp32 steps)
- *   amax    = max |y| over the head's S x D values       (fp32)
- *   descale = amax / 448 in fp32, or 1 when amax == 0
- *   code    = e4m3 of y / descale (fp32 quotient), rounded to nearest with
- *             ties to the even code, saturating at +-448; the sign bit is the
- *             quotient's.
+ * RMS over the head dimension with eps and no weight.  In exact arithmetic
+ * (here fp64), per head:
+ *   r_s     = 1 / sqrt( (1/D) sum_d x_sd^2 + eps )   for each row s (1 without
+ *             the normalisation)
+ *   y_sd    = x_sd * r_s
+ *   amax    = max |y| over the head's S x D values
+ *   descale = amax / 448, as the nearest fp32 (the descales travel as fp32),
+ *             or 1 when amax == 0
+ *   code    = e4m3 of y_sd / descale, rounded to nearest with ties to the
+ *             even code, saturating at +-448; the sign bit is the quotient's.
  */
 
-/* The 127 non-negative finite e4m3fn values in code order (codes 0x00..0x7E),
+/* The non-negative finite e4m3fn values in code order (codes 0x00..0x7E),
  * from the format definition; ascending. */
 static double e4m3_pos_value(int code) { return oracle_e4m3_to_double((uint8_t)code); }
 
-uint8_t oracle_e4m3_rne(float v) {
+uint8_t oracle_e4m3_rne(double v) {
     if (isnan(v)) return 0x7F;
-    const int neg = (MUT(32) ? v < 0.0f : signbit(v)) ? 1 : 0;
-    const double a = fabs((double)v);
+    const int neg = signbit(v) ? 1 : 0;
+    const double a = fabs(v);
     int code;
     if (a >= 448.0) {
         code = 0x7E;                           /* saturate */
@@ -386,55 +373,51 @@ uint8_t oracle_e4m3_rne(float v) {
         code = lo;
         if (e4m3_pos_value(code) < a) {        /* between code and code + 1 */
             const double dl = a - e4m3_pos_value(code), dh = e4m3_pos_value(code + 1) - a;
-            if (dh < dl || (dh == dl && ((code + 1) & 1) == (MUT(16) ? 1 : 0))) code = code + 1;
+            if (dh < dl || (dh == dl && ((code + 1) & 1) == 0)) code = code + 1;
         }
     }
     return (uint8_t)(code | (neg << 7));
 }
 
-int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, int B, int H, int S, int D,
-                         int rmsnorm, double eps) {
+/* x: [B,H,S,D] bf16 bit patterns.  codes: [B,H,S,D]; descale: [B*H] fp32.
+ * quotient (optional, may be NULL): [B,H,S,D] doubles, y / descale before
+ * rounding, for tests that need the distance to a rounding boundary. */
+int oracle_quantize_e4m3(const uint16_t* x, uint8_t* codes, float* descale, double* quotient,
+                         int B, int H, int S, int D, int rmsnorm, double eps) {
     if (B <= 0 || H <= 0 || S <= 0 || D <= 0 || !x || !codes || !descale) return -1;
-    if (rmsnorm && D != 128) return -1;
-    const float eps32 = (float)eps;
     const int64_t heads = (int64_t)B * H;
+    const int64_t n = (int64_t)S * D;
     int failed = 0;
     #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t bh = 0; bh < heads; ++bh) {
-        float* y = (float*)malloc(sizeof(float) * (size_t)S * D);
+        double* y = (double*)malloc(sizeof(double) * (size_t)n);
         if (!y) { failed = 1; continue; }
-        const uint16_t* xh = x + bh * (int64_t)S * D;
-        float amax = 0.f;
+        const uint16_t* xh = x + bh * n;
+        double amax = 0.0;
         for (int64_t s = 0; s < S; ++s) {
-            float r = 1.0f;
+            double r = 1.0;
             if (rmsnorm) {
-                volatile float part[16];               /* volatile: every step rounded to fp32 */
-                for (int k = 0; k < 16; ++k) {
-                    float acc = 0.0f;
-                    for (int t = 0; t < 8; ++t) {
-                        const float v = (float)bf16_to_double(xh[s * D + 8 * k + t]);
-                        const float sq = v * v;
-                        acc = acc + sq;
-                    }
-                    part[k] = acc;
+                double ss = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double xv = bf16_to_double(xh[s * D + d]);
+                    ss += xv * xv;
                 }
-                for (int width = 1; width < 16; width *= 2)
-                    for (int k = 0; k < 16; k += 2 * width) part[k] = part[k] + part[k + width];
-                const float mean = part[0] * (MUT(22) ? 1.0f / 127.0f : 0.0078125f);
-                const float den = sqrtf(mean + (MUT(17) ? 0.0f : eps32));
-                r = MUT(42) ? 1.0f / (sqrtf(mean) + eps32) : 1.0f / den;
+                r = 1.0 / sqrt(ss / D + eps);
             }
             for (int d = 0; d < D; ++d) {
-                const float v = (float)bf16_to_double(xh[s * D + d]);
-                const float yv = rmsnorm ? v * r : v;
+                const double yv = bf16_to_double(xh[s * D + d]) * r;
                 y[s * D + d] = yv;
-                if (!(MUT(41) && s == S - 1) && fabsf(MUT(21) ? v : yv) > amax) amax = fabsf(MUT(21) ? v : yv);
+                if (fabs(yv) > amax) amax = fabs(yv);
             }
         }
-        const float ds = amax > 0.f ? amax / (MUT(15) ? 447.0f : 448.0f) : 1.0f;
+        const float ds = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
         descale[bh] = ds;
-        uint8_t* ch = codes + bh * (int64_t)S * D;
-        for (int64_t i = 0; i < (int64_t)S * D; ++i) ch[i] = oracle_e4m3_rne(y[i] / ds);
+        uint8_t* ch = codes + bh * n;
+        for (int64_t i = 0; i < n; ++i) {
+            const double qv = y[i] / (double)ds;
+            ch[i] = oracle_e4m3_rne(qv);
+            if (quotient) quotient[bh * n + i] = qv;
+        }
         free(y);
     }
     return failed ? -2 : 0;

@@ -31,30 +31,27 @@ _lib = None
 F64, BF16, E4M3 = 0, 1, 2
 
 
-def _compile(out: str, mutant: int = 0) -> None:
+def compile_library(src: str, out: str) -> str:
+    """Compile a C source of the oracle into a shared library at `out` (gcc,
+    OpenMP, no fast-math, no contraction of multiply-adds)."""
     tmp = out + ".tmp.%d" % os.getpid()
     cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
-           "-Wall", "-shared", "-fPIC", "-DORACLE_MUTANT=%d" % mutant, "-o", tmp, _SRC, "-lm"]
+           "-Wall", "-shared", "-fPIC", "-o", tmp, src, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
+    return out
+
+
+def source_path() -> str:
+    """Path of the oracle's C source."""
+    return _SRC
 
 
 def build(force: bool = False) -> str:
     """Compile attn_oracle.c into liboracle.so next to it (gcc, OpenMP, no fast-math)."""
     if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
         return _LIB
-    _compile(_LIB)
-    return _LIB
-
-
-def build_mutant(mutant: int, out: str) -> str:
-    """A build with planted mistake number `mutant` (> 0) at `out`, for the test
-    that checks the pins catch it; loaded instead of liboracle.so when the
-    environment variable ORACLE_LIB names it."""
-    if mutant <= 0:
-        raise ValueError("mutant numbers start at 1")
-    _compile(out, mutant)
-    return out
+    return compile_library(_SRC, _LIB)
 
 
 def _load():
@@ -76,9 +73,9 @@ def _load():
             lib.oracle_e4m3_to_double.restype = cd
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ci
-            lib.oracle_e4m3_rne.argtypes = [ctypes.c_float]
+            lib.oracle_e4m3_rne.argtypes = [ctypes.c_double]
             lib.oracle_e4m3_rne.restype = ctypes.c_uint8
-            lib.oracle_quantize_e4m3.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd]
+            lib.oracle_quantize_e4m3.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, cd]
             lib.oracle_quantize_e4m3.restype = ci
             _lib = lib
     return _lib
@@ -107,24 +104,26 @@ def e4m3_to_double(code: int) -> float:
 
 
 def e4m3_rne(v: float) -> int:
-    """e4m3fn code of an fp32 value: nearest, ties to the even code, saturating at +-448."""
-    return int(_load().oracle_e4m3_rne(float(np.float32(v))))
+    """e4m3fn code of a real value: nearest, ties to the even code, saturating at +-448."""
+    return int(_load().oracle_e4m3_rne(float(v)))
 
 
-def quantize_e4m3(x_bits, rmsnorm=False, eps=1e-6):
+def quantize_e4m3(x_bits, rmsnorm=False, eps=1e-6, with_quotient=False):
     """e4m3 prologue (see attn_oracle.c): bf16 bits [B,H,S,D] -> (codes uint8 [B,H,S,D],
-    descale float32 [B,H])."""
+    descale float32 [B,H]); with_quotient also returns the fp64 quotients
+    y / descale [B,H,S,D] that the codes round."""
     x_bits = np.ascontiguousarray(x_bits)
     if x_bits.dtype != np.uint16 or x_bits.ndim != 4:
         raise TypeError("quantize_e4m3 takes [B,H,S,D] uint16 bf16 bit patterns")
     B, H, S, D = x_bits.shape
     codes = np.empty(x_bits.shape, dtype=np.uint8)
     descale = np.empty((B, H), dtype=np.float32)
-    rc = _load().oracle_quantize_e4m3(_ptr(x_bits), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)),
-                                      float(eps))
+    quot = np.empty(x_bits.shape, dtype=np.float64) if with_quotient else None
+    rc = _load().oracle_quantize_e4m3(_ptr(x_bits), _ptr(codes), _ptr(descale), _ptr(quot), B, H, S, D,
+                                      int(bool(rmsnorm)), float(eps))
     if rc != 0:
         raise RuntimeError("oracle_quantize_e4m3 failed with code %d" % rc)
-    return codes, descale
+    return (codes, descale, quot) if with_quotient else (codes, descale)
 
 
 def attn_fwd(q, k, v, scale, causal=False, rows=None, descales=None):

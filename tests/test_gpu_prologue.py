@@ -1,14 +1,19 @@
 """GPU parity of the e4m3 quantisation prologue (attn_quantize_e4m3) against the
-oracle: codes and descales bit for bit, at small ragged shapes and on the full
-Q of the fp8 config; invariance under head slicing; and the whole fp8 pipeline
-(product prologue, then attn_fwd) against the oracle on the dequantized values."""
+oracle, at small ragged shapes and on the full Q of the fp8 config: the kernel
+normalises in fp32, the oracle in fp64, so descales agree within a relative
+2^-17 and codes agree except next to an e4m3 rounding midpoint (within a
+relative 2^-16 of the oracle's quotient), where they differ by one step (the
+rule and its derivation are in tests/parity.py); without normalisation the
+descales are bit-equal.  Also invariance under head slicing, and the whole
+fp8 pipeline (product prologue, then attn_fwd) against the oracle on the
+dequantized values."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads
-from parity import FP8_NRMS, fwd_errors, oracle_fwd
+from parity import FP8_NRMS, check_e4m3_codes, fwd_errors, oracle_fwd
 from workloads import Workload, bf16_bits, make_fwd_inputs, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -23,21 +28,26 @@ def h():
     return pkg
 
 
-def check_exact(h, x, rmsnorm, eps=1e-6):
+def check_exact(h, x, rmsnorm, eps=1e-6, max_frac=1e-4):
+    """Prologue on the GPU against the oracle under the e4m3 parity rule; the
+    number of codes that differ (each next to a rounding boundary) is reported
+    and bounded by max_frac of the elements."""
     codes, ds = h.quantize_e4m3(x.cuda(), rmsnorm=rmsnorm, eps=eps)
     assert h.get_device_error() == 0
-    ref_codes, ref_ds = oracle.quantize_e4m3(bf16_bits(x), rmsnorm=rmsnorm, eps=eps)
+    ref_codes, ref_ds, quot = oracle.quantize_e4m3(bf16_bits(x), rmsnorm=rmsnorm, eps=eps, with_quotient=True)
     got_ds = ds.cpu().numpy()
-    assert np.array_equal(got_ds.view(np.uint32), ref_ds.view(np.uint32))
-    got = codes.view(torch.uint8).cpu().numpy()
-    bad = np.flatnonzero(got != ref_codes)
-    assert bad.size == 0, (bad.size, bad[:5], got.ravel()[bad[:5]], ref_codes.ravel()[bad[:5]])
+    if not rmsnorm:
+        # y = x exactly: both sides round amax / 448 once to fp32
+        assert np.array_equal(got_ds.view(np.uint32), ref_ds.view(np.uint32))
+    n_diff = check_e4m3_codes(codes.view(torch.uint8).cpu().numpy(), got_ds, ref_codes, ref_ds, quot)
+    print("e4m3 codes differing next to a rounding boundary: %d of %d" % (n_diff, ref_codes.size))
+    assert n_diff <= max(2, max_frac * ref_codes.size), n_diff
     return codes, ds
 
 
 @pytest.mark.parametrize("B,H,S", [(1, 1, 1), (1, 3, 37), (2, 2, 300), (1, 4, 1000), (3, 1, 257)])
 @pytest.mark.parametrize("rmsnorm", [False, True])
-def test_prologue_small_bit_exact(h, B, H, S, rmsnorm):
+def test_prologue_small(h, B, H, S, rmsnorm):
     g = torch.Generator().manual_seed(1000 + S + B)
     x = (torch.randn(B, H, S, 128, generator=g) * 1.7).to(torch.bfloat16)
     check_exact(h, x, rmsnorm)
@@ -75,7 +85,7 @@ def test_prologue_more_than_65535_heads(h):
     check_exact(h, x, False)
 
 
-def test_prologue_fp8_config_q_bit_exact(h):
+def test_prologue_fp8_config_q(h):
     w = workloads.get("fp8")
     g = torch.Generator().manual_seed(w.seed)
     x = torch.randn(w.B, w.Hq, w.Sq, w.D, generator=g).to(torch.bfloat16)
