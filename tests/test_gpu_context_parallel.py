@@ -18,7 +18,7 @@ import pytest
 import torch
 import torch.distributed as dist
 
-from parity import LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
+from parity import LSE_MAX_ABS, O_MAX_ABS, O_NRMS, fwd_errors, oracle_fwd
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +58,7 @@ def test_context_parallel_one_rank_nccl(h):
     assert h.get_device_error() == 0
     o_ref, lse_ref = oracle_fwd(q, ks[0], vs[0], 1.0 / np.sqrt(128))
     e = fwd_errors(out, lse, o_ref, lse_ref)
-    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS and e["o_nrms"] <= O_NRMS, e
 
 
 @pytest.mark.parametrize("world,shard_len", [(2, 640), (4, 333), (8, 129)])
@@ -73,4 +73,4 @@ def test_rank_order_fold_of_gathered_shards(h, world, shard_len):
     assert torch.equal(runs[0][1].view(torch.int32), runs[1][1].view(torch.int32))
     o_ref, lse_ref = oracle_fwd(q, torch.cat(ks, dim=2), torch.cat(vs, dim=2), 1.0 / np.sqrt(128))
     e = fwd_errors(runs[0][0], runs[0][1], o_ref, lse_ref)
-    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS and e["o_nrms"] <= O_NRMS, e

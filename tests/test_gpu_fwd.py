@@ -2,8 +2,11 @@
 the bitwise properties: repeat runs, batch composition, head slicing, and
 canary bytes around the outputs.
 
-Bars: bf16 max |dO| <= 2e-2, max |dLSE| <= 1e-3; e4m3 normalised RMS of O
-<= 1e-2 against the oracle on the dequantized inputs.
+Bars: bf16 max |dO| <= 2e-2, max |dLSE| <= 1e-3 and normalised RMS of O
+<= 1e-2 (at long Sk the outputs are small, |O| ~ 1e-2, so the max-abs bar
+alone would let a badly wrong P V pass; bf16 rounding of O alone is ~0.3 %);
+e4m3 normalised RMS of O <= 1e-2 against the oracle on the dequantized
+inputs.  The long configs are checked on 256 seeded query rows per head.
 """
 import math
 
@@ -12,7 +15,7 @@ import pytest
 import torch
 
 import workloads
-from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
+from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, O_NRMS, fwd_errors, oracle_fwd
 from workloads import Workload, make_fwd_inputs, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -46,7 +49,7 @@ def check_bf16(h, w, rows=None):
     out, lse = run_fwd(h, x, w.causal)
     o_ref, lse_ref = oracle_fwd(x_cpu["q"], x_cpu["k"], x_cpu["v"], w.scale, w.causal, rows=rows)
     e = fwd_errors(out, lse, o_ref, lse_ref, rows)
-    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS and e["o_nrms"] <= O_NRMS, e
     return e
 
 
@@ -118,13 +121,20 @@ def test_llm_config_sampled_rows(h):
 
 def test_video_config_sampled_rows(h):
     w = workloads.get("video")
-    check_bf16(h, w, rows=sample_rows(w.Sq, 48, seed=w.seed))
+    check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
 def test_cross_attention_long_q_sampled_rows(h):
     # Sq >> Sk with an even head count (AITER PR #2911, Wan 2.2 cross-attention report)
-    w = Workload("cross", B=1, Hq=40, Hkv=40, Sq=90000, Sk=512, seed=7)
-    check_bf16(h, w, rows=sample_rows(w.Sq, 64, seed=7))
+    w = workloads.get("cross")
+    check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
+
+
+def test_window_sink_shape_sampled_rows(h):
+    # the raw SDPA call on the window-30 shape, 4680 queries against 51480 keys,
+    # 12 heads (FlashDreams issue #739, SDPA kernels on gfx950)
+    w = workloads.get("window")
+    check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
 # ------------------------------------------------------------------ e4m3
@@ -165,13 +175,13 @@ def test_fp8_persistent_causal_ragged(h):
 def test_fp8_at_video_shape_sampled_rows(h):
     # the e4m3 bench line at the 32760-token video shape (Q, K RMS-normalised)
     w = workloads.get("fp8_32760")
-    check_fp8(h, w, rows=sample_rows(w.Sq, 16, seed=w.seed))
+    check_fp8(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
 def test_bf16_at_fp8_shape_sampled_rows(h):
     # the bf16 bench line at the 75600-token shape
     w = workloads.get("bf16_75600")
-    check_bf16(h, w, rows=sample_rows(w.Sq, 32, seed=w.seed))
+    check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
 def test_fp8_entry_points_agree_bitwise(h):
@@ -195,7 +205,7 @@ def test_fp8_entry_points_agree_bitwise(h):
 
 def test_fp8_config_sampled_rows(h):
     w = workloads.get("fp8")
-    check_fp8(h, w, rows=sample_rows(w.Sq, 64, seed=w.seed))
+    check_fp8(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
 # ------------------------------------------------------------------ bitwise properties
@@ -261,6 +271,7 @@ def test_closed_forms_on_gpu(h):
     scale = 1 / math.sqrt(128)
     mean_v = v.double().mean(dim=2, keepdim=True)
     assert (out.double().cpu() - mean_v).abs().max() <= O_MAX_ABS
+    assert ((out.double().cpu() - mean_v).norm() / mean_v.expand_as(out).norm()) <= O_NRMS
     expect = math.log(Sk) + scale * torch.einsum("bhid,bhd->bhi", q.double(), k1[:, :, 0].double())
     assert (lse.double().cpu() - expect).abs().max() <= LSE_MAX_ABS
     out0, lse0 = h.attn_fwd(torch.zeros_like(q).cuda(), k.cuda(), v.cuda())

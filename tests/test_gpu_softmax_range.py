@@ -24,7 +24,7 @@ import pytest
 import torch
 
 import oracle
-from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, fwd_errors, grad_errors, grad_ok, np_bits, oracle_fwd
+from parity import FP8_NRMS, LSE_MAX_ABS, O_MAX_ABS, O_NRMS, fwd_errors, grad_errors, grad_ok, np_bits, oracle_fwd
 from workloads.gen import quantize_e4m3_per_head
 
 pytestmark = pytest.mark.gpu
@@ -64,7 +64,7 @@ def test_fwd_rising_and_falling_scores(h, B, Hq, Hkv, Sq, Sk, causal):
     o_ref, lse_ref = oracle_fwd(q, k, v, SCALE, causal)
     assert float(np.max(lse_ref)) > 60.0                  # the steep rows reach large scores
     e = fwd_errors(out, lse, o_ref, lse_ref)
-    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS, e
+    assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS and e["o_nrms"] <= O_NRMS, e
 
 
 def test_fp8_rising_and_falling_scores(h):
