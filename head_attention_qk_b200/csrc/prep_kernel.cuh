@@ -13,8 +13,11 @@
 //   r       = 1 / sqrt(ss / 128 + eps)          per row (only with rmsnorm), fp32
 //   y_d     = x_d * r (fp32), or x_d without rmsnorm
 //   descale = max |y| / 448 over the head (1 if that max is 0), fp32
-//   code    = e4m3 of y / descale: fp32 quotient, round to nearest even,
-//             saturating at +-448
+//   code    = e4m3 of the exact quotient y / descale (of the fp32 y and
+//             descale), round to nearest with ties to even, saturating at
+//             +-448: the fp32 quotient, moved one fp32 step towards the exact
+//             one when it lands exactly on an e4m3 midpoint that the exact
+//             quotient is not on
 // Every step is fixed in precision and order, so the codes and descales are a
 // function of the input alone: bit for bit the same for any grid, batch or
 // head split.  Two launches (after a memset of the descale array): the head
@@ -121,20 +124,70 @@ __device__ __forceinline__ float prep_descale_of(float slot) {
   return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// y / ds rounded to fp32, for a pair (rcp = 1/ds correctly rounded, ds >= 2^-60
-// so that no residual below is subnormal).  q0 = y * rcp is within an ulp of
-// the quotient; with the exact residual r = y - q0 ds (one fused multiply-add)
-// the correction q0 + r * rcp is the correctly rounded quotient (P. Markstein, "Computation
-// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
-// Dev. 34(1), 1990).  Below 2^-11 the correction is skipped: every value
-// there, exact or not, takes the e4m3 code of a signed zero (the smallest
-// e4m3 step is 2^-9), and the sign is the quotient's either way.
+// True when the fp32 value q lies exactly on a midpoint between two
+// neighbouring e4m3fn values: in the e4m3 normal range (2^-6 <= |q| < 2^9)
+// the midpoints are the values whose fraction has four bits ending in 1 (the
+// bit worth half an e4m3 step is bit 19 of the fp32 fraction); below it the
+// e4m3 step is 2^-9 and the midpoints are the odd multiples of 2^-10 (that bit
+// sits at fraction bit 13 - e for binary exponent e, and for e = -10 it is
+// the leading bit, so q = 2^-10 exactly).
+__device__ __forceinline__ bool e4m3_midpoint(float q) {
+  const uint32_t u = __float_as_uint(q) & 0x7FFFFFFFu;
+  const int e = (int)(u >> 23) - 127;
+  if (e > 8 || e < -10) return false;
+  if (e == -10) return u == (117u << 23);
+  const uint32_t half = e >= -6 ? (1u << 19) : (1u << (13 - e));
+  return (u & ((half << 1) - 1u)) == half;
+}
+
+// q = the fp32 quotient y / ds correctly rounded, res = y - q ds exactly (one
+// fused multiply-add).  The e4m3 code of the exact quotient is the code of q
+// unless q sits exactly on an e4m3 midpoint while the exact quotient does not
+// (res != 0): then no midpoint lies strictly between q and the exact quotient
+// (they are within half an fp32 step), so moving q one fp32 step towards it
+// gives the code the exact quotient rounds to.  Without this the fp32 rounding
+// would turn such a quotient into a tie (frequent when y and the descale come
+// from bf16 values: 448 y / amax is then often an exact e4m3 midpoint).
+__device__ __forceinline__ float e4m3_exact_tie(float q, float res) {
+  if (res == 0.f || !e4m3_midpoint(q)) return q;
+  return __uint_as_float(__float_as_uint(q) + (((res > 0.f) == (q > 0.f)) ? 1u : 0xFFFFFFFFu));
+}
+
+// Every e4m3 midpoint has the low 19 fraction bits of its fp32 value clear
+// (the half-step bit is bit 19 or above), so a pair with neither value in that
+// form skips the midpoint test (almost all of them).
+__device__ __forceinline__ bool maybe_e4m3_midpoint2(float2 q) {
+  return ((__float_as_uint(q.x) & 0x7FFFFu) == 0u) | ((__float_as_uint(q.y) & 0x7FFFFu) == 0u);
+}
+
+// y / ds for a pair, ready for the round-to-nearest e4m3 conversion (rcp =
+// 1/ds correctly rounded, ds >= 2^-60 so that no residual below is
+// subnormal).  q0 = y * rcp is within an ulp of the quotient; with the exact
+// residual r = y - q0 ds (one fused multiply-add) the correction q0 + r * rcp
+// is the correctly rounded quotient (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990), whose own residual settles an e4m3 midpoint (e4m3_exact_tie).  Below
+// 2^-11 the correction is skipped: every value there, exact or not, takes the
+// e4m3 code of a signed zero (the smallest e4m3 step is 2^-9, its first
+// midpoint 2^-10), and the sign is the quotient's either way.
 __device__ __forceinline__ float2 prep_quotient2(float2 y, float ds, float rcp) {
-  const float2 r2 = make_float2(rcp, rcp);
+  const float2 r2 = make_float2(rcp, rcp), nds = make_float2(-ds, -ds);
   const float2 q0 = __fmul2_rn(y, r2);
-  const float2 res = __ffma2_rn(q0, make_float2(-ds, -ds), y);
-  const float2 q = __ffma2_rn(res, r2, q0);
-  return make_float2(fabsf(q0.x) < 0x1p-11f ? q0.x : q.x, fabsf(q0.y) < 0x1p-11f ? q0.y : q.y);
+  const float2 res = __ffma2_rn(q0, nds, y);
+  const float2 q1 = __ffma2_rn(res, r2, q0);
+  float2 q = make_float2(fabsf(q0.x) < 0x1p-11f ? q0.x : q1.x, fabsf(q0.y) < 0x1p-11f ? q0.y : q1.y);
+  if (maybe_e4m3_midpoint2(q)) {
+    const float2 res2 = __ffma2_rn(q, nds, y);
+    q = make_float2(e4m3_exact_tie(q.x, res2.x), e4m3_exact_tie(q.y, res2.y));
+  }
+  return q;
+}
+
+// Exact division for a head of tiny values (descale < 2^-60), with the same
+// midpoint rule.
+__device__ __forceinline__ float prep_quotient_exact(float y, float ds) {
+  const float q = __fdiv_rn(y, ds);
+  return e4m3_exact_tie(q, __fmaf_rn(-q, ds, y));
 }
 
 __device__ __forceinline__ uint16_t e4m3x2_rn_satfinite(float lo, float hi) {
@@ -173,7 +226,8 @@ __device__ __forceinline__ void prep_quantize_head(const uint16_t* __restrict__ 
     for (int t = 0; t < 4; ++t) {
       float2 y = make_float2(p.v[2 * t], p.v[2 * t + 1]);
       if (rmsnorm) y = __fmul2_rn(y, make_float2(r, r));
-      const float2 q = tiny_ds ? make_float2(__fdiv_rn(y.x, ds), __fdiv_rn(y.y, ds)) : prep_quotient2(y, ds, rcp);
+      const float2 q = tiny_ds ? make_float2(prep_quotient_exact(y.x, ds), prep_quotient_exact(y.y, ds))
+                               : prep_quotient2(y, ds, rcp);
       c[t] = e4m3x2_rn_satfinite(q.x, q.y);
     }
     const int s = r0 + 16 * k;

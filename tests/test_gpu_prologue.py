@@ -28,10 +28,14 @@ def h():
     return pkg
 
 
-def check_exact(h, x, rmsnorm, eps=1e-6, max_frac=1e-4):
+def check_exact(h, x, rmsnorm, eps=1e-6, max_frac=1e-3):
     """Prologue on the GPU against the oracle under the e4m3 parity rule; the
     number of codes that differ (each next to a rounding boundary) is reported
-    and bounded by max_frac of the elements."""
+    and bounded: by max_frac of the elements with the norm, by zero without it
+    (y = x exactly, and both sides round the exact quotient).  With the norm
+    the bound is loose for heads of few rows: in the row of a head's largest
+    value, 448 x / x_max is often exactly an e4m3 midpoint, and which side the
+    fp32 and fp64 values of y fall on is then a matter of their rounding."""
     codes, ds = h.quantize_e4m3(x.cuda(), rmsnorm=rmsnorm, eps=eps)
     assert h.get_device_error() == 0
     ref_codes, ref_ds, quot = oracle.quantize_e4m3(bf16_bits(x), rmsnorm=rmsnorm, eps=eps, with_quotient=True)
@@ -41,7 +45,7 @@ def check_exact(h, x, rmsnorm, eps=1e-6, max_frac=1e-4):
         assert np.array_equal(got_ds.view(np.uint32), ref_ds.view(np.uint32))
     n_diff = check_e4m3_codes(codes.view(torch.uint8).cpu().numpy(), got_ds, ref_codes, ref_ds, quot)
     print("e4m3 codes differing next to a rounding boundary: %d of %d" % (n_diff, ref_codes.size))
-    assert n_diff <= max(2, max_frac * ref_codes.size), n_diff
+    assert n_diff <= (max_frac * ref_codes.size if rmsnorm else 0), n_diff
     return codes, ds
 
 
@@ -89,7 +93,8 @@ def test_prologue_fp8_config_q(h):
     w = workloads.get("fp8")
     g = torch.Generator().manual_seed(w.seed)
     x = torch.randn(w.B, w.Hq, w.Sq, w.D, generator=g).to(torch.bfloat16)
-    check_exact(h, x, True)
+    check_exact(h, x, True, max_frac=1e-5)
+    check_exact(h, x, False)
 
 
 def test_prologue_head_slice_bitwise(h):
