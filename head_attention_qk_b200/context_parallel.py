@@ -51,8 +51,17 @@ def gather_kv_shards(k, v, group=None):
 def attn_fwd_context_parallel(q, k, v, group=None, scale=None, out=None, lse=None, stream=None):
     """O [B, Hq, Sq, D] bf16 and LSE [B, Hq, Sq] fp32 of this rank's queries q
     against the K/V shards of all ranks of ``group`` (this rank's k, v
-    [B, Hkv, L, D]), folded in rank order."""
+    [B, Hkv, L, D]), folded in rank order.  The all-gather runs on torch's
+    current stream; with a ``stream`` of the caller's, the attention kernel
+    waits there for the gather, and the gathered buffers stay reserved for
+    that stream until its work on them is done."""
     kg, vg = gather_kv_shards(k, v, group)
     world = kg.shape[0]
+    if stream is not None and kg.is_cuda:
+        cur = torch.cuda.current_stream(kg.device)
+        if stream != cur:
+            stream.wait_stream(cur)
+            kg.record_stream(stream)
+            vg.record_stream(stream)
     return hattn.attn_fwd_kvblocks(q, [kg[r] for r in range(world)], [vg[r] for r in range(world)], scale=scale,
                                    out=out, lse=lse, stream=stream)

@@ -16,12 +16,23 @@
 //   warps 4-7  softmax group 1: query tile 1 (rows q0+128 .. q0+255)
 //   warp 8     TMA producer: Q once, then K_j / V_j into one ring
 //   warp 9     MMA issuer (one thread) and tensor-memory owner
-//   warps 10-11  no role (they hold the registers the softmax groups give up)
+//   warps 10-11  e4m3 V widened here (kWidenV): e4m3 V tile -> fp16 in shared
+//              memory; otherwise no role (they hold the registers the softmax
+//              groups give up)
 //
-// e4m3 inputs: Q and K stay e4m3 (S = Q K^T runs as an 8-bit MMA); V arrives
-// already widened to fp16 (exact) by a separate pass, so P V is an fp16 MMA with
-// P in fp16 and no conversion competes with the softmax for issue slots or
-// shared-memory bandwidth.
+// e4m3 inputs: Q and K stay e4m3 (S = Q K^T runs as an 8-bit MMA) and P V is an
+// fp16 MMA with P in fp16.  V reaches it as fp16 (exact) in one of two ways:
+// already widened in global memory by a separate pass (the fast form, for
+// callers that give scratch memory), or loaded as e4m3 and widened in shared
+// memory by warps 10-11 (kWidenV: no scratch; the conversion competes with the
+// softmax for issue slots and shared-memory bandwidth, about 2 % slower).
+//
+// Descales (e4m3): per (b, head) and, for the block-KV forward, per block.  The
+// K descale scales block b's scores (c = scale log2(e) q_ds k_ds[b]); the V
+// descale of block b enters as the factor vd_b / vd_max <= 1 on that block's
+// probabilities before they are rounded to fp16 for P V (added to the exponent
+// as log2(vd_b / vd_max), so no multiply per element), with the row sum l
+// corrected once per tile; the epilogue multiplies by vd_max / l.
 //
 // Tensor memory (512 columns x 128 lanes, fp32):
 //   [  0,128) S0 = Q0 K_j^T   (P0 = softmax numerators, 16-bit, aliases its first 64 columns)
@@ -86,8 +97,8 @@ struct FwdArgs {
   float scale_log2;              // scale * log2(e)
   void* out;                     // bf16 [B,Hq,Sq,D]  or  fp32 partials [blk][B,Hq,Sq,D]
   float* lse;                    // fp32 [B,Hq,Sq]    or  fp32 partials [blk][B,Hq,Sq]
-  const float* q_descale;        // fp8 only: [B*Hq], [B*Hkv], [B*Hkv]
-  const float* k_descale;
+  const float* q_descale;        // fp8 only: [B*Hq]
+  const float* k_descale;        // fp8 only: [n_blocks][B*Hkv] (one block for attn_fwd)
   const float* v_descale;
   int block_offset;              // index of this launch's first block among all blocks
   int total_units;               // work units of this launch; CTAs loop over them
@@ -95,20 +106,28 @@ struct FwdArgs {
   int fused_tiles;               // KV tiles over all fused blocks
 };
 
-template <bool kFp8>
+template <bool kFp8, bool kWidenV = false>
 struct FwdSmemLayout {
+  static_assert(!kWidenV || kFp8, "only e4m3 V is widened in shared memory");
   static constexpr int kElt = kFp8 ? 1 : 2;                            // Q and K element bytes
   static constexpr int kTileBytes = kBlockM * kHeadDim * kElt;         // Q or K tile as loaded
-  static constexpr int kVTileBytes = kBlockN * kHeadDim * 2;           // V tile: bf16, or fp16 widened from e4m3
-  static constexpr int kSlotBytes = kVTileBytes;
+  static constexpr int kVTileBytes = kBlockN * kHeadDim * 2;           // V tile as P V reads it: bf16 or fp16
+  static constexpr int kVLoadBytes = kWidenV ? kTileBytes : kVTileBytes;   // V tile as loaded
+  static constexpr int kSlotBytes = kVLoadBytes;
   // One ring holds the K and V tiles in load order K_0, V_0, K_1, V_1, ...; they
   // are also released in that order (K_j when S1_j completes, V_j when PV1_j
-  // completes), so the producer can run kRing tiles ahead of the MMAs.
-  static constexpr int kRing = kFp8 ? 6 : 5;
+  // completes, or when it is widened), so the producer can run kRing tiles
+  // ahead of the MMAs.  With kWidenV the ring has an even number of slots, so
+  // every slot keeps one role (K in even slots, V in odd ones), and the widened
+  // V tiles go through kStagesV16 fp16 buffers.
+  static constexpr int kRing = kWidenV ? 8 : (kFp8 ? 6 : 5);
+  static_assert(!kWidenV || kRing % 2 == 0, "widening needs slots of one role");
+  static constexpr int kStagesV16 = kWidenV ? 2 : 0;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTilesPerCta * kTileBytes;
-  static constexpr int kBarOff = kRingOff + kRing * kSlotBytes;
-  static constexpr int kNumBars = 3 + 2 * kRing + 8;
+  static constexpr int kV16Off = kRingOff + kRing * kSlotBytes;
+  static constexpr int kBarOff = kV16Off + kStagesV16 * kVTileBytes;
+  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -120,6 +139,8 @@ struct FwdBars {
   uint64_t* mma_drain;  // every MMA of the CTA has completed (committed once, at exit)
   uint64_t* ring_full;   // [kRing]
   uint64_t* ring_empty;  // [kRing]
+  uint64_t* v16_full;    // [kStagesV16]: widened V tile written (one arrival per widening warp)
+  uint64_t* v16_empty;   // [kStagesV16]: the P V MMAs of that tile have completed
   uint64_t* s_full;   // [2]: S_t ready
   uint64_t* p_full;   // [2 tiles][2 halves of 64 keys]: P_t,h written (128 arrivals)
   uint64_t* o_done;   // [2]: last P V of the tile completed
@@ -129,7 +150,7 @@ struct FwdBars {
 // Barrier sites recorded in the error word when a wait times out.
 enum : int {
   kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty,
-  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain
+  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain, kSiteV16Full, kSiteV16Empty
 };
 
 __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int q_row0) {
@@ -195,9 +216,9 @@ __device__ __forceinline__ bool fwd_more_units(int u, int u_first, int u_end, bo
   return kPersist ? (u < u_end && ok) : (u == u_first);
 }
 
-template <bool kFp8, bool kPartial, bool kPersist>
+template <bool kFp8, bool kPartial, bool kPersist, bool kWidenV = false>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
-  using L = FwdSmemLayout<kFp8>;
+  using L = FwdSmemLayout<kFp8, kWidenV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -216,6 +237,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     bb.mma_drain = p; p += 1;
     bb.ring_full = p; p += L::kRing;
     bb.ring_empty = p; p += L::kRing;
+    bb.v16_full = p; p += L::kStagesV16;
+    bb.v16_empty = p; p += L::kStagesV16;
     bb.s_full = p; p += 2;
     bb.p_full = p; p += 4;
     bb.o_done = p; p += 2;
@@ -228,7 +251,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     mbar_init(bb.mma_drain, 1);
     for (int s = 0; s < L::kRing; ++s) {
       mbar_init(&bb.ring_full[s], 1);
-      mbar_init(&bb.ring_empty[s], 1);
+      // widened V (odd slots) is released by the two widening warps, every
+      // other slot by one MMA commit
+      mbar_init(&bb.ring_empty[s], (kWidenV && (s & 1)) ? 2 : 1);
+    }
+    for (int s = 0; s < L::kStagesV16; ++s) {
+      mbar_init(&bb.v16_full[s], 2);
+      mbar_init(&bb.v16_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bb.s_full[i], 1);
@@ -253,6 +282,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
 
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sRing = smem + L::kRingOff;
+  uint8_t* sV16 = smem + L::kV16Off;
 
   // Register split (see kRegsSoftmax): the producer / MMA warpgroup gives
   // registers up, the two softmax warpgroups take them.
@@ -264,7 +294,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       constexpr int kBoxes = kFp8 ? 1 : 2;                 // 128-byte-wide boxes per 128-column Q/K row
       constexpr int kBoxBytes = L::kTileBytes / kBoxes;
       constexpr int kBoxCols = 128 / L::kElt;
-      constexpr int kVBoxBytes = L::kVTileBytes / 2;       // V: two boxes of 64 16-bit columns
+      constexpr int kVBoxes = kWidenV ? 1 : 2;             // V: one e4m3 box, or two of 64 16-bit columns
+      constexpr int kVBoxBytes = L::kVLoadBytes / kVBoxes;
+      constexpr int kVBoxCols = kWidenV ? 128 : 64;
       bool ok = true;
       int slot = 0, units = 0;
       uint32_t ph = 0;
@@ -287,9 +319,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           if (!ok) break;
           uint8_t* dst = sRing + slot * L::kSlotBytes;
           if (n & 1) {
-            mbar_arrive_expect_tx(&bb.ring_full[slot], L::kVTileBytes);
-            for (int x = 0; x < 2; ++x)
-              tma_load_3d(dst + x * kVBoxBytes, &args.tm_v[b], &bb.ring_full[slot], x * 64, lt * kBlockN, w.kvh);
+            mbar_arrive_expect_tx(&bb.ring_full[slot], L::kVLoadBytes);
+            for (int x = 0; x < kVBoxes; ++x)
+              tma_load_3d(dst + x * kVBoxBytes, &args.tm_v[b], &bb.ring_full[slot], x * kVBoxCols, lt * kBlockN,
+                          w.kvh);
             if (++lt == nt && n + 1 < 2 * w.n_kv) {         // next block
               ++b;
               lt = 0;
@@ -319,7 +352,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       constexpr uint32_t kIdescPV = kFp8 ? make_idesc(0, 0, 1, 128, 128) : make_idesc(1, 1, 1, 128, 128);
       constexpr int kQKSteps = kFp8 ? 4 : 8;               // K = 32 (e4m3) or 16 (bf16) per MMA
       constexpr int kQKStepBytes = 32;
-      const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
+      const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing), sV16a = smem_u32(sV16);
       // Descriptor halves: Q / K tiles K-major (SBO 1024 B), V MN-major (LBO 16 KB
       // between the two 64-column halves of the head dim, SBO 1024 B).
       constexpr uint32_t kHi = sdesc_hi(1024);
@@ -363,8 +396,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       };
 
       bool ok = true;
-      int kslot = 0, units = 0;
-      uint32_t kph = 0, jg = 0;
+      int kslot = 0, units = 0, vs16 = 0;
+      uint32_t kph = 0, jg = 0, vph16 = 0;
       for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u = fwd_unit_index<kPersist>(++units)) {
         const FwdUnit w = fwd_unit(args, u);
         const int n_kv = w.n_kv;
@@ -382,8 +415,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           int vslot = kslot;
           uint32_t vph = kph;
           next_pos(vslot, vph);                            // V_j follows K_j
-          ok = mbar_wait(&bb.ring_full[vslot], vph, kSiteVFull);
-          const uint32_t vbase = sRa + vslot * L::kSlotBytes;
+          uint32_t vbase;
+          if (kWidenV) {
+            ok = mbar_wait(&bb.v16_full[vs16], vph16, kSiteV16Full);
+            vbase = sV16a + vs16 * L::kVTileBytes;
+          } else {
+            ok = mbar_wait(&bb.ring_full[vslot], vph, kSiteVFull);
+            vbase = sRa + vslot * L::kSlotBytes;
+          }
           if (ok) ok = pv(0, vbase, jg, j);
           if (!ok) break;
           if (j == n_kv - 1) mma_commit(&bb.o_done[0]);
@@ -400,7 +439,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           }
           ok = pv(1, vbase, jg, j);
           if (!ok) break;
-          mma_commit(&bb.ring_empty[vslot]);
+          if (kWidenV) {
+            mma_commit(&bb.v16_empty[vs16]);
+            if (++vs16 == L::kStagesV16) { vs16 = 0; vph16 ^= 1u; }
+          } else {
+            mma_commit(&bb.ring_empty[vslot]);
+          }
           if (j == n_kv - 1) mma_commit(&bb.o_done[1]);
           if (more) {
             issue_qk(1, kslot);
@@ -416,6 +460,56 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_wait_drain(bb.mma_drain, 0, kSiteDrain);
     }
     __syncwarp();
+  } else if constexpr (kWidenV) {
+    // ------------------------------------------------------------ warps 10-11: widen e4m3 V to fp16
+    const int t = threadIdx.x - 320;                     // 0..63
+    bool ok = true;
+    uint32_t jg = 0;                                     // this CTA's tile count
+    int units = 0;
+    for (int u = u_first; fwd_more_units<kPersist>(u, u_first, u_end, ok); u = fwd_unit_index<kPersist>(++units)) {
+      const int n_kv = fwd_unit(args, u).n_kv;
+      for (int j = 0; j < n_kv && ok; ++j, ++jg) {
+        // V of tile jg sits at ring position 2 jg + 1 (an odd slot: the ring is even)
+        const int vslot = (int)((2u * jg + 1u) % L::kRing);
+        const uint32_t vph = ((2u * jg + 1u) / L::kRing) & 1u;
+        const int s16 = (int)(jg % L::kStagesV16);
+        const uint32_t u16 = jg / L::kStagesV16;
+        ok = warp_wait(&bb.ring_full[vslot], vph, kSiteVFull);
+        if (ok && jg >= (uint32_t)L::kStagesV16) ok = warp_wait(&bb.v16_empty[s16], (u16 - 1) & 1, kSiteV16Empty);
+        if (!ok) break;
+        const uint8_t* src = sRing + vslot * L::kSlotBytes;
+        uint8_t* dst = sV16 + s16 * L::kVTileBytes;
+        // e4m3 tile (128-byte swizzle): key row r is 128 bytes, 16-byte chunk c
+        // holds head dims [16 c, 16 c + 16) and sits at chunk c ^ (r & 7).  fp16
+        // tile: two 16 KB halves of 64 head dims; row r of a half is 128 bytes,
+        // chunk c8 holds dims [8 c8, 8 c8 + 8) of the half at chunk c8 ^ (r & 7).
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+          const int idx = t + 64 * it;
+          const int r = idx >> 3, c = idx & 7;
+          const uint4 in = *reinterpret_cast<const uint4*>(src + r * 128 + ((c ^ (r & 7)) << 4));
+          const uint32_t wv[4] = {in.x, in.y, in.z, in.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            o[2 * q] = e4m3x2_to_f16x2((uint16_t)(wv[q] & 0xFFFFu));
+            o[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(wv[q] >> 16));
+          }
+          const int half = c >> 2;
+          const int c8 = (c & 3) * 2;
+          uint8_t* rowp = dst + half * 16384 + r * 128;
+          *reinterpret_cast<uint4*>(rowp + ((c8 ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(rowp + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        // the MMAs read the fp16 tile through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bb.v16_full[s16]);
+          mbar_arrive(&bb.ring_empty[vslot]);             // this warp is done reading the e4m3 slot
+        }
+      }
+    }
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax) : "memory");
@@ -435,20 +529,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       const int n_kv = w.n_kv, sk = w.sk, bh = w.bh;
       const int row = w.q_row0 + tile * kBlockM + r;
       const int kv_limit = args.causal ? min(sk - 1, row + (sk - args.Sq)) : sk - 1;
-      float c = args.scale_log2;
-      float v_scale = 1.f;
+      const bool fused = args.fused_blocks > 1;
+      // Score factor c (base 2) and, for e4m3, the V descale v_scale the
+      // epilogue applies; with fused e4m3 blocks both change per block: c_b
+      // per tile, and block b's probabilities enter P V scaled by
+      // vd_b / v_scale (v_scale = the largest of the unit's V descales) through
+      // the exponent offset lg_pv = log2(vd_b / v_scale) <= 0, its row sum by
+      // inv_pv = v_scale / vd_b.
+      const size_t bhkv = (size_t)args.B * args.Hkv;
+      float cq = args.scale_log2, c = cq;
+      float v_scale = 1.f, lg_pv = 0.f, inv_pv = 1.f;
       if (kFp8) {
-        c *= __ldg(&args.q_descale[bh]) * __ldg(&args.k_descale[w.kvh]);
-        v_scale = __ldg(&args.v_descale[w.kvh]);
+        cq *= __ldg(&args.q_descale[bh]);
+        const size_t d0 = (size_t)(args.block_offset + w.blk) * bhkv + w.kvh;
+        c = cq * __ldg(&args.k_descale[d0]);
+        v_scale = __ldg(&args.v_descale[d0]);
+        if (fused) {
+          for (int b = 1; b < args.fused_blocks; ++b)
+            v_scale = fmaxf(v_scale, __ldg(&args.v_descale[(size_t)b * bhkv + w.kvh]));
+          const float vd0 = __ldg(&args.v_descale[d0]);
+          lg_pv = __log2f(vd0 / v_scale);
+          inv_pv = v_scale / vd0;
+        }
       }
 
       float m = -INFINITY;     // running max of x = s * c (base-2 units)
       float l = 0.f;           // running sum of 2^(x - m)
-      const bool fused = args.fused_blocks > 1;
       int fb = 0, flt = 0, fsk = args.sk[0], fnt = fwd_block_tiles(fsk);   // fused: block / tile walk
       for (int j = 0; j < n_kv; ++j, ++jg) {
         // last unmasked key column of this tile (>= 127: none masked)
         int lim;
+        float c_t = c, lg_t = lg_pv, inv_t = inv_pv;    // this tile's block factors
         if (fused) {
           lim = fsk - flt * kBlockN - 1;
           if (++flt == fnt && j + 1 < n_kv) {
@@ -456,6 +567,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
             flt = 0;
             fsk = args.sk[fb];
             fnt = fwd_block_tiles(fsk);
+            if (kFp8) {                                  // the next tile starts block fb
+              const size_t db = (size_t)fb * bhkv + w.kvh;
+              c = cq * __ldg(&args.k_descale[db]);
+              const float vdb = __ldg(&args.v_descale[db]);
+              lg_pv = __log2f(vdb / v_scale);
+              inv_pv = v_scale / vdb;
+            }
           }
         } else {
           lim = kv_limit - j * kBlockN;
@@ -489,7 +607,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
-        const float m_tile = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
+        const float m_tile = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_t;
         const bool need = m_tile > m + kRescaleThreshold || (m == -INFINITY && m_tile > -INFINITY);
         float f = 1.f;
         if (need) {
@@ -511,8 +629,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           }
           tmem_wait_st();
         }
-        const float mneg = (m == -INFINITY) ? 0.f : -m;
-        const float2 c2 = make_float2(c, c), mneg2 = make_float2(mneg, mneg);
+        const float mneg = ((m == -INFINITY) ? 0.f : -m) + lg_t;
+        const float2 c2 = make_float2(c_t, c_t), mneg2 = make_float2(mneg, mneg);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         // Two halves of 64 keys: each half is written to TMEM and released to the
         // MMA warp as soon as it is ready, so P V can start on keys 0..63.
@@ -546,7 +664,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         }
         const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
         const float2 a2 = __fadd2_rn(a01, a23);
-        l += a2.x + a2.y;
+        l += (a2.x + a2.y) * inv_t;
       }
       if (ok) ok = warp_wait(&bb.o_done[tile], units & 1, kSiteODone);
       if (!ok) break;

@@ -1,8 +1,9 @@
 // hattn.cu -- host side of libhattn.so: argument checks, TMA descriptor
 // encoding, launch configuration and the extern "C" entry points of hattn.h.
 //
-// The library holds no device memory of its own and never synchronises the
-// host except in attn_get_device_error().  cuTensorMapEncodeTiled is resolved
+// The library allocates no device memory (its one static array serves
+// attn_bwd_noalloc) and never synchronises the host except in
+// attn_get_device_error().  cuTensorMapEncodeTiled is resolved
 // through cudaGetDriverEntryPoint so the library links only the static CUDA
 // runtime and loads on machines without a GPU driver (calls then fail with
 // HATTN_ELAUNCH).
@@ -19,6 +20,7 @@
 #include "../../include/hattn.h"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "per_device.h"
 #include "prep_kernel.cuh"
 
 namespace hattn {
@@ -80,19 +82,25 @@ int device_sm_count() {
   return n;
 }
 
-template <bool kFp8, bool kPartial, bool kPersist>
+int current_device() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+template <bool kFp8, bool kPartial, bool kPersist, bool kWidenV>
 int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
-  using L = FwdSmemLayout<kFp8>;
-  static std::once_flag once;
-  static bool attr_ok = false;
-  std::call_once(once, [] {
-    cudaFuncAttributes fa;
-    attr_ok = set_smem_attr(attn_fwd_kernel<kFp8, kPartial, kPersist>, L::kAlloc) &&
-              cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8, kPartial, kPersist>) == cudaSuccess &&
-              fa.numRegs * kFwdThreads >= kRegsNeeded;   // the setmaxnreg split must fit the launch
-  });
-  if (!attr_ok) return HATTN_ELAUNCH;
-  attn_fwd_kernel<kFp8, kPartial, kPersist><<<grid, kFwdThreads, L::kAlloc, st>>>(a);
+  using L = FwdSmemLayout<kFp8, kWidenV>;
+  auto kernel = attn_fwd_kernel<kFp8, kPartial, kPersist, kWidenV>;
+  // once per device: the shared-memory limit, and the check that the
+  // setmaxnreg split fits the registers the launch holds
+  static PerDeviceOnce setup;
+  if (!setup.ensure(current_device(), [&] {
+        cudaFuncAttributes fa;
+        return set_smem_attr(kernel, L::kAlloc) && cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
+               fa.numRegs * kFwdThreads >= kRegsNeeded;
+      }))
+    return HATTN_ELAUNCH;
+  kernel<<<grid, kFwdThreads, L::kAlloc, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
@@ -105,7 +113,7 @@ int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
 // balances them.
 constexpr int kPersistMaxKvTiles = 8;
 
-template <bool kFp8, bool kPartial>
+template <bool kFp8, bool kPartial, bool kWidenV = false>
 int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, long long max_tiles, cudaStream_t st) {
   const long long units = (long long)a.n_qpairs * a.B * a.Hq * n_blocks_in_launch;
   if (units <= 0 || units > INT_MAX) return HATTN_EUNSUPPORTED;
@@ -114,8 +122,8 @@ int launch_fwd(const FwdArgs& a, int n_blocks_in_launch, long long max_tiles, cu
   FwdArgs args = a;
   args.total_units = (int)units;
   const bool persist = max_tiles <= (a.causal ? 2 : 1) * kPersistMaxKvTiles && units > sms;
-  if (persist) return launch_fwd_grid<kFp8, kPartial, true>(args, sms, st);
-  return launch_fwd_grid<kFp8, kPartial, false>(args, (int)units, st);
+  if (persist) return launch_fwd_grid<kFp8, kPartial, true, kWidenV>(args, sms, st);
+  return launch_fwd_grid<kFp8, kPartial, false, kWidenV>(args, (int)units, st);
 }
 
 int check_common(int B, int Hq, int Hkv, int Sq, int D, float scale) {
@@ -139,15 +147,16 @@ bool sizes_fit(long long B, long long H, long long S) {
   return B * H <= 65535LL * 1024 && B * H * S < (1LL << 40) && S < (1LL << 30);
 }
 
-// The backward's launch sizes: the persistent dQ kernel counts its units
-// (B*Hq*ceil(Sq/128)) in an int, the Delta kernel takes one CTA per 64 rows in
-// grid x, and dK/dV puts B*Hkv in grid x and the key tiles in grid y.
+// The backward's launch sizes: the persistent dQ and dK/dV kernels count
+// their units (B*Hq*ceil(Sq/128), B*Hkv*ceil(Sk/128)) in an int, and the Delta
+// kernel takes one CTA per 64 rows in grid x.  (launch_bwd also bounds the
+// steps one persistent CTA counts.)
 bool bwd_sizes_ok(int B, int Hq, int Hkv, int Sq, int Sk) {
   if (!sizes_fit(B, Hq, Sq) || !sizes_fit(B, Hkv, Sk)) return false;
   const long long rows = (long long)B * Hq * Sq;
   if ((long long)B * Hq * ((Sq + kTile - 1) / kTile) > INT_MAX) return false;
-  if ((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta > INT_MAX) return false;
-  return (Sk + kTile - 1) / kTile <= 65535;
+  if ((long long)B * Hkv * ((Sk + kTile - 1) / kTile) > INT_MAX) return false;
+  return (rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta <= INT_MAX;
 }
 
 }  // namespace
@@ -187,8 +196,9 @@ size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtype) {
 
 namespace {
 
-// Forward with the e4m3 V widened to fp16 in `v16` (B*Hkv*Sk*D*2 bytes) when
-// dtype is e4m3; v16 is unused for bf16.
+// Forward.  e4m3 with `v16` (B*Hkv*Sk*D*2 bytes): V is widened to fp16 there by
+// a separate pass first; e4m3 without it: V is widened in shared memory inside
+// the attention kernel (nothing allocated).  v16 is unused for bf16.
 int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                   int Sq, int Sk, float scale, int causal, int dtype, const float* q_descale,
                   const float* k_descale, const float* v_descale, void* v16, cudaStream_t st) {
@@ -197,7 +207,9 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
   memset(&a, 0, sizeof(a));
   if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
   if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
-  if (fp8) {
+  if (fp8 && !v16) {
+    if (!encode_rows(&a.tm_v[0], v, true, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+  } else if (fp8) {
     // V widened to fp16 once (exact), read by the attention kernel's P V MMAs
     const long long n16 = (long long)B * Hkv * Sk * kHeadDim / 16;
     const int sms = device_sm_count();
@@ -221,42 +233,8 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
   a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
   a.block_offset = 0;
   const long long kv_tiles = (Sk + kBlockN - 1) / kBlockN;
-  return fp8 ? launch_fwd<true, false>(a, 1, kv_tiles, st) : launch_fwd<false, false>(a, 1, kv_tiles, st);
-}
-
-// Stream-ordered scratch for attn_fwd callers that pass no workspace.  Outside
-// graph capture it comes from a private pool per device that keeps up to
-// kPoolKeepBytes mapped between calls (a larger block goes back to the device
-// when the stream synchronizes; remapping ~100 MB costs about a millisecond);
-// under capture it becomes a graph allocation node.
-constexpr uint64_t kPoolKeepBytes = 256ull << 20;
-
-int scratch_alloc(void** p, size_t bytes, cudaStream_t st) {
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return HATTN_ELAUNCH;
-  if (cs != cudaStreamCaptureStatusNone) return cudaMallocAsync(p, bytes, st) == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
-  constexpr int kMaxDevices = 64;
-  static std::mutex mu;
-  static cudaMemPool_t pools[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HATTN_ELAUNCH;
-  cudaMemPool_t pool;
-  {
-    std::lock_guard<std::mutex> g(mu);
-    if (!pools[dev]) {
-      cudaMemPoolProps props = {};
-      props.allocType = cudaMemAllocationTypePinned;
-      props.location.type = cudaMemLocationTypeDevice;
-      props.location.id = dev;
-      cudaMemPool_t np;
-      if (cudaMemPoolCreate(&np, &props) != cudaSuccess) return HATTN_ELAUNCH;
-      uint64_t keep = kPoolKeepBytes;
-      cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep);
-      pools[dev] = np;
-    }
-    pool = pools[dev];
-  }
-  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
+  if (!fp8) return launch_fwd<false, false>(a, 1, kv_tiles, st);
+  return v16 ? launch_fwd<true, false>(a, 1, kv_tiles, st) : launch_fwd<true, false, true>(a, 1, kv_tiles, st);
 }
 
 int check_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
@@ -297,19 +275,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              const float* v_descale, void* stream) {
   int rc = check_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, dtype, q_descale, k_descale, v_descale);
   if (rc) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t need = attn_fwd_workspace_size(B, Hkv, Sk, D, dtype);
-  if (!need)
-    return attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale,
-                         v_descale, nullptr, st);
-  // e4m3 without a caller workspace: stream-ordered scratch, released on the
-  // same stream after the kernels.
-  void* v16 = nullptr;
-  if ((rc = scratch_alloc(&v16, need, st))) return rc;
-  rc = attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale, v_descale,
-                     v16, st);
-  if (cudaFreeAsync(v16, st) != cudaSuccess && rc == HATTN_OK) rc = HATTN_ELAUNCH;
-  return rc;
+  // e4m3 without a caller workspace: V is widened inside the attention kernel
+  return attn_fwd_core(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal, dtype, q_descale, k_descale, v_descale,
+                       nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H, int S, int D, int rmsnorm,
@@ -354,8 +322,8 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
   int rc = check_common(B, Hq, Hkv, Sq, D, scale);
   if (rc) return rc;
   if ((rc = check_descales(dtype, q_descale, k_descale, v_descale))) return rc;
-  if (dtype != HATTN_BF16) return HATTN_EUNSUPPORTED;
   if (!sizes_fit(B, Hq, Sq)) return HATTN_EUNSUPPORTED;
+  const bool fp8 = dtype == HATTN_E4M3;
   for (int i = 0; i < n_blocks; ++i) {
     if (!k_blocks[i] || !v_blocks[i]) return HATTN_EINVAL;
     if (blk_len[i] <= 0) return HATTN_EUNSUPPORTED;
@@ -374,11 +342,11 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     // order: its online softmax folds block after block, so no per-block
     // partials are written and no merge pass is needed.
     memset(&a, 0, sizeof(a));
-    if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
     long long tiles = 0;
     for (int i = 0; i < n_blocks; ++i) {
-      if (!encode_rows(&a.tm_k[i], k_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
-      if (!encode_rows(&a.tm_v[i], v_blocks[i], false, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+      if (!encode_rows(&a.tm_k[i], k_blocks[i], fp8, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
+      if (!encode_rows(&a.tm_v[i], v_blocks[i], fp8, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
       a.sk[i] = blk_len[i];
       tiles += (blk_len[i] + kBlockN - 1) / kBlockN;
     }
@@ -388,10 +356,11 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     a.scale_log2 = scale * 1.4426950408889634f;
     a.out = out;
     a.lse = lse;
+    a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
     a.fused_blocks = n_blocks;
     a.fused_tiles = (int)tiles;   // < 32 * 2^23
     if (n_blocks == 1) a.fused_blocks = 0;   // a single block is a plain forward
-    return launch_fwd<false, false>(a, 1, tiles, st);
+    return fp8 ? launch_fwd<true, false, true>(a, 1, tiles, st) : launch_fwd<false, false>(a, 1, tiles, st);
   }
 
   const long long rows = (long long)B * Hq * Sq;
@@ -401,13 +370,13 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
   for (int first = 0; first < n_blocks; first += kMaxKvBlocks) {
     const int cnt = n_blocks - first < kMaxKvBlocks ? n_blocks - first : kMaxKvBlocks;
     memset(&a, 0, sizeof(a));
-    if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
     int max_len = 0;
     for (int i = 0; i < cnt; ++i) {
       max_len = blk_len[first + i] > max_len ? blk_len[first + i] : max_len;
-      if (!encode_rows(&a.tm_k[i], k_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
+      if (!encode_rows(&a.tm_k[i], k_blocks[first + i], fp8, blk_len[first + i], (uint64_t)B * Hkv))
         return HATTN_ELAUNCH;
-      if (!encode_rows(&a.tm_v[i], v_blocks[first + i], false, blk_len[first + i], (uint64_t)B * Hkv))
+      if (!encode_rows(&a.tm_v[i], v_blocks[first + i], fp8, blk_len[first + i], (uint64_t)B * Hkv))
         return HATTN_ELAUNCH;
       a.sk[i] = blk_len[first + i];
     }
@@ -417,8 +386,11 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     a.scale_log2 = scale * 1.4426950408889634f;
     a.out = o_parts;
     a.lse = lse_parts;
+    a.q_descale = q_descale; a.k_descale = k_descale; a.v_descale = v_descale;
     a.block_offset = first;
-    if ((rc = launch_fwd<false, true>(a, cnt, (max_len + kBlockN - 1) / kBlockN, st))) return rc;
+    const long long max_tiles = (max_len + kBlockN - 1) / kBlockN;
+    rc = fp8 ? launch_fwd<true, true, true>(a, cnt, max_tiles, st) : launch_fwd<false, true>(a, cnt, max_tiles, st);
+    if (rc) return rc;
   }
   const unsigned grid = (unsigned)((rows + 7) / 8);
   lse_merge_kernel<<<grid, 256, 0, st>>>(o_parts, lse_parts, n_blocks, rows, reinterpret_cast<uint16_t*>(out), lse);

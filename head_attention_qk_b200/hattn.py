@@ -76,7 +76,11 @@ def _ptr(t):
 # (a buffer smaller than the sizes say would be read or written out of
 # bounds).  Shapes and dtypes are checked first, then that every tensor is a
 # contiguous CUDA tensor on one device; the call runs with that device current
-# and, by default, on its current stream.
+# and, by default, on its current stream.  Outputs and scratch the binding
+# allocates are taken from torch's caching allocator while the launch stream
+# is torch's current stream, so the allocator never hands them to work on
+# another stream while the kernels may still use them (scratch is released
+# on return, and its next owner is ordered after the kernels on that stream).
 
 def _shape(t, name, shape):
     if not isinstance(t, torch.Tensor):
@@ -114,10 +118,15 @@ def _device(named):
 
 
 def _stream(stream, dev=None):
+    """The torch stream a call runs on: `stream`, else the device's current stream."""
     if stream is None:
         stream = torch.cuda.current_stream(dev)
     elif dev is not None and stream.device != dev:
         raise ValueError("stream is on %s, the tensors on %s" % (stream.device, dev))
+    return stream
+
+
+def _sp(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -150,12 +159,14 @@ def fwd_workspace_size(B, Hkv, Sk, D, dtype) -> int:
 
 
 def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, v_descale=None,
-             out=None, lse=None, workspace=None, stream=None):
+             out=None, lse=None, workspace=None, stream=None, use_scratch=True):
     """O [B,Hq,Sq,D] bf16 and LSE [B,Hq,Sq] fp32 for q [B,Hq,Sq,D], k/v [B,Hkv,Sk,D].
 
-    e4m3 inputs need scratch for the fp16 copy of V: `workspace` (a CUDA byte
-    tensor of at least fwd_workspace_size() bytes), else one from torch's
-    allocator; the library itself then allocates nothing.
+    e4m3 inputs take scratch for the fp16 copy of V (the faster of the
+    library's two e4m3 forms, same results): `workspace` (a CUDA byte tensor of
+    at least fwd_workspace_size() bytes), else one from torch's allocator.
+    With use_scratch=False the call takes none and the library widens V in
+    shared memory (attn_fwd of the C ABI).
     """
     B, Hq, Sq, D = _dims4(q, "q")
     _, Hkv, Sk, _ = _dims4(k, "k")
@@ -174,17 +185,24 @@ def attn_fwd(q, k, v, causal=False, scale=None, q_descale=None, k_descale=None, 
     dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("q_descale", q_descale),
                    ("k_descale", k_descale), ("v_descale", v_descale), ("workspace", workspace)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
-    if lse is None:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
-    ws_bytes = fwd_workspace_size(B, Hkv, Sk, D, dt)
-    if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    with torch.cuda.device(dev):
-        rc = lib.attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
-                             int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
-                             _ptr(workspace), _nbytes(workspace), _stream(stream, dev))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        if out is None:
+            out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+        if not use_scratch:
+            if workspace is not None:
+                raise ValueError("workspace given with use_scratch=False")
+            rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+                              int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _sp(st))
+        else:
+            ws_bytes = fwd_workspace_size(B, Hkv, Sk, D, dt)
+            if ws_bytes and workspace is None:
+                workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+            rc = lib.attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+                                 int(bool(causal)), dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
+                                 _ptr(workspace), _nbytes(workspace), _sp(st))
     _check(rc, "attn_fwd")
     return out, lse
 
@@ -202,13 +220,14 @@ def quantize_e4m3(x, rmsnorm=False, eps=1e-6, codes=None, descale=None, stream=N
         if descale.numel() != B * H:
             raise ValueError("descale must hold %d values (one per batch and head)" % (B * H))
     dev = _device([("x", x), ("codes", codes), ("descale", descale)])
-    if codes is None:
-        codes = torch.empty((B, H, S, D), dtype=torch.float8_e4m3fn, device=dev)
-    if descale is None:
-        descale = torch.empty((B, H), dtype=torch.float32, device=dev)
-    with torch.cuda.device(dev):
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        if codes is None:
+            codes = torch.empty((B, H, S, D), dtype=torch.float8_e4m3fn, device=dev)
+        if descale is None:
+            descale = torch.empty((B, H), dtype=torch.float32, device=dev)
         rc = lib.attn_quantize_e4m3(_ptr(x), _ptr(codes), _ptr(descale), B, H, S, D, int(bool(rmsnorm)),
-                                    float(eps), _stream(stream, dev))
+                                    float(eps), _sp(st))
     _check(rc, "attn_quantize_e4m3")
     return codes, descale
 
@@ -217,8 +236,13 @@ def kvblocks_workspace_size(B, Hq, Sq, D, n_blocks) -> int:
     return lib.attn_fwd_kvblocks_workspace_size(B, Hq, Sq, D, n_blocks)
 
 
-def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=None, lse=None, stream=None):
-    """Unmasked attention of q to the concatenation of the KV blocks, folded in block order."""
+def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=None, lse=None, stream=None,
+                      q_descale=None, k_descale=None, v_descale=None):
+    """Unmasked attention of q to the concatenation of the KV blocks, folded in block order.
+
+    e4m3 blocks (an FP8 KV cache) take q_descale [B, Hq] and k_descale,
+    v_descale [n_blocks, B, Hkv] (one scale per block and head; any shape with
+    that many fp32 values, block-major)."""
     B, Hq, Sq, D = _dims4(q, "q")
     n = len(k_blocks)
     if n != len(v_blocks) or n == 0:
@@ -233,13 +257,20 @@ def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=Non
         _dtype(kb, "k_blocks[%d]" % i, q.dtype)
         _dtype(vb, "v_blocks[%d]" % i, q.dtype)
         lens.append(L)
+    for d, name, cnt in ((q_descale, "q_descale", B * Hq), (k_descale, "k_descale", n * B * Hkv),
+                         (v_descale, "v_descale", n * B * Hkv)):
+        if d is not None:
+            _dtype(d, name, torch.float32)
+            if d.numel() != cnt:
+                raise ValueError("%s must hold %d values, got %d" % (name, cnt, d.numel()))
     if out is not None:
         _shape(out, "out", (B, Hq, Sq, D))
         _dtype(out, "out", torch.bfloat16)
     if lse is not None:
         _shape(lse, "lse", (B, Hq, Sq))
         _dtype(lse, "lse", torch.float32)
-    dev = _device([("q", q), ("out", out), ("lse", lse), ("workspace", workspace)]
+    dev = _device([("q", q), ("out", out), ("lse", lse), ("workspace", workspace), ("q_descale", q_descale),
+                   ("k_descale", k_descale), ("v_descale", v_descale)]
                   + [("k_blocks[%d]" % i, t) for i, t in enumerate(k_blocks)]
                   + [("v_blocks[%d]" % i, t) for i, t in enumerate(v_blocks)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -247,17 +278,18 @@ def attn_fwd_kvblocks(q, k_blocks, v_blocks, scale=None, workspace=None, out=Non
     vp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in v_blocks])
     ln = (ctypes.c_int * n)(*lens)
     ws_bytes = kvblocks_workspace_size(B, Hq, Sq, D, n)
-    if workspace is None and ws_bytes:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    if out is None:
-        out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
-    if lse is None:
-        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
-    with torch.cuda.device(dev):
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        if workspace is None and ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        if out is None:
+            out = torch.empty((B, Hq, Sq, D), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
         rc = lib.attn_fwd_kvblocks(_ptr(q), ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p),
                                    ctypes.cast(ln, ctypes.c_void_p), n, _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, D,
-                                   scale, dt, None, None, None, _ptr(workspace), _nbytes(workspace),
-                                   _stream(stream, dev))
+                                   scale, dt, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale), _ptr(workspace),
+                                   _nbytes(workspace), _sp(st))
     _check(rc, "attn_fwd_kvblocks")
     return out, lse
 
@@ -289,15 +321,16 @@ def attn_bwd(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, 
     dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout), ("dq", dq),
                    ("dk", dk), ("dv", dv), ("workspace", workspace)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    if workspace is None:
-        workspace = torch.empty(bwd_workspace_size(B, Hq, Sq), dtype=torch.uint8, device=dev)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    with torch.cuda.device(dev):
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        if workspace is None:
+            workspace = torch.empty(bwd_workspace_size(B, Hq, Sq), dtype=torch.uint8, device=dev)
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
         rc = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                           _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
-                          _nbytes(workspace), _stream(stream, dev))
+                          _nbytes(workspace), _sp(st))
     _check(rc, "attn_bwd")
     return dq, dk, dv
 
@@ -309,13 +342,14 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, causal=False, scale=None, dq=None,
     dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout), ("dq", dq),
                    ("dk", dk), ("dv", dv)])
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    with torch.cuda.device(dev):
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
         rc = lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
                                   _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)),
-                                  _stream(stream, dev))
+                                  _sp(st))
     _check(rc, "attn_bwd_noalloc")
     return dq, dk, dv
 
@@ -323,5 +357,5 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, causal=False, scale=None, dq=None,
 def get_device_error(stream=None) -> int:
     """Synchronise and read-and-clear the kernels' bounded-wait error word (0 = none)."""
     code = ctypes.c_int(0)
-    _check(lib.attn_get_device_error(_stream(stream), ctypes.byref(code)), "attn_get_device_error")
+    _check(lib.attn_get_device_error(_sp(_stream(stream)), ctypes.byref(code)), "attn_get_device_error")
     return code.value

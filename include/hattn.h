@@ -20,10 +20,9 @@
  *  - causal != 0 masks key j for query i unless j <= i + (Sk - Sq)
  *    (bottom-right aligned); it requires Sq <= Sk so every row sees a key.
  *  - All device pointers must be 16-byte aligned.
- *  - The caller owns every buffer.  Calls allocate nothing (one exception:
- *    attn_fwd with e4m3 inputs, see there), never synchronise the host, and
- *    enqueue their kernels on `stream` (a cudaStream_t; NULL is the legacy
- *    default stream), so they may be captured into a CUDA graph.
+ *  - The caller owns every buffer.  Calls allocate nothing, never synchronise
+ *    the host, and enqueue their kernels on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream), so they may be captured into a CUDA graph.
  *  - Results are bitwise reproducible: every output element is written by one
  *    thread block, reductions run in a fixed order, and tile sizes do not depend
  *    on B, H or the number of SMs, so a row's result does not change with the
@@ -74,13 +73,11 @@ enum {
  *     one value per tensor is the case where all entries are equal); all three
  *     must be NULL for bf16.  Descales must be positive.
  * Softmax statistics and both matrix products accumulate in fp32.  For e4m3
- * inputs S = Q K^T is an 8-bit product; V is first widened to fp16 (exactly)
- * in scratch memory, and the probabilities are rounded to fp16 before the P V
- * product.  attn_fwd takes that scratch (attn_fwd_workspace_size() bytes)
- * stream-ordered from a memory pool of the library's own, which keeps up to
- * 256 MB mapped between calls, and releases it on `stream` (under graph capture
- * it becomes a graph allocation); attn_fwd_ws takes it from the caller instead
- * and allocates nothing.
+ * inputs S = Q K^T is an 8-bit product; V is widened to fp16 (exactly) and the
+ * probabilities are rounded to fp16 before the P V product.  attn_fwd widens
+ * each V tile in shared memory inside the attention kernel and allocates
+ * nothing; attn_fwd_ws, given scratch memory, widens V there first in one
+ * pass and runs about 2 % faster.  Both give the same bits.
  */
 HATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int dtype,
@@ -88,10 +85,11 @@ HATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, f
              void* stream);
 
 /*
- * attn_fwd with caller-provided scratch: workspace must hold at least
- * attn_fwd_workspace_size(B, Hkv, Sk, D, dtype) bytes (B*Hkv*Sk*D*2 for e4m3,
- * 0 for bf16, where workspace may be NULL); its contents on entry do not
- * matter.  Too small a workspace returns HATTN_EWORKSPACE.
+ * attn_fwd with caller-provided scratch for the fp16 copy of an e4m3 V:
+ * workspace must hold at least attn_fwd_workspace_size(B, Hkv, Sk, D, dtype)
+ * bytes (B*Hkv*Sk*D*2 for e4m3, 0 for bf16, where workspace may be NULL); its
+ * contents on entry do not matter.  Too small a workspace returns
+ * HATTN_EWORKSPACE.  Same results as attn_fwd, bit for bit.
  */
 HATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* out, float* lse,
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int dtype,
@@ -109,19 +107,22 @@ HATTN_API size_t attn_fwd_workspace_size(int B, int Hkv, int Sk, int D, int dtyp
  *   descale [B*H] fp32 out: the real value of code c of head (b, h) is
  *           decode(c) * descale[b*H + h], ready for attn_fwd's descales.
  * Per head: with rmsnorm != 0 each row is first multiplied by
- * r = 1 / sqrt(ss / 128 + eps), giving y; without it y = x.  All in fp32 with
- * every operation rounded to nearest (eps > 0 is taken as fp32; ss is the sum
- * of the row's squares: the squares of d = 8k .. 8k+7 added in ascending d for
- * k = 0 .. 15, then those 16 partial sums added pairwise, neighbours first:
- * (s0 + s1), (s2 + s3), ..., then ((s0 + s1) + (s2 + s3)), ... up to one sum).
- * descale = max |y| / 448 (fp32; 1 if the head is
- * all zero), code = y / descale (fp32 quotient) rounded to the nearest e4m3fn
- * value, ties to even, saturating at +-448.  The result is bitwise the same for
- * any batch or head split.  Enqueues a memset of descale and two kernels
- * (head maxima; codes, which also turn each maximum into its descale); x is
- * read twice (the second pass starts with the rows read last, which L2 may
- * still hold) and the codes are written once: at most 5 bytes of HBM traffic
- * per element.
+ * r = 1 / sqrt(ss / 128 + eps), giving y; without it y = x.  The norm runs in
+ * fp32 with every operation rounded to nearest (eps > 0 is taken as fp32; ss,
+ * the sum of the row's squares, adds the squares of d = 8k .. 8k+7 in
+ * ascending d for k = 0 .. 15, then those 16 partial sums pairwise, neighbours
+ * first), so y has a relative error below 68 * 2^-24 (a sum of 128
+ * non-negative terms in any order is within 127 * 2^-24 of the exact sum).
+ * descale = max |y| / 448 (fp32; 1 if the head is all zero); code = the
+ * e4m3fn value nearest to the exact quotient y / descale of those fp32 values,
+ * ties to even, saturating at +-448 (the fp32 quotient is correctly rounded,
+ * and when it lands exactly on an e4m3 midpoint the exact residual decides).
+ * Without the norm the codes and descales are exactly those of the definition.
+ * The result is bitwise the same for any batch or head split.  Enqueues a
+ * memset of descale and two kernels (head maxima; codes, which also turn each
+ * maximum into its descale); x is read twice (the second pass starts with the
+ * rows read last, which L2 may still hold) and the codes are written once: at
+ * most 5 bytes of HBM traffic * per element.
  */
 HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int B, int H, int S, int D,
                                  int rmsnorm, double eps, void* stream);
@@ -137,11 +138,21 @@ HATTN_API int attn_quantize_e4m3(const void* x, void* codes, float* descale, int
  * (O_b, LSE_b), then the blocks are folded in ascending order:
  *     M = max(L, L_b); w = e^(L - M); w_b = e^(L_b - M);
  *     L = M + ln(w + w_b); O = (w O + w_b O_b) / (w + w_b),  from (O, L) = (0, -inf).
- *   q          [B, Hq, Sq, D] bf16 (dtype must be HATTN_BF16 in this version)
+ *   q          [B, Hq, Sq, D] bf16, or e4m3fn codes when dtype == HATTN_E4M3
  *   k_blocks, v_blocks: HOST arrays of n_blocks device pointers; block i is
- *              [B, Hkv, blk_len[i], D] bf16
+ *              [B, Hkv, blk_len[i], D] of q's element type
  *   blk_len    HOST array of n_blocks lengths, each > 0
  *   out, lse   as for attn_fwd
+ *   q_descale  e4m3 only: [B*Hq] fp32, as for attn_fwd
+ *   k_descale, v_descale  e4m3 only: [n_blocks * B*Hkv] fp32, block-major: the
+ *              value of code x of block i, head (b, h) is
+ *              x * descale[i*B*Hkv + b*Hkv + h] (an FP8 KV cache whose blocks
+ *              were each quantised with their own scales, e.g. by
+ *              attn_quantize_e4m3 writing a block's codes and its B*Hkv
+ *              descales in place).  NULL for bf16.
+ * e4m3 arithmetic as for attn_fwd (V widened in shared memory); within one
+ * launch block i's probabilities enter P V scaled by vd_i / max_i vd_i, and
+ * the output by max_i vd_i.
  *   workspace  device buffer of at least attn_fwd_kvblocks_workspace_size() bytes
  *              (may be NULL when that is 0); its contents on entry do not matter.
  */
@@ -192,7 +203,10 @@ HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.  The graph-capture remark at the top of this
- *    file does not cover this entry point.
+ *    file does not cover this entry point.  The address is kept for the
+ *    process: after a cudaDeviceReset (or anything else that destroys the
+ *    device's primary context) it is stale, and this entry point must not be
+ *    called again in that process.
  *  - All calls share the one array: calls that overlap on the GPU (different
  *    streams, or several host threads) race on it and must be serialised by
  *    the caller.  Every call rewrites all the rows it reads, so no clearing is

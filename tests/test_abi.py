@@ -174,7 +174,9 @@ def test_kvblocks_fails_closed(h):
     assert call([100, 0], 2) == -2                       # a zero-length block
     assert call([100, 50], 0) == -1
     assert call([100, 50], 2, D=64) == -2
-    assert call([100, 50], 2, dtype=1, qd=A) == -2       # fp8 block-KV not offered
+    assert call([100, 50], 2, dtype=1) == -1             # e4m3 blocks without descales
+    assert call([100, 50], 2, dtype=0, qd=A) == -1       # descales given for bf16
+    assert call([100, 50], 2, dtype=2, qd=A) == -1       # no such element type
     # more blocks than one launch folds: per-block partials need the workspace
     many = [40 + i for i in range(33)]
     need = h.kvblocks_workspace_size(1, 2, 64, 128, 33)

@@ -184,22 +184,32 @@ def test_bf16_at_fp8_shape_sampled_rows(h):
     check_bf16(h, w, rows=sample_rows(w.Sq, 256, seed=w.seed))
 
 
-def test_fp8_entry_points_agree_bitwise(h):
-    # attn_fwd takes its fp16 scratch for V from the stream-ordered pool,
-    # attn_fwd_ws (the binding's path) from the caller: same kernels, same bits
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,causal", [
+    (1, 4, 2, 333, 517, False),
+    (1, 4, 2, 700, 900, True),
+    (1, 40, 20, 1200, 640, False),      # persistent, short KV
+    (2, 40, 8, 1000, 1100, True),       # persistent causal
+    (1, 2, 2, 1, 1, False),
+])
+def test_fp8_entry_points_agree_bitwise(h, B, Hq, Hkv, Sq, Sk, causal):
+    # attn_fwd widens each e4m3 V tile in shared memory inside the attention
+    # kernel (nothing allocated), attn_fwd_ws (the binding's path) widens V
+    # into the caller's scratch first: the same fp16 values reach the same
+    # MMAs, so the results are the same bits
     import ctypes
 
-    w = Workload("f8ws", B=1, Hq=4, Hkv=2, Sq=333, Sk=517, dtype="e4m3", seed=23)
+    w = Workload("f8ws", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, dtype="e4m3", seed=23 + Sq)
     x = cuda(make_fwd_inputs(w))
-    o1, l1 = run_fwd(h, x, False)
+    o1, l1 = run_fwd(h, x, causal)
     o2 = torch.empty_like(o1)
     l2 = torch.empty_like(l1)
     P = lambda t: ctypes.c_void_p(t.data_ptr())
-    rc = h.lib.attn_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(o2), P(l2), 1, 4, 2, 333, 517, 128, w.scale, 0, 1,
-                        P(x["q_descale"]), P(x["k_descale"]), P(x["v_descale"]),
+    rc = h.lib.attn_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(o2), P(l2), B, Hq, Hkv, Sq, Sk, 128, w.scale,
+                        int(causal), 1, P(x["q_descale"]), P(x["k_descale"]), P(x["v_descale"]),
                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 0
     torch.cuda.synchronize()
+    assert h.get_device_error() == 0
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
 
 

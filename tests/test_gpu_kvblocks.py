@@ -67,12 +67,13 @@ def test_kvblocks_more_blocks_than_one_launch(h):
 
 
 def test_kvblocks_persistent_short_blocks(h):
-    # 3 query pairs x 40 heads x 3 blocks = 360 units of at most 4 KV tiles: persistent kernel
+    # 5 query pairs x 40 heads = 200 units (> 148 SMs), each folding 3 blocks
+    # of 8 KV tiles in all: the persistent kernel
     g = torch.Generator().manual_seed(57)
-    q = torch.randn(1, 40, 700, 128, generator=g).to(torch.bfloat16)
+    q = torch.randn(1, 40, 1200, 128, generator=g).to(torch.bfloat16)
     blocks = [(torch.randn(1, 8, n, 128, generator=g).to(torch.bfloat16),
                torch.randn(1, 8, n, 128, generator=g).to(torch.bfloat16)) for n in (512, 77, 300)]
-    out, lse = check_blocks(h, q, blocks, rows=sample_rows(700, 64, seed=57))
+    out, lse = check_blocks(h, q, blocks, rows=sample_rows(1200, 64, seed=57))
     # the same query heads in a launch too small to run persistently: bitwise equal
     o5, l5 = h.attn_fwd_kvblocks(q[:, :5].contiguous().cuda(), [k[:, :1].contiguous().cuda() for k, _ in blocks],
                                  [v[:, :1].contiguous().cuda() for _, v in blocks])

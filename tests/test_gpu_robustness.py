@@ -4,8 +4,11 @@
   reports the site in the device error word, and the context stays usable.
 - The forward and backward calls allocate nothing and never synchronise, so
   they can be captured into a CUDA graph; replay equals the eager results bit
-  for bit.
+  for bit.  The e4m3 forward without a workspace leaves device memory as it was.
 - Unsupported requests raise instead of being approximated.
+- Calls on a stream that is not torch's current one keep their outputs and
+  scratch to that stream: allocations on the current stream meanwhile cannot
+  take them over while the kernels still use them.
 """
 import ctypes
 
@@ -13,7 +16,7 @@ import pytest
 import torch
 
 from parity import LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
-from workloads import Workload, make_bwd_inputs, make_fwd_inputs
+from workloads import Workload, make_bwd_inputs, make_fwd_inputs, make_kvblock_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -70,22 +73,31 @@ def test_cuda_graph_capture_matches_eager(h):
     assert torch.equal(lse_g, lse_e)
 
 
-def test_cuda_graph_capture_fp8_stream_ordered_scratch(h):
-    # the C attn_fwd with e4m3 allocates its fp16 V scratch stream-ordered; under
-    # capture that becomes a graph allocation, and replays equal the eager result
-    w = Workload("graph8", B=1, Hq=4, Hkv=2, Sq=300, Sk=400, dtype="e4m3", seed=79)
+def test_fp8_attn_fwd_allocates_nothing_and_captures(h):
+    # the C attn_fwd with e4m3 inputs and no workspace widens V inside the
+    # kernel: no device memory changes hands (an fp16 copy of this V would be
+    # 64 MB), and the call captures into a graph whose replays equal the eager
+    # result
+    w = Workload("graph8", B=1, Hq=4, Hkv=2, Sq=300, Sk=131072, dtype="e4m3", seed=79)
     x = {k: v.cuda() for k, v in make_fwd_inputs(w).items()}
     P = lambda t: ctypes.c_void_p(t.data_ptr())
 
     def call(out, lse, stream):
-        return h.lib.attn_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(out), P(lse), 1, 4, 2, 300, 400, 128, w.scale, 0, 1,
-                              P(x["q_descale"]), P(x["k_descale"]), P(x["v_descale"]),
+        return h.lib.attn_fwd(P(x["q"]), P(x["k"]), P(x["v"]), P(out), P(lse), 1, 4, 2, 300, w.Sk, 128, w.scale, 0,
+                              1, P(x["q_descale"]), P(x["k_descale"]), P(x["v_descale"]),
                               ctypes.c_void_p(stream.cuda_stream))
 
     out_e = torch.empty(1, 4, 300, 128, dtype=torch.bfloat16, device="cuda")
     lse_e = torch.empty(1, 4, 300, dtype=torch.float32, device="cuda")
-    assert call(out_e, lse_e, torch.cuda.current_stream()) == 0
+    assert call(out_e, lse_e, torch.cuda.current_stream()) == 0      # first call: module load, kernel setup
     torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        assert call(out_e, lse_e, torch.cuda.current_stream()) == 0
+        assert torch.cuda.mem_get_info()[0] == free0                   # nothing taken while enqueued
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert h.get_device_error() == 0
     out_g = torch.zeros_like(out_e)
     lse_g = torch.zeros_like(lse_e)
     s = torch.cuda.Stream()
@@ -148,3 +160,44 @@ def test_fail_closed_on_device(h):
         h.attn_fwd(q8, q8, q8)                                              # e4m3 without descales
     assert ei.value.code == -1
     assert h.get_device_error() == 0
+
+
+def test_side_stream_eager_calls_keep_their_scratch(h):
+    # Each call runs on a side stream s behind a ~50 ms spin, so its kernels
+    # start long after it returns.  Right after each call the current stream
+    # allocates buffers of the scratch's size and fills them: had the binding
+    # taken the scratch on the current stream (and released it on return),
+    # the fill would land in it before the kernels read it.  Results must
+    # equal default-stream calls bit for bit.
+    w = Workload("side", B=2, Hq=4, Hkv=2, Sq=700, Sk=900, causal=True, seed=81)
+    x = {k: v.cuda() for k, v in make_bwd_inputs(w).items()}
+    w8 = Workload("side8", B=1, Hq=4, Hkv=2, Sq=500, Sk=600, dtype="e4m3", seed=82)
+    x8 = {k: v.cuda() for k, v in make_fwd_inputs(w8).items()}
+    ds8 = dict(q_descale=x8["q_descale"], k_descale=x8["k_descale"], v_descale=x8["v_descale"])
+    kv = make_kvblock_inputs(Workload("side_kv", B=1, Hq=2, Hkv=2, Sq=130, Sk=37 * 40, seed=83),
+                             n_blocks=37, block_len=40, text_len=0)
+    qb, kb, vb = kv["q"].cuda(), [t.cuda() for t, _ in kv["blocks"]], [t.cuda() for _, t in kv["blocks"]]
+
+    def run(stream):
+        out, lse = h.attn_fwd(x["q"], x["k"], x["v"], causal=True, stream=stream)
+        grads = h.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True, stream=stream)
+        o8, l8 = h.attn_fwd(x8["q"], x8["k"], x8["v"], stream=stream, **ds8)
+        ob, lb = h.attn_fwd_kvblocks(qb, kb, vb, stream=stream)
+        return (out, lse, o8, l8, ob, lb) + tuple(grads)
+
+    ref = run(None)
+    torch.cuda.synchronize()
+    sizes = [h.bwd_workspace_size(2, 4, 700), h.fwd_workspace_size(1, 2, 600, 128, h.E4M3),
+             h.kvblocks_workspace_size(1, 2, 130, 128, 37)]
+    assert all(n > 0 for n in sizes)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(100_000_000)
+    got = run(s)
+    junk = [torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda") for n in sizes for _ in range(4)]
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    for a, b in zip(got, ref):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    del junk
