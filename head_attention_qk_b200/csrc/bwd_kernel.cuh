@@ -9,9 +9,10 @@
 // fixed order, with no atomics and no S x S buffer:
 //
 //   bwd_delta_kernel  Delta (fp32) from the forward's bf16 O and dO.
-//   bwd_dkdv_kernel   one CTA per (b, kv head, 128-key tile); loops over the
-//                     group's query heads (ascending) and their 128-row query
-//                     tiles (ascending).  Per step, four tcgen05 MMAs:
+//   bwd_dkdv_kernel   persistent, one CTA per SM; each (b, kv head, 128-key
+//                     tile) unit loops over the group's query heads
+//                     (ascending) and their 128-row query tiles (ascending).
+//                     Per step, four tcgen05 MMAs:
 //                       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q
 //                     (S^T of the next step and dV in two query halves).
 //   bwd_dq_kernel     persistent, one CTA per SM; each (b, q head, 128-row query
@@ -34,6 +35,7 @@
 #pragma once
 
 #include "fwd_kernel.cuh"
+#include "per_device.h"
 #include "sm100.cuh"
 
 namespace hattn {
@@ -187,6 +189,12 @@ __device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, u
   }
 }
 
+// The k-th unit of CTA c among G persistent CTAs (the dK/dV and the dQ
+// kernels): the heaviest-first list is dealt out in snake order (c, then
+// 2G-1-c, then 2G+c, ...), which evens out the causal unit sizes.  Increasing
+// in k, so the first index past the list ends the CTA's loop.
+__device__ __forceinline__ int dq_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
+
 // ---------------------------------------------------------------------------- dK / dV
 struct DkdvSmem {
   // Q is read by S^T_n early in a step and by dK_n at its end, so it gets a
@@ -200,7 +208,7 @@ struct DkdvSmem {
   static constexpr int kDO = kQ + kQStages * kTileBytesBf16;
   static constexpr int kStats = kDO + kDOStages * kTileBytesBf16;   // [stage] x (128 lse2 + 128 delta) fp32
   static constexpr int kBars = kStats + kStatStages * 2 * kTile * 4;
-  static constexpr int kBytes = kBars + 24 * 8;
+  static constexpr int kBytes = kBars + 26 * 8;
   // No alignment slack: this layout fills the 227 KB a CTA may hold.  The
   // dynamic shared window starts 1024-byte aligned on sm_100a (after the 1 KB
   // the driver reserves); the kernel checks that and refuses to run otherwise.
@@ -214,6 +222,38 @@ __device__ __forceinline__ int bwd_first_q_tile(int j, int Sq, int Sk, int causa
   return first_q <= 0 ? 0 : first_q / kTile;
 }
 
+// One unit of dK/dV work: key tile j of (batch, KV head) bkv; its steps run
+// over the group's query heads g (ascending) and their query tiles i0 ..
+// nq - 1 (ascending).
+struct DkdvUnit {
+  int j, bkv, i0, nqi, steps;
+};
+
+// Unit t of the work list, heaviest first: key tiles are the slow index, so
+// under a causal mask the tiles seen by the most query tiles (small j) come
+// first.  Every key tile has at least one query tile (causal needs Sq <= Sk,
+// bottom-right aligned), so steps >= 1.
+__device__ __forceinline__ DkdvUnit dkdv_unit(const BwdArgs& a, int t) {
+  const int BH = a.B * a.Hkv;
+  DkdvUnit u;
+  u.j = t / BH;
+  u.bkv = t - u.j * BH;
+  const int nq = (a.Sq + kTile - 1) / kTile;
+  u.i0 = bwd_first_q_tile(u.j, a.Sq, a.Sk, a.causal);
+  u.nqi = nq - u.i0;
+  u.steps = (a.Hq / a.Hkv) * u.nqi;
+  return u;
+}
+
+// Persistent: one CTA per SM walks its units (dealt out in snake order, as in
+// the dQ kernel).  A unit's dK / dV rows are summed over its steps in the same
+// order whichever CTA runs it.  Across units the Q / dO / statistics rings,
+// the S^T / dP^T buffers and every barrier phase continue on one global step
+// count; the next unit's K and V load as soon as the current unit's last S^T
+// and dP^T have read the old ones (kv_empty), and its first S^T and dP^T run
+// during the current unit's last step and epilogue.  Its first dV MMA cannot
+// overwrite the accumulators early: it waits for that unit's first P^T, which
+// the compute warps write only after reading dV and dK out.
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using L = DkdvSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -223,16 +263,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   }
   uint8_t* smem = smem_raw;
   const int warp = warp_id(), lane = lane_id();
-
-  // Key tiles are the slow grid index so that, under a causal mask, the tiles
-  // with the most query tiles (small j) are launched first.
-  const int j = blockIdx.y;                      // key tile
-  const int bkv = blockIdx.x;                    // b * Hkv + kv head
-  const int b = bkv / a.Hkv, kvh = bkv - b * a.Hkv;
+  const int n_units = ((a.Sk + kTile - 1) / kTile) * a.B * a.Hkv;
+  const int cta = blockIdx.x, n_cta = gridDim.x;
   const int G = a.Hq / a.Hkv;
-  const int nq = (a.Sq + kTile - 1) / kTile;
-  const int i0 = bwd_first_q_tile(j, a.Sq, a.Sk, a.causal);
-  const int steps = G * (nq - i0);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* kv_full = bars + 0;
@@ -243,14 +276,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   uint64_t* s_full = bars + 11;      // [2] S^T columns of query half 0 / 1
   uint64_t* dp_full = bars + 13;
   uint64_t* p_full = bars + 14;      // [2] P^T of query half 0 / 1 written
-  uint64_t* acc_done = bars + 16;
+  uint64_t* acc_done = bars + 16;    // a unit's dK / dV MMAs have completed
   uint64_t* ds_full = bars + 17;     // dS^T written
   uint64_t* st_full = bars + 18;     // [2] LSE / Delta of a step staged (32 producer lanes)
   uint64_t* st_empty = bars + 20;    // [2] the compute warps are done with them (one arrival per warp)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* kv_empty = bars + 22;    // a unit's last S^T and dP^T have read K and V
+  uint64_t* mma_drain = bars + 23;   // every MMA of the CTA has completed (committed once, at exit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(mma_drain, 1);
     for (int s = 0; s < L::kQStages; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < L::kDOStages; ++s) { mbar_init(&do_full[s], 1); mbar_init(&do_empty[s], 1); }
     for (int s = 0; s < L::kStatStages; ++s) { mbar_init(&st_full[s], 32); mbar_init(&st_empty[s], kBwdComputeWarps); }
@@ -272,58 +309,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * kTileBytesBf16);
-      tma_tile_bf16(smem + L::kK, &a.tm_k, kv_full, j * kTile, bkv);
-      tma_tile_bf16(smem + L::kV, &a.tm_v, kv_full, j * kTile, bkv);
-    }
     bool ok = true;
-    for (int n = 0; n < steps && ok; ++n) {
-      const int g = n / (nq - i0), i = i0 + n % (nq - i0);
-      const int bh = b * a.Hq + kvh * G + g;
-      const int qs = n % L::kQStages, qu = n / L::kQStages;
-      if (n >= L::kQStages) ok = warp_wait(&q_empty[qs], (qu - 1) & 1, kSiteBwdStEmpty);
+    int ul = 0, n0 = 0;                          // units started, global step count at the unit's start
+    for (int k = 0; ok; ++k) {
+      const int t = dq_unit_index(k, cta, n_cta);
+      if (t >= n_units) break;
+      const DkdvUnit u = dkdv_unit(a, t);
+      const int b = u.bkv / a.Hkv, kvh = u.bkv - b * a.Hkv;
+      if (ul > 0) ok = warp_wait(kv_empty, (ul - 1) & 1, kSiteBwdKV);   // the last unit's S^T / dP^T are done
       if (!ok) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[qs], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kQ + qs * kTileBytesBf16, &a.tm_q, &q_full[qs], i * kTile, bh);
+        mbar_arrive_expect_tx(kv_full, 2 * kTileBytesBf16);
+        tma_tile_bf16(smem + L::kK, &a.tm_k, kv_full, u.j * kTile, u.bkv);
+        tma_tile_bf16(smem + L::kV, &a.tm_v, kv_full, u.j * kTile, u.bkv);
       }
-      const int ds = n % L::kDOStages, du = n / L::kDOStages;
-      if (n >= L::kDOStages) ok = warp_wait(&do_empty[ds], (du - 1) & 1, kSiteBwdStEmpty);
-      if (!ok) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&do_full[ds], kTileBytesBf16);
-        tma_tile_bf16(smem + L::kDO + ds * kTileBytesBf16, &a.tm_do, &do_full[ds], i * kTile, bh);
-      }
-      const int ss = n % L::kStatStages, su = n / L::kStatStages;
-      if (n >= L::kStatStages) ok = warp_wait(&st_empty[ss], (su - 1) & 1, kSiteBwdStEmpty);
-      if (!ok) break;
-      float* stats = reinterpret_cast<float*>(smem + L::kStats + ss * 2 * kTile * 4);
-      {
-        // all eight global loads in flight before the first store
-        float lv[kTile / 32], dv[kTile / 32];
-#pragma unroll
-        for (int k = 0; k < kTile / 32; ++k) {
-          const int qi = i * kTile + lane + 32 * k;
-          const bool valid = qi < a.Sq;
-          const size_t idx = (size_t)bh * a.Sq + (valid ? qi : 0);
-          lv[k] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
-          dv[k] = valid ? __ldg(&a.delta[idx]) : 0.f;
+      for (int s = 0; s < u.steps && ok; ++s) {
+        const int n = n0 + s;
+        const int g = s / u.nqi, i = u.i0 + s % u.nqi;
+        const int bh = b * a.Hq + kvh * G + g;
+        const int qs = n % L::kQStages, qu = n / L::kQStages;
+        if (n >= L::kQStages) ok = warp_wait(&q_empty[qs], (qu - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full[qs], kTileBytesBf16);
+          tma_tile_bf16(smem + L::kQ + qs * kTileBytesBf16, &a.tm_q, &q_full[qs], i * kTile, bh);
         }
-#pragma unroll
-        for (int k = 0; k < kTile / 32; ++k) {
-          stats[lane + 32 * k] = lv[k];
-          stats[kTile + lane + 32 * k] = dv[k];
+        const int ds = n % L::kDOStages, du = n / L::kDOStages;
+        if (n >= L::kDOStages) ok = warp_wait(&do_empty[ds], (du - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&do_full[ds], kTileBytesBf16);
+          tma_tile_bf16(smem + L::kDO + ds * kTileBytesBf16, &a.tm_do, &do_full[ds], i * kTile, bh);
         }
+        const int ss = n % L::kStatStages, su = n / L::kStatStages;
+        if (n >= L::kStatStages) ok = warp_wait(&st_empty[ss], (su - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        float* stats = reinterpret_cast<float*>(smem + L::kStats + ss * 2 * kTile * 4);
+        {
+          // all eight global loads in flight before the first store
+          float lv[kTile / 32], dv[kTile / 32];
+#pragma unroll
+          for (int kk = 0; kk < kTile / 32; ++kk) {
+            const int qi = i * kTile + lane + 32 * kk;
+            const bool valid = qi < a.Sq;
+            const size_t idx = (size_t)bh * a.Sq + (valid ? qi : 0);
+            lv[kk] = valid ? __ldg(&a.lse[idx]) * 1.4426950408889634f : INFINITY;   // P = 0 past Sq
+            dv[kk] = valid ? __ldg(&a.delta[idx]) : 0.f;
+          }
+#pragma unroll
+          for (int kk = 0; kk < kTile / 32; ++kk) {
+            stats[lane + 32 * kk] = lv[kk];
+            stats[kTile + lane + 32 * kk] = dv[kk];
+          }
+        }
+        mbar_arrive(&st_full[ss]);
       }
-      mbar_arrive(&st_full[ss]);
+      n0 += u.steps;
+      ++ul;
     }
     // drain: every load issued must land before the CTA exits
     if (lane == 0) {
-      mbar_wait_drain(kv_full, 0, kSiteBwdKV);
-      for (int n = max(0, steps - L::kQStages); n < steps; ++n)
+      if (ul > 0) mbar_wait_drain(kv_full, (ul - 1) & 1, kSiteBwdKV);
+      for (int n = max(0, n0 - L::kQStages); n < n0; ++n)
         mbar_wait_drain(&q_full[n % L::kQStages], (n / L::kQStages) & 1, kSiteBwdStFull);
-      for (int n = max(0, steps - L::kDOStages); n < steps; ++n)
+      for (int n = max(0, n0 - L::kDOStages); n < n0; ++n)
         mbar_wait_drain(&do_full[n % L::kDOStages], (n / L::kDOStages) & 1, kSiteBwdStFull);
     }
     __syncwarp();
@@ -343,53 +392,68 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       // one thread's MMAs run in order); then dK_n (once dS^T_n is written)
       // and dP^T_{n+1}.  The next step's first half of S^T thus runs while the
       // compute warps form the second half of P^T and then dS^T of this one.
-      bool ok = mbar_wait(kv_full, 0, kSiteBwdKV);
-      if (ok && steps > 0) ok = wait_q(0) && wait_do(0);
-      if (ok && steps > 0) {
+      bool ok = true;
+      int ul = 0, n0 = 0;
+      for (int k = 0; ok; ++k) {
+        const int t = dq_unit_index(k, cta, n_cta);
+        if (t >= n_units) break;
+        const int steps = dkdv_unit(a, t).steps;
+        const int n_end = n0 + steps;
+        ok = mbar_wait(kv_full, ul & 1, kSiteBwdKV);
+        if (ok) ok = wait_q(n0) && wait_do(n0);
+        if (!ok) break;
         tc_fence_after();
-        mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(0), 0);   // S^T  = K Q^T
+        mma_tile_ss_kmajor(tmem + 256, sK, sQ_of(n0), 0);   // S^T  = K Q^T
         mma_commit(&s_full[0]);
         mma_commit(&s_full[1]);
-        mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(0), 0);  // dP^T = V dO^T
+        mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(n0), 0);  // dP^T = V dO^T
         mma_commit(dp_full);
-      }
-      for (int n = 0; n < steps && ok; ++n) {
-        const bool more = n + 1 < steps;
-        ok = mbar_wait(&p_full[0], n & 1, kSiteBwdP);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tile_ts_mnmajor<0, 4>(tmem + 0, tmem + 256, sDO_of(n), n > 0);   // dV += P^T dO, queries 0..63
-        if (more) {
-          ok = wait_q(n + 1);
+        if (steps == 1) mma_commit(kv_empty);               // K and V read for the last time
+        for (int n = n0; n < n_end && ok; ++n) {
+          const bool more = n + 1 < n_end;
+          ok = mbar_wait(&p_full[0], n & 1, kSiteBwdP);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss_kmajor_n64(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step, half 0
-          mma_commit(&s_full[0]);
-        }
-        ok = mbar_wait(&p_full[1], n & 1, kSiteBwdP);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tile_ts_mnmajor<4, 8>(tmem + 0, tmem + 256, sDO_of(n), 1);       // queries 64..127
-        mma_commit(&do_empty[n % L::kDOStages]);
-        if (more) {
-          mma_tile_ss_kmajor_n64(tmem + 320, sK, sQ_of(n + 1), 1);          // half 1
-          mma_commit(&s_full[1]);
-        }
-        ok = mbar_wait(ds_full, n & 1, kSiteBwdP);
-        if (!ok) break;
-        tc_fence_after();
-        mma_tile_ts_mnmajor<0, 8>(tmem + 128, tmem + 384, sQ_of(n), n > 0);  // dK += dS^T Q
-        mma_commit(&q_empty[n % L::kQStages]);
-        if (more) {
-          ok = wait_do(n + 1);
+          mma_tile_ts_mnmajor<0, 4>(tmem + 0, tmem + 256, sDO_of(n), n > n0);   // dV += P^T dO, queries 0..63
+          if (more) {
+            ok = wait_q(n + 1);
+            if (!ok) break;
+            tc_fence_after();
+            mma_tile_ss_kmajor_n64(tmem + 256, sK, sQ_of(n + 1), 0);          // S^T of the next step, half 0
+            mma_commit(&s_full[0]);
+          }
+          ok = mbar_wait(&p_full[1], n & 1, kSiteBwdP);
           if (!ok) break;
           tc_fence_after();
-          mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(n + 1), 0);         // dP^T of the next step
-          mma_commit(dp_full);
+          mma_tile_ts_mnmajor<4, 8>(tmem + 0, tmem + 256, sDO_of(n), 1);       // queries 64..127
+          mma_commit(&do_empty[n % L::kDOStages]);
+          if (more) {
+            mma_tile_ss_kmajor_n64(tmem + 320, sK, sQ_of(n + 1), 1);          // half 1
+            mma_commit(&s_full[1]);
+          }
+          ok = mbar_wait(ds_full, n & 1, kSiteBwdP);
+          if (!ok) break;
+          tc_fence_after();
+          mma_tile_ts_mnmajor<0, 8>(tmem + 128, tmem + 384, sQ_of(n), n > n0);  // dK += dS^T Q
+          mma_commit(&q_empty[n % L::kQStages]);
+          if (more) {
+            ok = wait_do(n + 1);
+            if (!ok) break;
+            tc_fence_after();
+            mma_tile_ss_kmajor(tmem + 384, sV, sDO_of(n + 1), 0);         // dP^T of the next step
+            mma_commit(dp_full);
+            if (n + 2 == n_end) mma_commit(kv_empty);                    // the unit's last S^T and dP^T
+          }
         }
+        if (!ok) break;
+        mma_commit(acc_done);
+        n0 = n_end;
+        ++ul;
       }
-      mma_commit(acc_done);
-      mbar_wait(acc_done, 0, kSiteBwdDone);
+      // Drain (normal and error paths): no MMA may be in flight when tensor
+      // memory is freed.
+      mma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0, kSiteBwdDone);
     }
     __syncwarp();
   } else {
@@ -399,99 +463,107 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 256 + hc * 32;   // S^T (then P^T) columns of chunk 0; chunk 1 at +64
     const uint32_t tP = tmem + lane_base + 384 + hc * 32;   // dP^T (then dS^T) columns, same layout
-    const int kj = j * kTile + r;
     const float c = a.scale_log2;
     const float2 c2 = make_float2(c, c);
     bool ok = true;
-    for (int n = 0; n < steps && ok; ++n) {
-      const int i = i0 + n % (nq - i0);
-      const int ss = n % L::kStatStages;
-      ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
-      if (!ok) break;
-      // LSE (log2 domain) then Delta of the tile's 128 queries
-      const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + ss * 2 * kTile * 4) + hc * 8;
+    int ul = 0, n0 = 0;
+    for (int k = 0; ok; ++k) {
+      const int t = dq_unit_index(k, cta, n_cta);
+      if (t >= n_units) break;
+      const DkdvUnit u = dkdv_unit(a, t);
+      const int kj = u.j * kTile + r;
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
-      // P^T as bf16 pairs, per chunk: the values dV's MMA consumes, reused for dS^T
-      uint32_t pk[2][16];
+      for (int s = 0; s < u.steps && ok; ++s) {
+        const int n = n0 + s;
+        const int i = u.i0 + s % u.nqi;
+        const int ss = n % L::kStatStages;
+        ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
+        if (!ok) break;
+        // LSE (log2 domain) then Delta of the tile's 128 queries
+        const float4* stats4 = reinterpret_cast<const float4*>(smem + L::kStats + ss * 2 * kTile * 4) + hc * 8;
+        // P^T as bf16 pairs, per chunk: the values dV's MMA consumes, reused for dS^T
+        uint32_t pk[2][16];
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        ok = warp_wait(&s_full[ch], n & 1, kSiteBwdS);
+        for (int ch = 0; ch < 2; ++ch) {
+          ok = warp_wait(&s_full[ch], n & 1, kSiteBwdS);
+          if (!ok) break;
+          tc_fence_after();
+          const int q_first = i * kTile + ch * 64 + hc * 32;   // first query of these 32 columns
+          const bool need_mask = a.causal && (q_first < lim);
+          uint32_t uu[32];
+          tmem_ld32(tS + ch * 64, uu);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const int e = 4 * k4;
+            const float4 l4 = lds128(&stats4[ch * 16 + k4]);   // queries e .. e+3 of the chunk (broadcast)
+            const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1])), c2,
+                                         make_float2(-l4.x, -l4.y));
+            const float2 x1 = __ffma2_rn(make_float2(__uint_as_float(uu[e + 2]), __uint_as_float(uu[e + 3])), c2,
+                                         make_float2(-l4.z, -l4.w));
+            float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x), p3 = ex2_approx(x1.y);
+            if (need_mask) {
+              const int q0 = q_first + e;
+              p0 = q0 < lim ? 0.f : p0;
+              p1 = q0 + 1 < lim ? 0.f : p1;
+              p2 = q0 + 2 < lim ? 0.f : p2;
+              p3 = q0 + 3 < lim ? 0.f : p3;
+            }
+            pk[ch][e / 2] = pack_bf16x2(p0, p1);
+            pk[ch][e / 2 + 1] = pack_bf16x2(p2, p3);
+          }
+          __syncwarp();
+          tmem_st16(tS + ch * 64, pk[ch]);             // P^T over the first 16 of these columns
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[ch]);
+        }
+        if (!ok) break;
+        ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
         if (!ok) break;
         tc_fence_after();
-        const int q_first = i * kTile + ch * 64 + hc * 32;   // first query of these 32 columns
-        const bool need_mask = a.causal && (q_first < lim);
-        uint32_t u[32];
-        tmem_ld32(tS + ch * 64, u);
-        tmem_wait_ld();
 #pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const int e = 4 * k4;
-          const float4 l4 = lds128(&stats4[ch * 16 + k4]);   // queries e .. e+3 of the chunk (broadcast)
-          const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
-                                       make_float2(-l4.x, -l4.y));
-          const float2 x1 = __ffma2_rn(make_float2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3])), c2,
-                                       make_float2(-l4.z, -l4.w));
-          float p0 = ex2_approx(x0.x), p1 = ex2_approx(x0.y), p2 = ex2_approx(x1.x), p3 = ex2_approx(x1.y);
-          if (need_mask) {
-            const int q0 = q_first + e;
-            p0 = q0 < lim ? 0.f : p0;
-            p1 = q0 + 1 < lim ? 0.f : p1;
-            p2 = q0 + 2 < lim ? 0.f : p2;
-            p3 = q0 + 3 < lim ? 0.f : p3;
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t uu[32];
+          tmem_ld32(tP + ch * 64, uu);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            const int e = 4 * k4;
+            const float4 d4 = lds128(&stats4[kTile / 4 + ch * 16 + k4]);   // Delta of queries e .. e+3
+            const uint32_t w0 = pk[ch][e / 2], w1 = pk[ch][e / 2 + 1];
+            const float2 pa = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
+            const float2 pb = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
+            const float2 a0 = __fmul2_rn(pa, __fadd2_rn(make_float2(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1])),
+                                                        make_float2(-d4.x, -d4.y)));
+            const float2 a1 = __fmul2_rn(pb, __fadd2_rn(make_float2(__uint_as_float(uu[e + 2]), __uint_as_float(uu[e + 3])),
+                                                        make_float2(-d4.z, -d4.w)));
+            pk[ch][e / 2] = pack_bf16x2(a0.x, a0.y);
+            pk[ch][e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
           }
-          pk[ch][e / 2] = pack_bf16x2(p0, p1);
-          pk[ch][e / 2 + 1] = pack_bf16x2(p2, p3);
+          __syncwarp();
+          tmem_st16(tP + ch * 64, pk[ch]);             // dS^T over the first 16 of these columns
         }
-        __syncwarp();
-        tmem_st16(tS + ch * 64, pk[ch]);             // P^T over the first 16 of these columns
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[ch]);
-      }
-      if (!ok) break;
-      ok = warp_wait(dp_full, n & 1, kSiteBwdDP);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t uu[32];
-        tmem_ld32(tP + ch * 64, uu);
-        tmem_wait_ld();
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const int e = 4 * k4;
-          const float4 d4 = lds128(&stats4[kTile / 4 + ch * 16 + k4]);   // Delta of queries e .. e+3
-          const uint32_t w0 = pk[ch][e / 2], w1 = pk[ch][e / 2 + 1];
-          const float2 pa = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
-          const float2 pb = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
-          const float2 a0 = __fmul2_rn(pa, __fadd2_rn(make_float2(__uint_as_float(uu[e]), __uint_as_float(uu[e + 1])),
-                                                      make_float2(-d4.x, -d4.y)));
-          const float2 a1 = __fmul2_rn(pb, __fadd2_rn(make_float2(__uint_as_float(uu[e + 2]), __uint_as_float(uu[e + 3])),
-                                                      make_float2(-d4.z, -d4.w)));
-          pk[ch][e / 2] = pack_bf16x2(a0.x, a0.y);
-          pk[ch][e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
+        if (lane == 0) {
+          mbar_arrive(ds_full);
+          mbar_arrive(&st_empty[ss]);                  // done with this step's LSE / Delta
         }
-        __syncwarp();
-        tmem_st16(tP + ch * 64, pk[ch]);             // dS^T over the first 16 of these columns
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(ds_full);
-        mbar_arrive(&st_empty[ss]);                  // done with this step's LSE / Delta
-      }
-    }
-    if (ok) ok = warp_wait(acc_done, 0, kSiteBwdDone);
-    if (ok) {
+      if (ok) ok = warp_wait(acc_done, ul & 1, kSiteBwdDone);
+      if (!ok) break;
       tc_fence_after();
       // this warp stores head dims 64 hc .. 64 hc + 63 of its rows of dV and dK
       const bool store = kj < a.Sk;
-      const size_t off = ((size_t)bkv * a.Sk + (store ? kj : 0)) * kHeadDim + hc * 64;
+      const size_t off = ((size_t)u.bkv * a.Sk + (store ? kj : 0)) * kHeadDim + hc * 64;
       store_half_row_bf16(tmem + lane_base + 0 + hc * 64, 1.f, a.dv + off, store);
       store_half_row_bf16(tmem + lane_base + 128 + hc * 64, a.scale, a.dk + off, store);
+      n0 += u.steps;
+      ++ul;
     }
   }
 
@@ -540,12 +612,6 @@ __device__ __forceinline__ DqUnit dq_unit(const BwdArgs& a, int t) {
   }
   return u;
 }
-
-// The k-th unit of CTA c among G persistent CTAs: the heaviest-first list is
-// dealt out in snake order (c, then 2G-1-c, then 2G+c, ...), which evens out
-// the causal unit sizes.  Increasing in k, so the first index past the list
-// ends the CTA's loop.
-__device__ __forceinline__ int dq_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
 
 // Persistent: one CTA per SM walks its units.  Every unit's dQ rows are summed
 // over its KV tiles in ascending order by one CTA, as before; only which CTA
@@ -791,13 +857,17 @@ bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uin
 inline int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
                       float scale, bool causal, float* delta, int n_sm, cudaStream_t st) {
-  static bool attr_ok = [] {
-    return cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvSmem::kAlloc) ==
-               cudaSuccess &&
-           cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem::kAlloc) ==
-               cudaSuccess;
-  }();
-  if (!attr_ok) return -5;
+  // the shared-memory limits, once per device
+  static PerDeviceOnce setup;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -5;
+  if (!setup.ensure(dev, [] {
+        return cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    DkdvSmem::kAlloc) == cudaSuccess &&
+               cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem::kAlloc) ==
+                   cudaSuccess;
+      }))
+    return -5;
   static thread_local BwdArgs a;
   memset(&a, 0, sizeof(a));
   if (!encode_rows(&a.tm_q, q, false, Sq, (uint64_t)B * Hq)) return -5;
@@ -814,11 +884,17 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
   const long long rows = (long long)B * Hq * Sq;
+  const long long n_kt = (Sk + kTile - 1) / kTile, nq = (Sq + kTile - 1) / kTile;
+  const long long kv_units = n_kt * B * Hkv, dq_units = nq * B * Hq;
+  const int kv_grid = (int)std::min<long long>(kv_units, n_sm);
+  const int dq_grid = (int)std::min<long long>(dq_units, n_sm);
+  // each persistent CTA counts its steps (tile pairs) in an int
+  if ((kv_units + kv_grid - 1) / kv_grid * (Hq / Hkv) * nq >= (1LL << 31) ||
+      (dq_units + dq_grid - 1) / dq_grid * n_kt >= (1LL << 31))
+    return -2;
   bwd_delta_kernel<<<(unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta), 256, 0, st>>>(
       reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows);
-  bwd_dkdv_kernel<<<dim3(B * Hkv, (Sk + kTile - 1) / kTile), kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
-  const long long dq_units = (long long)((Sq + kTile - 1) / kTile) * B * Hq;
-  const int dq_grid = (int)std::min<long long>(dq_units, n_sm);
+  bwd_dkdv_kernel<<<kv_grid, kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
   bwd_dq_kernel<<<dq_grid, kBwdThreads, DqSmem::kAlloc, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }

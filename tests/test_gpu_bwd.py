@@ -56,6 +56,10 @@ def check(h, w):
     # take several units of different lengths
     (1, 24, 3, 1000, 1000, True),
     (2, 12, 4, 1100, 700, False),
+    # more key-tile units than SMs: the persistent dK/dV CTAs take several
+    # (352 and 160 units, causal, ragged tails, grouped heads)
+    (2, 16, 16, 1300, 1300, True),
+    (1, 40, 20, 900, 1000, True),
 ])
 def test_bwd_ragged(h, B, Hq, Hkv, Sq, Sk, causal):
     check(h, Workload("bw", B=B, Hq=Hq, Hkv=Hkv, Sq=Sq, Sk=Sk, causal=causal, seed=200 + Sq + Sk, backward=True))
