@@ -58,8 +58,13 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)",
                   "bf16_75600": "bf16 attention fwd at the fp8 shape (B1 H5 S75600 D128)",
                   "fp8_32760": "fp8 e4m3 attention fwd at the video shape (B1 H40 S32760 D128, Q/K RMS-norm)",
-                  "fp8_prep": "e4m3 prologue of the fp8 config (Q, K RMS-normalised; V plain; per-head descales)"}
+                  "fp8_prep": "e4m3 prologue of the fp8 config (Q, K RMS-normalised; V plain; per-head descales)",
+                  "fp8_noscratch": "fp8 e4m3 attention fwd without scratch, V widened in shared memory "
+                                   "(B1 H5 S75600 D128)",
+                  "fp8_streaming": "streaming block-KV fwd over an FP8 e4m3 KV cache (B1 H40 Sq1560, 21x1560 blocks "
+                                   "with per-block descales, + 512 e4m3 text keys)"}
 FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window", "bf16_75600", "fp8_32760")
+SUB_ONLY = ("fp8_prep", "fp8_noscratch", "fp8_streaming")     # measured as sub-results only
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
 
@@ -195,7 +200,7 @@ class Step:
     def __init__(self, name, h, heads=None, rank=0):
         self.name = name
         self.h = h
-        base = "fp8" if name == "fp8_prep" else name
+        base = {"fp8_prep": "fp8", "fp8_noscratch": "fp8", "fp8_streaming": "streaming"}.get(name, name)
         self.w = workloads.get(base)
         if heads:
             self.w = workloads.get(base, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
@@ -238,6 +243,37 @@ class Step:
             self.bytes = sum(5.0 * t.numel() for t in self.src)   # x read twice, codes written once
             self.launches = 6                                       # 3 x 2 kernels (and a memset each)
             self.dtype = "e4m3"
+        elif name == "fp8_noscratch":
+            x = make_fwd_inputs(w)
+            self.host = x
+            self.x = {k: v.cuda() for k, v in x.items()}
+            self.out = torch.empty((w.B, w.Hq, w.Sq, w.D), dtype=torch.bfloat16, device="cuda")
+            self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
+            self.flops = w.fwd_flops()
+            self.dtype = "e4m3"
+        elif name == "fp8_streaming":
+            # an FP8 KV cache: every block (and the text keys) quantised with its
+            # own per-head descales by the product prologue, outside the timed step
+            x = make_kvblock_inputs(w)
+            self.q, self.qd = h.quantize_e4m3(x["q"].cuda(), rmsnorm=True)
+            n = len(x["blocks"])
+            self.kds = torch.empty(n, w.B, w.Hkv, dtype=torch.float32, device="cuda")
+            self.vds = torch.empty_like(self.kds)
+            self.kb, self.vb = [], []
+            for i, (kb, vb) in enumerate(x["blocks"]):
+                self.kb.append(h.quantize_e4m3(kb.cuda(), rmsnorm=True, descale=self.kds[i])[0])
+                self.vb.append(h.quantize_e4m3(vb.cuda(), descale=self.vds[i])[0])
+            self.tk, self.tkd = h.quantize_e4m3(x["text"][0].cuda(), rmsnorm=True)
+            self.tv, self.tvd = h.quantize_e4m3(x["text"][1].cuda())
+            self.out = torch.empty((w.B, w.Hq, w.Sq, w.D), dtype=torch.bfloat16, device="cuda")
+            self.lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device="cuda")
+            self.out_t = torch.empty_like(self.out)
+            self.lse_t = torch.empty_like(self.lse)
+            self.ws = torch.empty(h.fwd_workspace_size(w.B, w.Hkv, w.text_len, w.D, h.E4M3), dtype=torch.uint8,
+                                  device="cuda")
+            self.flops = 4.0 * w.B * w.Hq * w.Sq * w.D * (w.Sk + w.text_len)
+            self.launches = 3                       # the block-KV kernel; text keys: V widening + attention
+            self.dtype = "e4m3"
         elif name == "streaming":
             x = make_kvblock_inputs(w)
             self.host = x
@@ -265,6 +301,15 @@ class Step:
             if w.dtype == "e4m3":
                 ds = dict(q_descale=x["q_descale"], k_descale=x["k_descale"], v_descale=x["v_descale"])
             h.attn_fwd(x["q"], x["k"], x["v"], out=self.out, lse=self.lse, **ds)
+        elif self.name == "fp8_noscratch":
+            x = self.x
+            h.attn_fwd(x["q"], x["k"], x["v"], out=self.out, lse=self.lse, q_descale=x["q_descale"],
+                       k_descale=x["k_descale"], v_descale=x["v_descale"], use_scratch=False)
+        elif self.name == "fp8_streaming":
+            h.attn_fwd_kvblocks(self.q, self.kb, self.vb, out=self.out, lse=self.lse, q_descale=self.qd,
+                                k_descale=self.kds, v_descale=self.vds)
+            h.attn_fwd(self.q, self.tk, self.tv, out=self.out_t, lse=self.lse_t, q_descale=self.qd,
+                       k_descale=self.tkd, v_descale=self.tvd, workspace=self.ws)
         elif self.name == "fp8_prep":
             for i, (t, (c, d)) in enumerate(zip(self.src, self.dst)):
                 h.quantize_e4m3(t, rmsnorm=i < 2, codes=c, descale=d)
@@ -456,7 +501,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=[n for n in WORKLOAD_NAMES if n != "fp8_prep"], default="video")
+    ap.add_argument("--workload", choices=[n for n in WORKLOAD_NAMES if n not in SUB_ONLY], default="video")
     ap.add_argument("--no-sub", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true")

@@ -7,7 +7,9 @@ The GPU test calls it through the C ABI twice in a row, on two different
 problems, and checks each result against the workspace-taking attn_bwd with
 the gradient tolerance the parity tests use (max abs <= 2e-2 * max(1, max|ref|),
 normalised RMS <= 1e-2); both run the same kernels, so the results are also
-expected to be bit-identical.  This file is collected last on purpose.
+expected to be bit-identical.  A second GPU case fills the static array to
+its last row (B*Hq*Sq equal to the limit) and compares bit for bit with
+attn_bwd.  This file is collected last on purpose.
 """
 import ctypes
 
@@ -61,3 +63,28 @@ def test_noalloc_matches_workspace_backward_on_two_calls_in_a_row():
             e = grad_errors(g, r.double().cpu().numpy())
             assert grad_ok(e), (w.name, name, e)
             assert torch.equal(g.view(torch.int16), r.view(torch.int16)), (w.name, name)
+
+
+@pytest.mark.gpu
+def test_noalloc_at_the_row_limit_matches_workspace_backward():
+    # B*Hq*Sq == HATTN_NOALLOC_MAX_ROWS: 2048 query heads of 2048 rows against
+    # 128 keys each, so Delta fills the whole static array up to its last row
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    h = _h()
+    B, H, Sq, Sk = 1, 2048, 2048, 128
+    assert B * H * Sq == h.NOALLOC_MAX_ROWS
+    g = torch.Generator(device="cuda").manual_seed(403)
+    q, dout = (torch.randn(B, H, Sq, 128, generator=g, device="cuda").to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn(B, H, Sk, 128, generator=g, device="cuda").to(torch.bfloat16) for _ in range(2))
+    out, lse = h.attn_fwd(q, k, v)
+    rdq, rdk, rdv = h.attn_bwd(q, k, v, out, lse, dout)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    rc = h.lib.attn_bwd_noalloc(p(q), p(k), p(v), p(out), p(lse), p(dout), p(dq), p(dk), p(dv), B, H, H, Sq, Sk,
+                                128, 1.0 / 128 ** 0.5, 0, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, h.lib.attn_error_string(rc)
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    for name, a, b in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), name
