@@ -56,6 +56,8 @@ struct BwdArgs {
   uint16_t* dq;           // [B,Hq,Sq,D] bf16
   uint16_t* dk;           // [B,Hkv,Sk,D]
   uint16_t* dv;
+  float* dq_acc;          // one-pass backward: fp32 dQ accumulator [B,Hq,Sq,D]
+  uint32_t* dq_cnt;       // one-pass backward: contributions added, per (b, q head, query tile)
 };
 
 enum : int {

@@ -19,6 +19,7 @@
 
 #include "../../include/hattn.h"
 #include "bwd_kernel.cuh"
+#include "bwd_onepass_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "per_device.h"
 #include "prep_kernel.cuh"
@@ -38,6 +39,12 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait_for(&bar, 0, kSiteSelfTest, limit_ns);
   __syncwarp();
+}
+
+// Self-test of the bounded counter wait the one-pass backward orders its dQ
+// additions with: one thread waits for a counter that nothing increments.
+__global__ void selftest_counter_kernel(const uint32_t* counter, unsigned long long limit_ns) {
+  if (threadIdx.x == 0) wait_counter_geq(counter, 1u, kSiteOpOrder, limit_ns);
 }
 
 namespace {
@@ -421,6 +428,31 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
                     reinterpret_cast<float*>(workspace), sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  size_t off_acc = 0, off_cnt = 0;
+  return onepass_workspace_parts(B, Hq, Sq, &off_acc, &off_cnt);
+}
+
+int attn_bwd_onepass(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                     float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if (Sk <= 0) return HATTN_EINVAL;
+  if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
+  if (!bwd_sizes_ok(B, Hq, Hkv, Sq, Sk)) return HATTN_EUNSUPPORTED;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return HATTN_EALIGN;
+  if (workspace_bytes < attn_bwd_onepass_workspace_size(B, Hq, Sq)) return HATTN_EWORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HATTN_ELAUNCH;
+  return launch_bwd_onepass(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, workspace,
+                            sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------- allocation-free backward
 // Scratch for attn_bwd_noalloc: the Delta vector (one fp32 per query row) lives
 // in this file-scope device array instead of a caller-provided workspace.
@@ -474,6 +506,14 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
 int attn_selftest_bounded_wait(void* stream, unsigned int timeout_us) {
   if (timeout_us == 0 || timeout_us > 10000000u) return HATTN_EINVAL;
   selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(1000ull * timeout_us);
+  return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
+}
+
+int attn_selftest_counter_wait(const void* counter, void* stream, unsigned int timeout_us) {
+  if (!counter || timeout_us == 0 || timeout_us > 10000000u) return HATTN_EINVAL;
+  if (reinterpret_cast<uintptr_t>(counter) & 3u) return HATTN_EALIGN;
+  selftest_counter_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(counter), 1000ull * timeout_us);
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 

@@ -226,6 +226,13 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt
          ((uint32_t)(M >> 4) << 24);
 }
 
+// The same with A's major order chosen too (bit 15: 1 = A is MN-major, i.e.
+// contiguous along M, as when A is held transposed in shared memory).
+__host__ __device__ constexpr uint32_t make_idesc_ab(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn_major,
+                                                     uint32_t b_mn_major, int M, int N) {
+  return make_idesc(a_fmt, b_fmt, b_mn_major, M, N) | (a_mn_major << 15);
+}
+
 // Shared-memory matrix descriptor (sm100 layout, version 1), 128-byte swizzle.
 //   [0,14) start address >> 4; [16,30) leading byte offset >> 4;
 //   [32,46) stride byte offset >> 4; [46,48) version = 1; [61,64) layout (2 = SWIZZLE_128B).
@@ -274,6 +281,46 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// ----------------------------------------------------------------- global memory ordering
+// Acquire load / release reduction of a 32-bit counter at GPU scope, for
+// ordering work between thread blocks.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// The fence releases this thread's earlier writes and, cumulatively, those of
+// other threads it has synchronised with (e.g. by __syncwarp) before it.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Four fp32 additions at a 16-byte aligned global address, performed in memory.
+__device__ __forceinline__ void red_add_v4(float* p, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// Wait until *p >= target (acquire).  Gives up like mbar_wait (returns false,
+// error word 0x100 | site) after limit_ns or once another thread block has
+// raised an error.
+__device__ __forceinline__ bool wait_counter_geq(const uint32_t* p, uint32_t target, int site,
+                                                 uint64_t limit_ns = 2000ull * 1000ull * 1000ull) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if ((it & 63u) == 0) {
+      if (error_raised()) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        raise_error(0x100 | site);
+        return false;
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -189,6 +189,31 @@ HATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* 
 HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
 
 /*
+ * One-pass deterministic backward (RL-Kernel PR #319: deterministic mha_bwd,
+ * "What the strict contract costs"): the same dQ, dK, dV as attn_bwd (same
+ * arguments and layouts, bf16 only), computed by one kernel that forms each
+ * tile pair's dQ contribution where dS is made (5 matrix products per pair of
+ * 128-row tiles instead of attn_bwd's 7) and adds it into an fp32 dQ
+ * accumulator in ascending key-tile order, ordered by counters in the
+ * workspace (bounded waits; a wait that gives up sets the device error word).
+ * Results are bitwise reproducible and independent of batch composition and
+ * head split; they are not bitwise those of attn_bwd (dK and dV sum the
+ * query tiles in another fixed order).  The kernel is launched cooperatively
+ * (all its thread blocks resident at once), which the ordering relies on.
+ *   workspace: at least attn_bwd_onepass_workspace_size(B, Hq, Sq) bytes:
+ *   Delta, the fp32 dQ accumulator (B*Hq*Sq*D*4 bytes) and the counters; its
+ *   contents on entry do not matter (the counters are cleared by a memset
+ *   enqueued on `stream`).
+ */
+HATTN_API int attn_bwd_onepass(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_bwd_onepass needs (for D = 128). */
+HATTN_API size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq);
+
+/*
  * Backward without a workspace argument, for callers that cannot allocate
  * device memory at call time -- for example a plug-in running inside a host
  * framework that owns the GPU allocator and its memory budget, or an engine
@@ -235,6 +260,17 @@ HATTN_API int attn_get_device_error(void* stream, int* code_out);
  * or HATTN_ELAUNCH.
  */
 HATTN_API int attn_selftest_bounded_wait(void* stream, unsigned int timeout_us);
+
+/*
+ * Failure-detection self-test of the bounded wait on a global counter that
+ * attn_bwd_onepass orders its dQ additions with (no counterpart on the
+ * pages): one thread waits for the 32-bit device word `counter` (4-byte
+ * aligned; the caller keeps it below 1 while the kernel runs) to reach 1,
+ * with a limit of timeout_us microseconds (1 .. 10^7).  The wait gives up,
+ * sets the device error word to 0x12A (0x100 | site 0x2A) and the kernel
+ * returns normally.  Returns 0, HATTN_EINVAL, HATTN_EALIGN or HATTN_ELAUNCH.
+ */
+HATTN_API int attn_selftest_counter_wait(const void* counter, void* stream, unsigned int timeout_us);
 
 /* Static text for a return code. */
 HATTN_API const char* attn_error_string(int code);

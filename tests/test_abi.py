@@ -200,6 +200,24 @@ def test_bwd_fails_closed(h):
     assert call(causal=1, Sq=256, Sk=128) == -2
 
 
+def test_bwd_onepass_fails_closed(h):
+    lib = h.lib
+    need = h.bwd_onepass_workspace_size(1, 2, 128)
+    assert need >= 2 * 128 * 128 * 4 + 2 * 128 * 4                 # dQ accumulator and Delta at least
+
+    def call(ws=A, wsb=need, causal=0, Sq=128, Sk=128, D=128, dq=A):
+        return lib.attn_bwd_onepass(A, A, A, A, A, A, dq, A, A, 1, 2, 2, Sq, Sk, D, 0.088, causal, ws, wsb, None)
+
+    assert call(wsb=need - 1) == -4
+    assert call(ws=None) == -1
+    assert call(dq=None) == -1
+    assert call(dq=MIS) == -3
+    assert call(D=96) == -2
+    assert call(causal=1, Sq=256, Sk=128) == -2
+    # a counter that is not 4-byte aligned is refused before anything is launched
+    assert lib.attn_selftest_counter_wait(ctypes.c_void_p(0x20001), None, 1000) == -3
+
+
 def test_error_strings(h):
     for c in (0, -1, -2, -3, -4, -5, -6, -99):
         assert isinstance(h.lib.attn_error_string(c), bytes)

@@ -46,9 +46,28 @@ def test_bounded_wait_gives_up_and_context_survives(h):
     assert e["o_max_abs"] <= O_MAX_ABS and e["lse_max_abs"] <= LSE_MAX_ABS
 
 
+def test_counter_wait_gives_up_and_context_survives(h):
+    # the bounded wait the one-pass backward orders its dQ additions with: a
+    # counter that nothing increments, a 100 ms limit
+    counter = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert h.get_device_error() == 0
+    assert h.lib.attn_selftest_counter_wait(ctypes.c_void_p(counter.data_ptr()), stream, 100_000) == 0
+    assert h.get_device_error() == 0x12A                                  # 0x100 | ordered-add site
+    assert h.get_device_error() == 0
+    w = Workload("after2", B=1, Hq=2, Hkv=1, Sq=300, Sk=300, causal=True, seed=76)
+    x = {k: v.cuda() for k, v in make_bwd_inputs(w).items()}
+    out, lse = h.attn_fwd(x["q"], x["k"], x["v"], causal=True)
+    dq, dk, dv = h.attn_bwd_onepass(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True)
+    dq2, dk2, dv2 = h.attn_bwd(x["q"], x["k"], x["v"], out, lse, x["dout"], causal=True)
+    assert h.get_device_error() == 0
+    assert (dq.float() - dq2.float()).abs().max() < 2e-2
+
+
 def test_selftest_rejects_bad_limits(h):
     assert h.lib.attn_selftest_bounded_wait(None, 0) == -1
     assert h.lib.attn_selftest_bounded_wait(None, 20_000_000) == -1
+    assert h.lib.attn_selftest_counter_wait(None, None, 1000) == -1
 
 
 def test_cuda_graph_capture_matches_eager(h):
