@@ -27,11 +27,12 @@
 // Ordered dQ: an fp32 accumulator per (b, query head, query tile) in the
 // workspace and a counter next to it.  The key tiles that see query tile i are
 // j = 0 .. jlast(i) (causal masks are bottom-right aligned, so key tile 0 sees
-// every query), and tile j adds its part only after tiles 0 .. j-1 have:
-// each compute warp waits until the counter has reached 8 j (eight warps per
-// contributor), stores (j = 0), adds in memory (red.add) or, as the last
-// contributor, adds, scales and writes the bf16 dQ rows, then releases one
-// count.  Every dQ element is therefore summed over j in ascending order,
+// every query), and tile j adds its part only after tiles 0 .. j-1 have.  Four
+// writer warps take the dQ tile out of tensor memory (so the next step's MMAs
+// can use the columns at once) and then each waits until the counter has
+// reached 4 j (four writer warps per contributor), stores (j = 0), adds in
+// memory (red.add) or, as the last contributor, adds, scales and writes the
+// bf16 dQ rows, then releases one count.  Every dQ element is therefore summed over j in ascending order,
 // whichever thread block adds which part: the result is bitwise the same
 // from run to run and for any batch composition or head split.  Because all
 // key tiles of a head visit their common (i, g) steps at the same step index,
@@ -40,6 +41,13 @@
 // and all CTAs are resident (cooperative launch, one CTA per SM), so the
 // unfinished unit with the smallest index can always proceed; waits are
 // bounded all the same and report through the device error word.
+//
+// Cost on B200 (interleaved A/B, same inputs): slower than the two-kernel
+// backward, e.g. 0.372 vs 0.261 ms on B2 Hq32 Hkv8 S2048 causal.  Every tile
+// pair moves a 64 KB fp32 dQ tile through L2 atomics (570 MB on that config;
+// an L2 reduction of 64 KB from every SM at once takes about 1.6 us, as much as
+// a step of the dQ kernel it replaces), and without any ordering at all (a
+// memset, unordered red.add, a conversion pass) it still takes 0.319 ms.
 #pragma once
 
 #include "bwd_kernel.cuh"
@@ -47,6 +55,20 @@
 namespace hattn {
 
 enum : int { kSiteOpDqFull = 40, kSiteOpDqFree, kSiteOpOrder };
+
+// 512 threads: warps 0-7 compute (P^T, dS^T, the dK / dV epilogue), warp 8 TMA
+// producer, warp 9 MMA issuer, warps 10-11 no role, warps 12-15 dQ writers
+// (warp 12 + q reads the dQ tile's TMEM lane quarter q, all 128 columns, into
+// registers, releases the columns, then adds the rows in key-tile order).
+// setmaxnreg split over the four warpgroups: compute 128 (as launched),
+// producer / MMA 80, writers 176; they sum to the 128 x 512 registers the
+// launch holds (checked on the host: an increase the pool cannot satisfy
+// would wait forever).
+constexpr int kOnePassThreads = 512;
+constexpr int kOpRegsCompute = 128, kOpRegsOther = 80, kOpRegsWriter = 176;
+constexpr int kOpRegsNeeded = (2 * kOpRegsCompute + kOpRegsOther + kOpRegsWriter) * 128;
+static_assert(kOpRegsNeeded <= 65536, "setmaxnreg split exceeds the register file");
+constexpr int kDqWriters = 4;
 
 struct OnePassSmem {
   static constexpr int kQStages = 2;
@@ -97,7 +119,7 @@ __device__ __forceinline__ void mma_tile_ss_mnA_mnB(uint32_t d, uint32_t sa, uin
     mma_f16_ss2(d, a_lo + k * (2048 >> 4), hi, b_lo + k * (2048 >> 4), hi, idesc, k > 0 ? 1u : 0u);
 }
 
-__global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(kOnePassThreads, 1) bwd_onepass_kernel(const __grid_constant__ BwdArgs a) {
   using L = OnePassSmem;
   extern __shared__ uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {              // the layout needs a 1024-byte aligned window
@@ -127,7 +149,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
   uint64_t* st_full = bars + 17;     // [2] LSE / Delta of a step staged (32 producer lanes)
   uint64_t* st_empty = bars + 19;    // [2] the compute warps are done with them
   uint64_t* dq_full = bars + 21;     // the step's dQ tile is in tensor memory
-  uint64_t* dq_free = bars + 22;     // the compute warps have read it out (one arrival per warp)
+  uint64_t* dq_free = bars + 22;     // the writers have read it out (one arrival per writer warp)
   uint64_t* mma_drain = bars + 23;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
 
@@ -146,7 +168,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
     mbar_init(ds_full, kBwdComputeWarps);
     mbar_init(acc_done, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, kBwdComputeWarps);
+    mbar_init(dq_free, kDqWriters);
     fence_barrier_init();
   }
   if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
@@ -155,6 +177,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8 && warp < 12) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOpRegsOther) : "memory");
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
     bool ok = true;
@@ -300,14 +324,89 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
       mbar_wait_drain(mma_drain, 0, kSiteBwdDone);
     }
     __syncwarp();
-  } else {
+  }
+  } else if (warp >= 12) {
+    // ---------------------------------------------------------------- dQ writers (warps 12-15)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kOpRegsWriter) : "memory");
+    const int r = (warp & 3) * 32 + lane;            // query row of the dQ tile (TMEM lane)
+    const uint32_t tQ = tmem + ((uint32_t)((warp & 3) * 32) << 16) + 384;
+    bool ok = true;
+    int n0 = 0;
+    for (int k = 0; ok; ++k) {
+      const int t = dq_unit_index(k, cta, n_cta);
+      if (t >= n_units) break;
+      const DkdvUnit u = dkdv_unit(a, t);
+      const int b = u.bkv / a.Hkv, kvh = u.bkv - b * a.Hkv;
+      for (int s = 0; s < u.steps && ok; ++s) {
+        const int n = n0 + s;
+        const int i = nq - 1 - s / G, g = s % G;
+        ok = warp_wait(dq_full, n & 1, kSiteOpDqFull);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t dq[128];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tQ + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&dq[32 * c4]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);          // the MMAs may take these columns again
+        const int bh = b * a.Hq + kvh * G + g;
+        const int jl = onepass_last_key_tile(a, i);
+        uint32_t* cnt = a.dq_cnt + (size_t)bh * nq + i;
+        if (u.j > 0) {
+          bool w = true;
+          if (lane == 0) w = wait_counter_geq(cnt, (uint32_t)kDqWriters * (uint32_t)u.j, kSiteOpOrder);
+          ok = __shfl_sync(0xffffffffu, w, 0);
+          if (!ok) break;
+        }
+        const int qi = i * kTile + r;
+        if (qi < a.Sq) {
+          const size_t row = (size_t)bh * a.Sq + qi;
+          float* acc = a.dq_acc + row * kHeadDim;
+          if (u.j == jl) {
+            // last contributor: dQ = scale * (sum of the earlier tiles + this one), bf16
+            uint4* dst = reinterpret_cast<uint4*>(a.dq + row * kHeadDim);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float v[8];
+#pragma unroll
+              for (int t2 = 0; t2 < 8; ++t2) v[t2] = __uint_as_float(dq[8 * e + t2]);
+              if (u.j > 0) {
+                const float4 p0 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * e));
+                const float4 p1 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * e + 4));
+                v[0] = p0.x + v[0]; v[1] = p0.y + v[1]; v[2] = p0.z + v[2]; v[3] = p0.w + v[3];
+                v[4] = p1.x + v[4]; v[5] = p1.y + v[5]; v[6] = p1.z + v[6]; v[7] = p1.w + v[7];
+              }
+              dst[e] = make_uint4(pack_bf16x2(v[0] * a.scale, v[1] * a.scale), pack_bf16x2(v[2] * a.scale, v[3] * a.scale),
+                                  pack_bf16x2(v[4] * a.scale, v[5] * a.scale), pack_bf16x2(v[6] * a.scale, v[7] * a.scale));
+            }
+          } else if (u.j == 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              __stcg(reinterpret_cast<float4*>(acc + 4 * e),
+                     make_float4(__uint_as_float(dq[4 * e]), __uint_as_float(dq[4 * e + 1]),
+                                 __uint_as_float(dq[4 * e + 2]), __uint_as_float(dq[4 * e + 3])));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              red_add_v4(acc + 4 * e, make_float4(__uint_as_float(dq[4 * e]), __uint_as_float(dq[4 * e + 1]),
+                                                  __uint_as_float(dq[4 * e + 2]), __uint_as_float(dq[4 * e + 3])));
+          }
+        }
+        if (u.j < jl) {
+          __syncwarp();
+          if (lane == 0) red_release_gpu_add(cnt, 1u);
+        }
+      }
+      n0 += u.steps;
+    }
+  } else if (warp < 8) {
     // ---------------------------------------------------------------- compute (warps 0-7)
-    const int r = (warp & 3) * 32 + lane;            // key row of S^T / P^T / dS^T; query row of the dQ tile
-    const int hc = warp >> 2;                        // queries 64 c + 32 hc .. +31 in chunk c; dQ dims 64 hc ..
+    const int r = (warp & 3) * 32 + lane;            // key row of S^T / P^T / dS^T
+    const int hc = warp >> 2;                        // queries 64 c + 32 hc .. +31 in chunk c
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + 256 + hc * 32;   // S^T (then P^T) columns of chunk 0; chunk 1 at +64
     const uint32_t tP = tmem + lane_base + 384 + hc * 32;   // dP^T columns, same layout
-    const uint32_t tQ = tmem + lane_base + 384 + hc * 64;   // this warp's 64 columns of the dQ tile
     uint8_t* sds_row = smem + L::kDS + r * 128;             // row r of each 64-query atom of dS^T
     const float c = a.scale_log2;
     const float2 c2 = make_float2(c, c);
@@ -317,12 +416,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
       const int t = dq_unit_index(k, cta, n_cta);
       if (t >= n_units) break;
       const DkdvUnit u = dkdv_unit(a, t);
-      const int b = u.bkv / a.Hkv, kvh = u.bkv - b * a.Hkv;
       const int kj = u.j * kTile + r;
       const int lim = kj - (a.Sk - a.Sq);            // key kj is masked for query qi iff qi < lim
       for (int s = 0; s < u.steps && ok; ++s) {
         const int n = n0 + s;
-        const int i = nq - 1 - s / G, g = s % G;
+        const int i = nq - 1 - s / G;
         const int ss = n % L::kStatStages;
         ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
         if (!ok) break;
@@ -402,64 +500,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_onepass_kernel(const __gri
           mbar_arrive(ds_full);
           mbar_arrive(&st_empty[ss]);
         }
-        // ---- this step's dQ tile: read it out, then add it in key-tile order
-        ok = warp_wait(dq_full, n & 1, kSiteOpDqFull);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t dq[64];
-        tmem_ld32(tQ, *reinterpret_cast<uint32_t(*)[32]>(&dq[0]));
-        tmem_ld32(tQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&dq[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dq_free);
-        const int bh = b * a.Hq + kvh * G + g;
-        const int jl = onepass_last_key_tile(a, i);
-        uint32_t* cnt = a.dq_cnt + (size_t)bh * nq + i;
-        if (u.j > 0) {
-          bool w = true;
-          if (lane == 0) w = wait_counter_geq(cnt, 8u * (uint32_t)u.j, kSiteOpOrder);
-          ok = __shfl_sync(0xffffffffu, w, 0);
-          if (!ok) break;
-        }
-        const int qi = i * kTile + r;
-        if (qi < a.Sq) {
-          const size_t row = (size_t)bh * a.Sq + qi;
-          float* acc = a.dq_acc + row * kHeadDim + hc * 64;
-          if (u.j == jl) {
-            // last contributor: dQ = scale * (sum of the earlier tiles + this one), bf16
-            uint4* dst = reinterpret_cast<uint4*>(a.dq + row * kHeadDim + hc * 64);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float v[8];
-#pragma unroll
-              for (int t2 = 0; t2 < 8; ++t2) v[t2] = __uint_as_float(dq[8 * e + t2]);
-              if (u.j > 0) {
-                const float4 p0 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * e));
-                const float4 p1 = __ldcg(reinterpret_cast<const float4*>(acc + 8 * e + 4));
-                v[0] = p0.x + v[0]; v[1] = p0.y + v[1]; v[2] = p0.z + v[2]; v[3] = p0.w + v[3];
-                v[4] = p1.x + v[4]; v[5] = p1.y + v[5]; v[6] = p1.z + v[6]; v[7] = p1.w + v[7];
-              }
-              dst[e] = make_uint4(pack_bf16x2(v[0] * a.scale, v[1] * a.scale), pack_bf16x2(v[2] * a.scale, v[3] * a.scale),
-                                  pack_bf16x2(v[4] * a.scale, v[5] * a.scale), pack_bf16x2(v[6] * a.scale, v[7] * a.scale));
-            }
-          } else if (u.j == 0) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              __stcg(reinterpret_cast<float4*>(acc + 4 * e),
-                     make_float4(__uint_as_float(dq[4 * e]), __uint_as_float(dq[4 * e + 1]),
-                                 __uint_as_float(dq[4 * e + 2]), __uint_as_float(dq[4 * e + 3])));
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              red_add_v4(acc + 4 * e, make_float4(__uint_as_float(dq[4 * e]), __uint_as_float(dq[4 * e + 1]),
-                                                  __uint_as_float(dq[4 * e + 2]), __uint_as_float(dq[4 * e + 3])));
-          }
-        }
-        if (u.j < jl) {
-          __syncwarp();
-          if (lane == 0) red_release_gpu_add(cnt, 1u);
-        }
       }
       if (ok) ok = warp_wait(acc_done, ul & 1, kSiteBwdDone);
       if (!ok) break;
@@ -498,9 +538,12 @@ inline int launch_bwd_onepass(const void* q, const void* k, const void* v, const
   if (cudaGetDevice(&dev) != cudaSuccess) return -5;
   if (!setup.ensure(dev, [dev] {
         int coop = 0;
+        cudaFuncAttributes fa;
         return cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop &&
                cudaFuncSetAttribute(bwd_onepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    OnePassSmem::kAlloc) == cudaSuccess;
+                                    OnePassSmem::kAlloc) == cudaSuccess &&
+               cudaFuncGetAttributes(&fa, bwd_onepass_kernel) == cudaSuccess &&
+               fa.numRegs * kOnePassThreads >= kOpRegsNeeded;   // the setmaxnreg split must fit the launch
       }))
     return -5;
   size_t off_acc = 0, off_cnt = 0;
@@ -535,7 +578,7 @@ inline int launch_bwd_onepass(const void* q, const void* k, const void* v, const
   if (cudaGetLastError() != cudaSuccess) return -5;
   // cooperative: every CTA is resident, which the ordered dQ adds rely on
   void* params[] = {&a};
-  if (cudaLaunchCooperativeKernel((const void*)bwd_onepass_kernel, dim3(grid), dim3(kBwdThreads), params,
+  if (cudaLaunchCooperativeKernel((const void*)bwd_onepass_kernel, dim3(grid), dim3(kOnePassThreads), params,
                                   OnePassSmem::kAlloc, st) != cudaSuccess)
     return -5;
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
