@@ -59,12 +59,13 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "bf16_75600": "bf16 attention fwd at the fp8 shape (B1 H5 S75600 D128)",
                   "fp8_32760": "fp8 e4m3 attention fwd at the video shape (B1 H40 S32760 D128, Q/K RMS-norm)",
                   "fp8_prep": "e4m3 prologue of the fp8 config (Q, K RMS-normalised; V plain; per-head descales)",
+                  "llm_gqa_onepass": "LLM GQA causal fwd + one-pass bwd (B2 Hq32 Hkv8 S2048 D128 bf16)",
                   "fp8_noscratch": "fp8 e4m3 attention fwd without scratch, V widened in shared memory "
                                    "(B1 H5 S75600 D128)",
                   "fp8_streaming": "streaming block-KV fwd over an FP8 e4m3 KV cache (B1 H40 Sq1560, 21x1560 blocks "
                                    "with per-block descales, + 512 e4m3 text keys)"}
 FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window", "bf16_75600", "fp8_32760")
-SUB_ONLY = ("fp8_prep", "fp8_noscratch", "fp8_streaming")     # measured as sub-results only
+SUB_ONLY = ("fp8_prep", "fp8_noscratch", "fp8_streaming", "llm_gqa_onepass")     # measured as sub-results only
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
 
@@ -200,7 +201,8 @@ class Step:
     def __init__(self, name, h, heads=None, rank=0):
         self.name = name
         self.h = h
-        base = {"fp8_prep": "fp8", "fp8_noscratch": "fp8", "fp8_streaming": "streaming"}.get(name, name)
+        base = {"fp8_prep": "fp8", "fp8_noscratch": "fp8", "fp8_streaming": "streaming",
+                "llm_gqa_onepass": "llm_gqa"}.get(name, name)
         self.w = workloads.get(base)
         if heads:
             self.w = workloads.get(base, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
@@ -219,7 +221,7 @@ class Step:
             self.dtype = w.dtype
             if w.dtype == "e4m3":
                 self.launches = 2          # V widened to fp16, then the attention kernel
-        elif name == "llm_gqa":
+        elif name in ("llm_gqa", "llm_gqa_onepass"):
             x = make_bwd_inputs(w)
             self.host = x
             self.x = {k: v.cuda() for k, v in x.items()}
@@ -228,9 +230,10 @@ class Step:
             self.dq = torch.empty_like(self.x["q"])
             self.dk = torch.empty_like(self.x["k"])
             self.dv = torch.empty_like(self.x["v"])
-            self.ws = torch.empty(h.bwd_workspace_size(w.B, w.Hq, w.Sq), dtype=torch.uint8, device="cuda")
+            wsb = h.bwd_onepass_workspace_size if name == "llm_gqa_onepass" else h.bwd_workspace_size
+            self.ws = torch.empty(wsb(w.B, w.Hq, w.Sq), dtype=torch.uint8, device="cuda")
             self.flops = w.fwd_flops() + w.bwd_flops()
-            self.launches = 4
+            self.launches = 4 if name == "llm_gqa" else 3      # fwd; Delta + dK/dV + dQ, or Delta + one pass
             self.dtype = "bf16"
         elif name == "fp8_prep":
             # the step before the fp8 forward: bf16 Q, K, V of the fp8 shape -> e4m3 + descales
@@ -313,11 +316,12 @@ class Step:
         elif self.name == "fp8_prep":
             for i, (t, (c, d)) in enumerate(zip(self.src, self.dst)):
                 h.quantize_e4m3(t, rmsnorm=i < 2, codes=c, descale=d)
-        elif self.name == "llm_gqa":
+        elif self.name in ("llm_gqa", "llm_gqa_onepass"):
             x = self.x
             h.attn_fwd(x["q"], x["k"], x["v"], causal=True, out=self.out, lse=self.lse)
-            h.attn_bwd(x["q"], x["k"], x["v"], self.out, self.lse, x["dout"], causal=True, workspace=self.ws,
-                       dq=self.dq, dk=self.dk, dv=self.dv)
+            bwd = h.attn_bwd_onepass if self.name == "llm_gqa_onepass" else h.attn_bwd
+            bwd(x["q"], x["k"], x["v"], self.out, self.lse, x["dout"], causal=True, workspace=self.ws,
+                dq=self.dq, dk=self.dk, dv=self.dv)
         else:
             h.attn_fwd_kvblocks(self.q, self.kb, self.vb, workspace=self.ws, out=self.out, lse=self.lse)
             h.attn_fwd(self.q, self.tk, self.tv, out=self.out_t, lse=self.lse_t)

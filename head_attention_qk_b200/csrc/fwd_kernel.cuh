@@ -72,22 +72,10 @@ constexpr int kRegsSoftmax = 208;
 constexpr int kRegsOther = 88;
 constexpr int kRegsNeeded = (2 * kRegsSoftmax + kRegsOther) * 128;
 static_assert(kRegsNeeded <= (65536 / 384) / 8 * 8 * 384, "setmaxnreg split exceeds a 384-thread launch");
-// Of every 8 pairs of softmax elements, this many take the software exp2
-// (FMA pipe) and the rest the MUFU ex2.  MUFU ex2 runs at 16 per clock per SM
-// in every format (measured: fp32, fp16 pairs and bf16 pairs alike), exactly
-// the bf16 MMA rate at D = 128 and three quarters of the fp8 QK^T + fp16 PV
-// rate, so the fp8 path moves a share of its exponentials to the FMA pipe.
-#ifndef HATTN_POLY_PAIRS_BF16
-#define HATTN_POLY_PAIRS_BF16 0
-#endif
-#ifndef HATTN_POLY_PAIRS_FP8
-#define HATTN_POLY_PAIRS_FP8 0
-#endif
-template <bool kFp8>
-struct PolyShare { static constexpr int kPairs = kFp8 ? HATTN_POLY_PAIRS_FP8 : HATTN_POLY_PAIRS_BF16; };
 
 struct FwdArgs {
   CUtensorMap tm_q;
+  CUtensorMap tm_o;              // bf16 O, stored by TMA from the persistent kernel
   CUtensorMap tm_k[kMaxKvBlocks];
   CUtensorMap tm_v[kMaxKvBlocks];
   int sk[kMaxKvBlocks];          // key length of each KV block (one block for attn_fwd)
@@ -106,7 +94,7 @@ struct FwdArgs {
   int fused_tiles;               // KV tiles over all fused blocks
 };
 
-template <bool kFp8, bool kWidenV = false>
+template <bool kFp8, bool kWidenV = false, bool kEpiStage = false>
 struct FwdSmemLayout {
   static_assert(!kWidenV || kFp8, "only e4m3 V is widened in shared memory");
   static constexpr int kElt = kFp8 ? 1 : 2;                            // Q and K element bytes
@@ -120,14 +108,21 @@ struct FwdSmemLayout {
   // ahead of the MMAs.  With kWidenV the ring has an even number of slots, so
   // every slot keeps one role (K in even slots, V in odd ones), and the widened
   // V tiles go through kStagesV16 fp16 buffers.
-  static constexpr int kRing = kWidenV ? 8 : (kFp8 ? 6 : 5);
+  // kEpiStage (the persistent kernel, bf16 O): one 32 KB slot's worth of the
+  // ring (two for the 16 KB e4m3 slots) becomes the O staging area.
+  static constexpr int kRing = kWidenV ? (kEpiStage ? 6 : 8) : (kFp8 ? (kEpiStage ? 5 : 6) : (kEpiStage ? 4 : 5));
   static_assert(!kWidenV || kRing % 2 == 0, "widening needs slots of one role");
   static constexpr int kStagesV16 = kWidenV ? 2 : 0;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = kQOff + kQTilesPerCta * kTileBytes;
   static constexpr int kV16Off = kRingOff + kRing * kSlotBytes;
-  static constexpr int kBarOff = kV16Off + kStagesV16 * kVTileBytes;
-  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8;
+  // O staging: per query tile, 128 rows x 64 columns of bf16 (16 KB, the
+  // layout of one 128-byte-swizzled TMA box); the epilogue stores each tile
+  // in two passes of 64 columns
+  static constexpr int kEpiTileBytes = kBlockM * 64 * 2;
+  static constexpr int kEpiOff = kV16Off + kStagesV16 * kVTileBytes;
+  static constexpr int kBarOff = kEpiOff + (kEpiStage ? kQTilesPerCta * kEpiTileBytes : 0);
+  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8 + 4;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -144,13 +139,15 @@ struct FwdBars {
   uint64_t* s_full;   // [2]: S_t ready
   uint64_t* p_full;   // [2 tiles][2 halves of 64 keys]: P_t,h written (128 arrivals)
   uint64_t* o_done;   // [2]: last P V of the tile completed
+  uint64_t* epi_full;   // [2]: a tile's staged O pass written (one arrival per warp of its group)
+  uint64_t* epi_empty;  // [2]: its TMA store has read the staging buffer
   uint32_t* tmem_slot;
 };
 
 // Barrier sites recorded in the error word when a wait times out.
 enum : int {
   kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty,
-  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain, kSiteV16Full, kSiteV16Empty
+  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain, kSiteV16Full, kSiteV16Empty, kSiteEpiFull, kSiteEpiEmpty
 };
 
 __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int q_row0) {
@@ -218,7 +215,8 @@ __device__ __forceinline__ bool fwd_more_units(int u, int u_first, int u_end, bo
 
 template <bool kFp8, bool kPartial, bool kPersist, bool kWidenV = false>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdArgs args) {
-  using L = FwdSmemLayout<kFp8, kWidenV>;
+  constexpr bool kEpiStage = kPersist && !kPartial;   // bf16 O staged in shared memory, stored by TMA
+  using L = FwdSmemLayout<kFp8, kWidenV, kEpiStage>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -242,6 +240,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     bb.s_full = p; p += 2;
     bb.p_full = p; p += 4;
     bb.o_done = p; p += 2;
+    bb.epi_full = p; p += 2;
+    bb.epi_empty = p; p += 2;
     bb.tmem_slot = reinterpret_cast<uint32_t*>(p);
   }
 
@@ -267,6 +267,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_init(&bb.p_full[2 * i], kBlockM / 32);
       mbar_init(&bb.p_full[2 * i + 1], kBlockM / 32);
       mbar_init(&bb.o_done[i], 1);
+      mbar_init(&bb.epi_full[i], kBlockM / 32);
+      mbar_init(&bb.epi_empty[i], 1);
     }
     fence_barrier_init();
   }
@@ -519,7 +521,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + tile * 128;
     const uint32_t tO = tmem + lane_base + 256 + tile * 128;
-    constexpr int kPolyPairs = PolyShare<kFp8>::kPairs;
+    const bool epi_leader = (threadIdx.x & (kBlockM - 1)) == 0;   // issues this group's O stores
 
     bool ok = true;
     uint32_t jg = 0;                                  // this CTA's tile count
@@ -641,17 +643,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           for (int e2 = 0; e2 < 32; ++e2) {
             const int e = half * 64 + 2 * e2;
             const float2 x = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, mneg2);
-            float2 p;
-            if ((e2 & 7) < kPolyPairs) {
-              // fp16 P (fp8 path) tolerates the quadratic, bf16 P takes the cubic
-              p = exp2_poly2<kFp8 ? 2 : 3>(x);
-              if (masked) {                               // the polynomial is never exactly 0
-                p.x = e > lim ? 0.f : p.x;
-                p.y = e + 1 > lim ? 0.f : p.y;
-              }
-            } else {
-              p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            }
+            const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
             pk[e2] = kFp8 ? pack_f16x2(p.x, p.y) : pack_bf16x2(p.x, p.y);
             acc[e2 & 3] = __fadd2_rn(acc[e2 & 3], p);
           }
@@ -675,6 +667,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       const bool store = row < args.Sq;
       const size_t orow = ((size_t)bh * args.Sq + (size_t)row) * kHeadDim;
       const size_t part = (size_t)(args.block_offset + w.blk);
+      if constexpr (kEpiStage) {
+        // O through shared memory, stored by TMA in two passes of 64 columns:
+        // each thread writes its row (128 bytes a pass, 16-byte chunks at
+        // chunk ^ (row & 7), the 128-byte swizzle of the tensor map), the
+        // group's leader stores the 128 x 64 box once all four warps have
+        // written; rows past Sq are clipped by the store.
+        uint8_t* stg = smem + L::kEpiOff + tile * L::kEpiTileBytes;
+        uint8_t* srow = stg + r * 128;
+        const int trow0 = w.q_row0 + tile * kBlockM;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t pc = 2u * (uint32_t)units + (uint32_t)h;    // this group's pass count
+          uint32_t uq[64];
+          __syncwarp();
+          tmem_ld32(tO + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&uq[0]));
+          tmem_ld32(tO + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&uq[32]));
+          tmem_wait_ld();
+          if (pc > 0) ok = warp_wait(&bb.epi_empty[tile], (pc - 1) & 1, kSiteEpiEmpty);   // last store has read it
+          if (!ok) break;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(srow + ((c ^ (r & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(uq[8 * c]) * inv_l, __uint_as_float(uq[8 * c + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(uq[8 * c + 2]) * inv_l, __uint_as_float(uq[8 * c + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(uq[8 * c + 4]) * inv_l, __uint_as_float(uq[8 * c + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(uq[8 * c + 6]) * inv_l, __uint_as_float(uq[8 * c + 7]) * inv_l));
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the TMA store reads it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bb.epi_full[tile]);
+          if (epi_leader) {
+            if (mbar_wait(&bb.epi_full[tile], pc & 1, kSiteEpiFull) && trow0 < args.Sq) {
+              tma_store_3d(&args.tm_o, stg, h * 64, trow0, bh);
+              bulk_commit();
+              bulk_wait_read();
+            }
+            mbar_arrive(&bb.epi_empty[tile]);
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t uq[32];
@@ -701,12 +732,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
           }
         }
       }
+      }
       if (store) {
         const float lse2 = (l > 0.f) ? (m + __log2f(l)) : -INFINITY;
         float* lse = args.lse + (kPartial ? part * ((size_t)args.B * args.Hq * args.Sq) : 0);
         lse[(size_t)bh * args.Sq + row] = lse2 * 0.69314718055994530942f;
       }
     }
+    if (kEpiStage && epi_leader) bulk_wait_all();   // O stores complete before the CTA exits
   }
 
   tc_fence_before();

@@ -96,7 +96,7 @@ int current_device() {
 
 template <bool kFp8, bool kPartial, bool kPersist, bool kWidenV>
 int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
-  using L = FwdSmemLayout<kFp8, kWidenV>;
+  using L = FwdSmemLayout<kFp8, kWidenV, kPersist && !kPartial>;
   auto kernel = attn_fwd_kernel<kFp8, kPartial, kPersist, kWidenV>;
   // once per device: the shared-memory limit, and the check that the
   // setmaxnreg split fits the registers the launch holds
@@ -213,6 +213,7 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
   static thread_local FwdArgs a;   // ~8 KB: kept off the stack
   memset(&a, 0, sizeof(a));
   if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+  if (!encode_rows(&a.tm_o, out, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
   if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
   if (fp8 && !v16) {
     if (!encode_rows(&a.tm_v[0], v, true, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
@@ -350,6 +351,7 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     // partials are written and no merge pass is needed.
     memset(&a, 0, sizeof(a));
     if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    if (!encode_rows(&a.tm_o, out, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
     long long tiles = 0;
     for (int i = 0; i < n_blocks; ++i) {
       if (!encode_rows(&a.tm_k[i], k_blocks[i], fp8, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;

@@ -142,6 +142,21 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// 3-D tiled TMA store from this CTA's shared memory (bulk-group completion).
+// Rows past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// This thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ----------------------------------------------------------------- tcgen05
 // Tensor memory address: bits [31:16] lane, bits [15:0] column.
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {
@@ -352,43 +367,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-// Software 2^x on the FMA/ALU pipes for a pair of values (Cody-Waite range
-// reduction, W. J. Cody and W. Waite 1980): j = floor(x), f = x - j in [0,1),
-// 2^x = 2^j * p(f), and 2^j is applied by adding j to p's exponent field.
-// p minimises the maximum relative error to 2^f on [0,1]; the coefficients are
-// fitted by csrc/fit_exp2_poly.py (degree 3: 7.5e-5, degree 2: 1.7e-3).  x is
-// clamped to >= -120 so the exponent never underflows (2^-120 is far below any
-// softmax row sum, which is >= 1).  floor(x) comes from a round-down add of
-// 1.5*2^23: the low mantissa bits of the sum then hold floor(x) in two's
-// complement, so (bits of the sum) * 2^23 is exactly j << 23 modulo 2^32,
-// added to p's bits by one integer multiply-add.
-constexpr float kExp2C0 = 9.999251962e-01f, kExp2C1 = 6.958335638e-01f, kExp2C2 = 2.260671407e-01f,
-                kExp2C3 = 7.802452892e-02f;
-constexpr float kExp2D2C0 = 1.001724720e+00f, kExp2D2C1 = 6.576362848e-01f, kExp2D2C2 = 3.371894360e-01f;
-
-template <int kDegree>
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  static_assert(kDegree == 2 || kDegree == 3, "degree 2 or 3");
-  x.x = fmaxf(x.x, -120.f);
-  x.y = fmaxf(x.y, -120.f);
-  const float2 t = __fadd2_rd(x, make_float2(12582912.f, 12582912.f));
-  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
-  float2 p;
-  if (kDegree == 3) {
-    p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-    p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
-    p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
-  } else {
-    p = __ffma2_rn(make_float2(kExp2D2C2, kExp2D2C2), f, make_float2(kExp2D2C1, kExp2D2C1));
-    p = __ffma2_rn(p, f, make_float2(kExp2D2C0, kExp2D2C0));
-  }
-  uint32_t rx, ry;
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(rx) : "r"(__float_as_uint(t.x)), "r"(__float_as_uint(p.x)));
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(ry) : "r"(__float_as_uint(t.y)), "r"(__float_as_uint(p.y)));
-  return make_float2(__uint_as_float(rx), __uint_as_float(ry));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
