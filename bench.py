@@ -494,6 +494,11 @@ def sub_result(other, h, flush, steps, warmup, peaks, heads=None):
         r = {"workload": WORKLOAD_NAMES[other], "ms_per_step": t, "tflops": st.flops / (t * 1e-3) / 1e12,
              "frac_of_peak": st.flops / (t * 1e-3) / 1e12 / pk, "peak_tflops": pk,
              "dtype": st.dtype, "launches_per_step": st.launches}
+        traffic = recorded_traffic(other)
+        if traffic is not None:
+            # DRAM bytes per launch of the attention kernel (ncu, profiles/traffic.json)
+            r["roofline"] = {"bound": "tensor", "traffic": traffic,
+                             "algorithmic_flops_per_launch": st.flops}
     del st
     torch.cuda.empty_cache()
     return r
