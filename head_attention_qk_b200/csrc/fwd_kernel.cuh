@@ -75,7 +75,7 @@ static_assert(kRegsNeeded <= (65536 / 384) / 8 * 8 * 384, "setmaxnreg split exce
 
 struct FwdArgs {
   CUtensorMap tm_q;
-  CUtensorMap tm_o;              // bf16 O, stored by TMA from the persistent kernel
+  CUtensorMap tm_o;              // bf16 O (boxes of 64 columns x 32 rows), stored by TMA from the persistent kernel
   CUtensorMap tm_k[kMaxKvBlocks];
   CUtensorMap tm_v[kMaxKvBlocks];
   int sk[kMaxKvBlocks];          // key length of each KV block (one block for attn_fwd)
@@ -122,7 +122,7 @@ struct FwdSmemLayout {
   static constexpr int kEpiTileBytes = kBlockM * 64 * 2;
   static constexpr int kEpiOff = kV16Off + kStagesV16 * kVTileBytes;
   static constexpr int kBarOff = kEpiOff + (kEpiStage ? kQTilesPerCta * kEpiTileBytes : 0);
-  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8 + 4;
+  static constexpr int kNumBars = 3 + 2 * kRing + 2 * kStagesV16 + 8;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;                       // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -139,15 +139,13 @@ struct FwdBars {
   uint64_t* s_full;   // [2]: S_t ready
   uint64_t* p_full;   // [2 tiles][2 halves of 64 keys]: P_t,h written (128 arrivals)
   uint64_t* o_done;   // [2]: last P V of the tile completed
-  uint64_t* epi_full;   // [2]: a tile's staged O pass written (one arrival per warp of its group)
-  uint64_t* epi_empty;  // [2]: its TMA store has read the staging buffer
   uint32_t* tmem_slot;
 };
 
 // Barrier sites recorded in the error word when a wait times out.
 enum : int {
   kSiteQFull = 1, kSiteKFull, kSiteKEmpty, kSiteVFull, kSiteVEmpty,
-  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain, kSiteV16Full, kSiteV16Empty, kSiteEpiFull, kSiteEpiEmpty
+  kSiteSFull, kSitePFull, kSiteODone, kSiteDrain, kSiteV16Full, kSiteV16Empty
 };
 
 __device__ __forceinline__ int fwd_num_kv_tiles(int sk, int Sq, int causal, int q_row0) {
@@ -240,8 +238,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     bb.s_full = p; p += 2;
     bb.p_full = p; p += 4;
     bb.o_done = p; p += 2;
-    bb.epi_full = p; p += 2;
-    bb.epi_empty = p; p += 2;
     bb.tmem_slot = reinterpret_cast<uint32_t*>(p);
   }
 
@@ -267,8 +263,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_init(&bb.p_full[2 * i], kBlockM / 32);
       mbar_init(&bb.p_full[2 * i + 1], kBlockM / 32);
       mbar_init(&bb.o_done[i], 1);
-      mbar_init(&bb.epi_full[i], kBlockM / 32);
-      mbar_init(&bb.epi_empty[i], 1);
     }
     fence_barrier_init();
   }
@@ -521,7 +515,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + tile * 128;
     const uint32_t tO = tmem + lane_base + 256 + tile * 128;
-    const bool epi_leader = (threadIdx.x & (kBlockM - 1)) == 0;   // issues this group's O stores
 
     bool ok = true;
     uint32_t jg = 0;                                  // this CTA's tile count
@@ -670,22 +663,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       if constexpr (kEpiStage) {
         // O through shared memory, stored by TMA in two passes of 64 columns:
         // each thread writes its row (128 bytes a pass, 16-byte chunks at
-        // chunk ^ (row & 7), the 128-byte swizzle of the tensor map), the
-        // group's leader stores the 128 x 64 box once all four warps have
-        // written; rows past Sq are clipped by the store.
-        uint8_t* stg = smem + L::kEpiOff + tile * L::kEpiTileBytes;
-        uint8_t* srow = stg + r * 128;
-        const int trow0 = w.q_row0 + tile * kBlockM;
+        // chunk ^ (row & 7), the 128-byte swizzle of the tensor map), and each
+        // warp's lane 0 stores the warp's 32 x 64 box as soon as the warp has
+        // written it; before the warp writes again, lane 0 waits until its
+        // previous store has read the rows.  Rows past Sq are clipped.
+        uint8_t* srow = smem + L::kEpiOff + tile * L::kEpiTileBytes + r * 128;
+        const uint8_t* wbox = smem + L::kEpiOff + tile * L::kEpiTileBytes + (warp & 3) * 32 * 128;
+        const int wrow0 = w.q_row0 + tile * kBlockM + (warp & 3) * 32;
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          const uint32_t pc = 2u * (uint32_t)units + (uint32_t)h;    // this group's pass count
           uint32_t uq[64];
           __syncwarp();
           tmem_ld32(tO + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&uq[0]));
           tmem_ld32(tO + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&uq[32]));
           tmem_wait_ld();
-          if (pc > 0) ok = warp_wait(&bb.epi_empty[tile], (pc - 1) & 1, kSiteEpiEmpty);   // last store has read it
-          if (!ok) break;
+          if (lane == 0) bulk_wait_read();             // this warp's last store has read its rows
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(srow + ((c ^ (r & 7)) << 4)) = make_uint4(
@@ -695,14 +688,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
                 pack_bf16x2(__uint_as_float(uq[8 * c + 6]) * inv_l, __uint_as_float(uq[8 * c + 7]) * inv_l));
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the TMA store reads it
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bb.epi_full[tile]);
-          if (epi_leader) {
-            if (mbar_wait(&bb.epi_full[tile], pc & 1, kSiteEpiFull) && trow0 < args.Sq) {
-              tma_store_3d(&args.tm_o, stg, h * 64, trow0, bh);
-              bulk_commit();
-              bulk_wait_read();
-            }
-            mbar_arrive(&bb.epi_empty[tile]);
+          if (lane == 0 && wrow0 < args.Sq) {
+            tma_store_3d(&args.tm_o, wbox, h * 64, wrow0, bh);
+            bulk_commit();
           }
         }
       } else {
@@ -739,7 +727,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
         lse[(size_t)bh * args.Sq + row] = lse2 * 0.69314718055994530942f;
       }
     }
-    if (kEpiStage && epi_leader) bulk_wait_all();   // O stores complete before the CTA exits
+    if (kEpiStage && lane == 0) bulk_wait_all();    // O stores complete before the CTA exits
   }
 
   tc_fence_before();

@@ -168,15 +168,16 @@ bool bwd_sizes_ok(int B, int Hq, int Hkv, int Sq, int Sk) {
 
 }  // namespace
 
-// 3-D view (D, S, heads) of a [.., heads, S, D] tensor, box (box_x, 128 rows, 1 head),
+// 3-D view (D, S, heads) of a [.., heads, S, D] tensor, box (box_x, box_rows, 1 head),
 // 128-byte swizzle.  box_x * elt_bytes == 128.
-bool encode_rows_typed(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t heads) {
+bool encode_rows_typed(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows, uint64_t heads,
+                       uint32_t box_rows = kBlockM) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const uint64_t eb = dt == CU_TENSOR_MAP_DATA_TYPE_UINT8 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)heads};
   cuuint64_t strides[2] = {(cuuint64_t)(kHeadDim * eb), (cuuint64_t)(rows * kHeadDim * eb)};
-  cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)kBlockM, 1};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -213,7 +214,8 @@ int attn_fwd_core(const void* q, const void* k, const void* v, void* out, float*
   static thread_local FwdArgs a;   // ~8 KB: kept off the stack
   memset(&a, 0, sizeof(a));
   if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
-  if (!encode_rows(&a.tm_o, out, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+  if (!encode_rows_typed(&a.tm_o, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Sq, (uint64_t)B * Hq, 32))
+    return HATTN_ELAUNCH;
   if (!encode_rows(&a.tm_k[0], k, fp8, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
   if (fp8 && !v16) {
     if (!encode_rows(&a.tm_v[0], v, true, Sk, (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
@@ -351,7 +353,8 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
     // partials are written and no merge pass is needed.
     memset(&a, 0, sizeof(a));
     if (!encode_rows(&a.tm_q, q, fp8, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
-    if (!encode_rows(&a.tm_o, out, false, Sq, (uint64_t)B * Hq)) return HATTN_ELAUNCH;
+    if (!encode_rows_typed(&a.tm_o, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Sq, (uint64_t)B * Hq, 32))
+      return HATTN_ELAUNCH;
     long long tiles = 0;
     for (int i = 0; i < n_blocks; ++i) {
       if (!encode_rows(&a.tm_k[i], k_blocks[i], fp8, blk_len[i], (uint64_t)B * Hkv)) return HATTN_ELAUNCH;
