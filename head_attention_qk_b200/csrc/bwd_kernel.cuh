@@ -19,6 +19,12 @@
 //                     tile) unit loops over KV tiles (ascending).  Per step,
 //                     three MMAs:
 //                       S = Q K^T, dP = dO V^T, dQ += dS K.
+//                     Launched as a programmatic dependent of bwd_dkdv_kernel
+//                     (the two read the same inputs and write different
+//                     outputs): its CTAs start on the SMs whose dK/dV CTAs
+//                     have finished and take units from a global counter,
+//                     heaviest first, so the dK/dV kernel's last, longest
+//                     units overlap dQ work instead of leaving SMs idle.
 //
 // Roles: warps 0-7 compute, warp 8 TMA producer, warp 9 MMA issuer and
 // tensor-memory owner.  Compute warp w owns tile rows 32 (w % 4) .. +31 (its
@@ -56,6 +62,7 @@ struct BwdArgs {
   uint16_t* dq;           // [B,Hq,Sq,D] bf16
   uint16_t* dk;           // [B,Hkv,Sk,D]
   uint16_t* dv;
+  uint32_t* dq_sched;     // dQ kernel: next unit to take (zeroed by the Delta kernel)
   float* dq_acc;          // one-pass backward: fp32 dQ accumulator [B,Hq,Sq,D]
   uint32_t* dq_cnt;       // one-pass backward: contributions added, per (b, q head, query tile)
 };
@@ -68,11 +75,14 @@ enum : int {
 // Delta_r = sum_d dO_rd O_rd.  16 threads share a row (8 values each, one
 // 16-byte load of O and of dO), so a warp reads two whole rows per load; each
 // thread has four rows in flight.  The 16 partial sums meet by a xor
-// butterfly in a fixed order: the result does not depend on the grid.
+// butterfly in a fixed order: the result does not depend on the grid.  It
+// also resets the dQ kernel's unit counter (sched, when given), which runs
+// after it on the same stream.
 constexpr int kDeltaRowsPerCta = 64;
 
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                                        float* __restrict__ delta, long long rows) {
+                                                        float* __restrict__ delta, long long rows, uint32_t* sched) {
+  if (sched && blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   const int sub = threadIdx.x & 15;
   const long long r0 = (long long)blockIdx.x * kDeltaRowsPerCta + (threadIdx.x >> 4);
   const uint4* o4 = reinterpret_cast<const uint4*>(o) + sub;
@@ -191,8 +201,8 @@ __device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, u
   }
 }
 
-// The k-th unit of CTA c among G persistent CTAs (the dK/dV and the dQ
-// kernels): the heaviest-first list is dealt out in snake order (c, then
+// The k-th unit of CTA c among G persistent CTAs (the dK/dV kernel and the
+// one-pass backward): the heaviest-first list is dealt out in snake order (c, then
 // 2G-1-c, then 2G+c, ...), which evens out the causal unit sizes.  Increasing
 // in k, so the first index past the list ends the CTA's loop.
 __device__ __forceinline__ int dq_unit_index(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
@@ -247,8 +257,8 @@ __device__ __forceinline__ DkdvUnit dkdv_unit(const BwdArgs& a, int t) {
   return u;
 }
 
-// Persistent: one CTA per SM walks its units (dealt out in snake order, as in
-// the dQ kernel).  A unit's dK / dV rows are summed over its steps in the same
+// Persistent: one CTA per SM walks its units (dealt out in snake order).  A
+// unit's dK / dV rows are summed over its steps in the same
 // order whichever CTA runs it.  Across units the Q / dO / statistics rings,
 // the S^T / dP^T buffers and every barrier phase continue on one global step
 // count; the next unit's K and V load as soon as the current unit's last S^T
@@ -308,6 +318,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384), dP^T / dS^T [384,512)
+  // The dQ kernel, launched next as a programmatic dependent, needs nothing
+  // this kernel writes: let it start on SMs as soon as they free up.
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
@@ -585,7 +598,7 @@ struct DqSmem {
   static constexpr int kK = kDO + kTileBytesBf16;
   static constexpr int kV = kK + kKStages * kTileBytesBf16;
   static constexpr int kBars = kV + kVStages * kTileBytesBf16;
-  static constexpr int kBytes = kBars + 20 * 8;
+  static constexpr int kBytes = kBars + 24 * 8;   // 22 barriers, the TMEM slot, the 2-entry unit ring
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
@@ -615,19 +628,23 @@ __device__ __forceinline__ DqUnit dq_unit(const BwdArgs& a, int t) {
   return u;
 }
 
-// Persistent: one CTA per SM walks its units.  Every unit's dQ rows are summed
-// over its KV tiles in ascending order by one CTA, as before; only which CTA
-// does a unit depends on the grid.  Across units the K/V ring, the S buffers
-// and every barrier phase continue with a global step count, so the next
-// unit's Q/dO load (once the last S and dP of a unit have read them) and its
-// first S and dP overlap the end of the current unit and its dQ epilogue.
+// Persistent: one CTA per SM walks units taken from a global counter in list
+// order (heaviest first); the producer warp takes them, one ahead, and hands
+// each to the MMA thread and the compute warps through a two-entry ring in
+// shared memory.  Every unit's dQ rows are summed over its KV tiles in
+// ascending order by one CTA; only which CTA does a unit depends on timing.
+// Across units the K/V ring, the S buffers and every barrier phase continue
+// with a global step count, so the next unit's Q/dO load (once the last S and
+// dP of a unit have read them) and its first S and dP overlap the end of the
+// current unit and its dQ epilogue.  Before exiting, the CTA waits for the
+// grid it was launched after (dK/dV) to complete, so the completion of this
+// grid implies that of the whole backward.
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
   using L = DqSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = warp_id(), lane = lane_id();
   const int n_units = ((a.Sq + kTile - 1) / kTile) * a.B * a.Hq;
-  const int cta = blockIdx.x, n_cta = gridDim.x;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
@@ -641,7 +658,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   uint64_t* dq_done = bars + 15;  // a unit's dQ MMAs have completed
   uint64_t* q_empty = bars + 16;  // a unit's last S and dP have read Q and dO
   uint64_t* mma_drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* unit_full = bars + 18;   // [2] ring entry written by the producer
+  uint64_t* unit_empty = bars + 20;  // [2] read by the MMA thread and the 8 compute warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(bars + 23);   // [2]
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -654,6 +674,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     mbar_init(dq_done, 1);
     mbar_init(q_empty, 1);
     mbar_init(mma_drain, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&unit_full[s], 1); mbar_init(&unit_empty[s], 1 + kBwdComputeWarps); }
     fence_barrier_init();
   }
   if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
@@ -663,13 +684,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S / dS buffer 0 [0,128), dP [128,256), dQ [256,384), S / dS buffer 1 [384,512)
   auto s_col = [](int g) { return (g & 1) ? 384u : 0u; };
+  // The k-th unit of this CTA, read from the ring (MMA thread, compute warps):
+  // n_units once the list is exhausted.  The entry is released after reading.
+  auto take_unit = [&](int k, bool whole_warp, int& t) -> bool {
+    const int slot = k & 1;
+    const bool ok = whole_warp ? warp_wait(&unit_full[slot], (k >> 1) & 1, kSiteBwdKV)
+                               : mbar_wait(&unit_full[slot], (k >> 1) & 1, kSiteBwdKV);
+    if (!ok) return false;
+    t = unit_ring[slot];
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || lane == 0) mbar_arrive(&unit_empty[slot]);
+    return true;
+  };
 
   if (warp == 8) {
     if (lane == 0) {
       bool ok = true;
       int ul = 0, gk = 0, gv = 0;   // units started, K and V tiles requested
       for (int k = 0; ok; ++k) {
-        const int t = dq_unit_index(k, cta, n_cta);
+        const int slot = k & 1;
+        if (k >= 2) ok = mbar_wait(&unit_empty[slot], ((k >> 1) - 1) & 1, kSiteBwdStEmpty);
+        if (!ok) break;
+        const uint32_t tu = atomicAdd(a.dq_sched, 1u);     // list order: heaviest first
+        const int t = tu < (uint32_t)n_units ? (int)tu : n_units;
+        unit_ring[slot] = t;
+        mbar_arrive(&unit_full[slot]);                      // releases the ring entry
         if (t >= n_units) break;
         const DqUnit u = dq_unit(a, t);
         // K_0 and V_0 go first: their ring stages free up while the previous
@@ -733,8 +772,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       bool ok = true;
       int ul = 0, g0 = 0;
       for (int k = 0; ok; ++k) {
-        const int t = dq_unit_index(k, cta, n_cta);
-        if (t >= n_units) break;
+        int t = n_units;
+        ok = take_unit(k, false, t);
+        if (!ok || t >= n_units) break;
         const int n = dq_unit(a, t).n_kv;
         ok = mbar_wait(q_full, ul & 1, kSiteBwdKV);
         if (ok) ok = issue_s(g0) && issue_dp(g0);
@@ -770,8 +810,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     bool ok = true;
     int ul = 0, g0 = 0;
     for (int k = 0; ok; ++k) {
-      const int t = dq_unit_index(k, cta, n_cta);
-      if (t >= n_units) break;
+      int t = n_units;
+      ok = take_unit(k, true, t);
+      if (!ok || t >= n_units) break;
       const DqUnit u = dq_unit(a, t);
       const int qi = u.i * kTile + r;
       const bool valid = qi < a.Sq;
@@ -851,6 +892,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   if (warp == 9) { tc_fence_after(); tmem_dealloc(tmem, 512); }
+  if (threadIdx.x == 0) griddep_wait();
 }
 
 // ---------------------------------------------------------------------------- host launch
@@ -858,7 +900,7 @@ bool encode_rows(CUtensorMap* m, const void* base, bool e4m3, uint64_t rows, uin
 
 inline int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                       const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk,
-                      float scale, bool causal, float* delta, int n_sm, cudaStream_t st) {
+                      float scale, bool causal, float* delta, uint32_t* dq_sched, int n_sm, cudaStream_t st) {
   // the shared-memory limits, once per device
   static PerDeviceOnce setup;
   int dev = -1;
@@ -885,6 +927,7 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   a.dq = reinterpret_cast<uint16_t*>(dq);
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
+  a.dq_sched = dq_sched;
   const long long rows = (long long)B * Hq * Sq;
   const long long n_kt = (Sk + kTile - 1) / kTile, nq = (Sq + kTile - 1) / kTile;
   const long long kv_units = n_kt * B * Hkv, dq_units = nq * B * Hq;
@@ -895,9 +938,21 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
       (dq_units + dq_grid - 1) / dq_grid * n_kt >= (1LL << 31))
     return -2;
   bwd_delta_kernel<<<(unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta), 256, 0, st>>>(
-      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows);
+      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows, dq_sched);
   bwd_dkdv_kernel<<<kv_grid, kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
-  bwd_dq_kernel<<<dq_grid, kBwdThreads, DqSmem::kAlloc, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return -5;
+  // dQ as a programmatic dependent of dK/dV (see bwd_dq_kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)dq_grid);
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.dynamicSmemBytes = DqSmem::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, bwd_dq_kernel, a) != cudaSuccess) return -5;
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 

@@ -574,7 +574,7 @@ inline int launch_bwd_onepass(const void* q, const void* k, const void* v, const
   if ((units + grid - 1) / grid * (Hq / Hkv) * nq >= (1LL << 31) || n_kt * 8 >= (1LL << 32)) return -2;
   if (cudaMemsetAsync(a.dq_cnt, 0, ws_bytes - off_cnt, st) != cudaSuccess) return -5;
   bwd_delta_kernel<<<(unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta), 256, 0, st>>>(
-      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows);
+      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows, nullptr);
   if (cudaGetLastError() != cudaSuccess) return -5;
   // cooperative: every CTA is resident, which the ordered dQ adds rely on
   void* params[] = {&a};

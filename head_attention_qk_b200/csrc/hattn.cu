@@ -409,9 +409,15 @@ int attn_fwd_kvblocks(const void* q, const void* const* k_blocks, const void* co
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
+namespace {
+// attn_bwd's workspace: Delta (one fp32 per query row), then at the next
+// 256-byte boundary the dQ kernel's unit counter.
+size_t bwd_sched_offset(int B, int Hq, int Sq) { return ((size_t)B * Hq * Sq * sizeof(float) + 255) & ~(size_t)255; }
+}  // namespace
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Sq) {
   if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
-  return (size_t)B * Hq * Sq * sizeof(float);
+  return bwd_sched_offset(B, Hq, Sq) + 256;
 }
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
@@ -429,8 +435,9 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   if (workspace_bytes < attn_bwd_workspace_size(B, Hq, Sq)) return HATTN_EWORKSPACE;
   const int sms = device_sm_count();
   if (sms <= 0) return HATTN_ELAUNCH;
+  uint32_t* sched = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + bwd_sched_offset(B, Hq, Sq));
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
-                    reinterpret_cast<float*>(workspace), sms, reinterpret_cast<cudaStream_t>(stream));
+                    reinterpret_cast<float*>(workspace), sched, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq) {
@@ -459,12 +466,13 @@ int attn_bwd_onepass(const void* q, const void* k, const void* v, const void* ou
 }
 
 // ---------------------------------------------------------------- allocation-free backward
-// Scratch for attn_bwd_noalloc: the Delta vector (one fp32 per query row) lives
-// in this file-scope device array instead of a caller-provided workspace.
+// Scratch for attn_bwd_noalloc: the Delta vector (one fp32 per query row),
+// followed by the dQ kernel's unit counter (in the last 256 bytes), lives in
+// this file-scope device array instead of a caller-provided workspace.
 // Every GPU that loads the library holds it until the process exits.  In host
 // code the name g_noalloc_delta is only a host-side stand-in; the device
 // address comes from cudaGetSymbolAddress, looked up once per device.
-static __device__ __align__(256) float g_noalloc_delta[HATTN_NOALLOC_MAX_ROWS];
+static __device__ __align__(256) float g_noalloc_delta[HATTN_NOALLOC_MAX_ROWS + 64];
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -504,7 +512,8 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* ou
   // no clearing between calls.
   const int sms = device_sm_count();
   if (sms <= 0) return HATTN_ELAUNCH;
-  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta, sms,
+  uint32_t* sched = reinterpret_cast<uint32_t*>(delta + HATTN_NOALLOC_MAX_ROWS);
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0, delta, sched, sms,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -338,6 +338,17 @@ __device__ __forceinline__ bool wait_counter_geq(const uint32_t* p, uint32_t tar
   }
 }
 
+// Programmatic dependent launch.  launch_dependents: once every thread block
+// of this grid has executed it (or exited), a grid launched after it on the
+// same stream with programmatic stream serialization may start, on SMs as
+// they free up.  wait: blocks until the grids this one was launched after
+// have completed and their memory operations are visible (returns at once
+// for a grid launched without that attribute).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 

@@ -185,7 +185,9 @@ HATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* 
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
              void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of workspace attn_bwd needs: B*Hq*Sq * 4 (the Delta vector). */
+/* Bytes of workspace attn_bwd needs: B*Hq*Sq * 4 (the Delta vector) rounded
+ * up to a multiple of 256, plus 256 (a work counter of the dQ kernel).  Its
+ * contents on entry do not matter. */
 HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
 
 /*
@@ -221,7 +223,7 @@ HATTN_API size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq);
  * counterpart; this is an interface convenience of this library.)
  * Same arguments, results and bitwise reproducibility as attn_bwd, minus the
  * workspace.  The Delta scratch lives in a static device array of
- * HATTN_NOALLOC_MAX_ROWS floats (16 MiB) that every GPU loading the library
+ * HATTN_NOALLOC_MAX_ROWS floats (16 MiB, plus 256 bytes for a work counter) that every GPU loading the library
  * holds until the process exits; this call allocates nothing.
  *  - B*Hq*Sq must be <= HATTN_NOALLOC_MAX_ROWS, else HATTN_EWORKSPACE and
  *    nothing is launched.

@@ -105,7 +105,8 @@ def test_binding_argtypes_match_the_header(h):
 def test_workspace_sizes(h):
     assert h.kvblocks_workspace_size(1, 40, 1560, 128, 21) == 0          # folded in one launch
     assert h.kvblocks_workspace_size(1, 40, 1560, 128, 40) == 40 * 40 * 1560 * 129 * 4
-    assert h.bwd_workspace_size(2, 32, 2048) == 2 * 32 * 2048 * 4
+    assert h.bwd_workspace_size(2, 32, 2048) == 2 * 32 * 2048 * 4 + 256   # Delta, then the dQ unit counter
+    assert h.bwd_workspace_size(1, 1, 3) == 256 + 256
     assert h.kvblocks_workspace_size(0, 1, 1, 128, 1) == 0
 
 
