@@ -82,6 +82,8 @@ constexpr int kDeltaRowsPerCta = 64;
 
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                         float* __restrict__ delta, long long rows, uint32_t* sched) {
+  griddep_wait();                                    // O comes from the grid before (the forward)
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (sched && blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   const int sub = threadIdx.x & 15;
   const long long r0 = (long long)blockIdx.x * kDeltaRowsPerCta + (threadIdx.x >> 4);
@@ -318,8 +320,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: dV [0,128), dK [128,256), S^T / P^T [256,384), dP^T / dS^T [384,512)
-  // The dQ kernel, launched next as a programmatic dependent, needs nothing
-  // this kernel writes: let it start on SMs as soon as they free up.
+  // Launched as a programmatic dependent of the Delta kernel: the setup above
+  // overlaps its end; Delta is read only after it has completed.  The dQ
+  // kernel, launched next the same way, needs nothing this kernel writes: let
+  // it start on SMs as soon as they free up.
+  griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
 
   if (warp == 8) {
@@ -937,21 +942,27 @@ inline int launch_bwd(const void* q, const void* k, const void* v, const void* o
   if ((kv_units + kv_grid - 1) / kv_grid * (Hq / Hkv) * nq >= (1LL << 31) ||
       (dq_units + dq_grid - 1) / dq_grid * n_kt >= (1LL << 31))
     return -2;
-  bwd_delta_kernel<<<(unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta), 256, 0, st>>>(
-      reinterpret_cast<const uint16_t*>(out), reinterpret_cast<const uint16_t*>(dout), delta, rows, dq_sched);
-  bwd_dkdv_kernel<<<kv_grid, kBwdThreads, DkdvSmem::kAlloc, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return -5;
-  // dQ as a programmatic dependent of dK/dV (see bwd_dq_kernel)
+  // Each grid is a programmatic dependent of the one before (see the kernels):
+  // Delta after the forward, dK/dV after Delta, dQ after dK/dV.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)dq_grid);
-  cfg.blockDim = dim3(kBwdThreads);
-  cfg.dynamicSmemBytes = DqSmem::kAlloc;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
+  cfg.attrs = pdl;
   cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)((rows + kDeltaRowsPerCta - 1) / kDeltaRowsPerCta));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, bwd_delta_kernel, reinterpret_cast<const uint16_t*>(out),
+                         reinterpret_cast<const uint16_t*>(dout), delta, rows, dq_sched) != cudaSuccess)
+    return -5;
+  cfg.gridDim = dim3((unsigned)kv_grid);
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.dynamicSmemBytes = DkdvSmem::kAlloc;
+  if (cudaLaunchKernelEx(&cfg, bwd_dkdv_kernel, a) != cudaSuccess) return -5;
+  cfg.gridDim = dim3((unsigned)dq_grid);
+  cfg.dynamicSmemBytes = DqSmem::kAlloc;
   if (cudaLaunchKernelEx(&cfg, bwd_dq_kernel, a) != cudaSuccess) return -5;
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }

@@ -275,6 +275,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *bb.tmem_slot;
+  // Launched as a programmatic dependent of whatever precedes it on the
+  // stream: the setup above overlaps that grid's end, and nothing in global
+  // memory is touched before it has completed.  The grid after this one may
+  // then launch (it waits for this one the same way).
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sRing = smem + L::kRingOff;

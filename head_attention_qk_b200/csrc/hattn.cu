@@ -107,7 +107,19 @@ int launch_fwd_grid(const FwdArgs& a, int grid, cudaStream_t st) {
                fa.numRegs * kFwdThreads >= kRegsNeeded;
       }))
     return HATTN_ELAUNCH;
-  kernel<<<grid, kFwdThreads, L::kAlloc, st>>>(a);
+  // a programmatic dependent of the grid before it on the stream (the kernel
+  // waits for that grid before touching global memory)
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kFwdThreads);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, a) != cudaSuccess) return HATTN_ELAUNCH;
   return cudaGetLastError() == cudaSuccess ? HATTN_OK : HATTN_ELAUNCH;
 }
 
