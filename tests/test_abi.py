@@ -195,6 +195,7 @@ def test_bwd_fails_closed(h):
         return lib.attn_bwd(A, A, A, A, A, A, dq, A, A, 1, 2, 2, Sq, Sk, D, 0.088, causal, ws, wsb, None)
 
     assert call(wsb=need - 4) == -4
+    assert call(wsb=1 * 2 * 128 * 4) == -4           # Delta alone: the dQ unit counter needs its bytes too
     assert call(dq=None) == -1
     assert call(dq=MIS) == -3
     assert call(D=96) == -2
