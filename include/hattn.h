@@ -223,8 +223,9 @@ HATTN_API size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq);
  * counterpart; this is an interface convenience of this library.)
  * Same arguments, results and bitwise reproducibility as attn_bwd, minus the
  * workspace.  The Delta scratch lives in a static device array of
- * HATTN_NOALLOC_MAX_ROWS floats (16 MiB, plus 256 bytes for a work counter) that every GPU loading the library
- * holds until the process exits; this call allocates nothing.
+ * HATTN_NOALLOC_MAX_ROWS floats (16 MiB), followed by 256 bytes for a work
+ * counter, that every GPU loading the library holds until the process
+ * exits; this call allocates nothing.
  *  - B*Hq*Sq must be <= HATTN_NOALLOC_MAX_ROWS, else HATTN_EWORKSPACE and
  *    nothing is launched.
  *  - The first call on each device looks up the array's device address
