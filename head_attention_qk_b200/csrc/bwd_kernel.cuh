@@ -716,6 +716,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         mbar_arrive(&unit_full[slot]);                      // releases the ring entry
         if (t >= n_units) break;
         const DqUnit u = dq_unit(a, t);
+        if (ul > 0) {   // its Q and dO into L2 while the previous unit still holds their buffers
+          for (int x = 0; x < 2; ++x) {
+            tma_prefetch_3d(&a.tm_q, x * 64, u.i * kTile, u.bh);
+            tma_prefetch_3d(&a.tm_do, x * 64, u.i * kTile, u.bh);
+          }
+        }
         // K_0 and V_0 go first: their ring stages free up while the previous
         // unit still runs, before its last S and dP release Q and dO
         for (int jj = 0; jj < u.n_kv && ok; ++jj) {
@@ -812,18 +818,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     const int hc = warp >> 2;                        // column half: keys 64 hc .. 64 hc + 63
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float c = a.scale_log2;
-    bool ok = true;
-    int ul = 0, g0 = 0;
-    for (int k = 0; ok; ++k) {
-      int t = n_units;
-      ok = take_unit(k, true, t);
-      if (!ok || t >= n_units) break;
+    // This thread's row of unit t, and the loads of its LSE and Delta (issued
+    // for the next unit before the current unit's dQ epilogue, which hides
+    // their latency).
+    auto row_of = [&](int t, bool& valid) -> size_t {
       const DqUnit u = dq_unit(a, t);
       const int qi = u.i * kTile + r;
-      const bool valid = qi < a.Sq;
-      const size_t ridx = (size_t)u.bh * a.Sq + (valid ? qi : 0);
-      const float lse2 = valid ? __ldg(&a.lse[ridx]) * 1.4426950408889634f : INFINITY;
-      const float dlt = valid ? __ldg(&a.delta[ridx]) : 0.f;
+      valid = qi < a.Sq;
+      return (size_t)u.bh * a.Sq + (valid ? qi : 0);
+    };
+    auto load_stats = [&](int t, float& lse_raw, float& dlt) {
+      lse_raw = 0.f;
+      dlt = 0.f;
+      if (t >= n_units) return;
+      bool valid;
+      const size_t ridx = row_of(t, valid);
+      if (valid) {
+        lse_raw = __ldg(&a.lse[ridx]);
+        dlt = __ldg(&a.delta[ridx]);
+      }
+    };
+    int ul = 0, g0 = 0;
+    int t = n_units;
+    bool ok = take_unit(0, true, t);
+    float lse_raw, dlt;
+    load_stats(t, lse_raw, dlt);
+    for (int k = 0; ok && t < n_units; ++k) {
+      const DqUnit u = dq_unit(a, t);
+      const int qi = u.i * kTile + r;
+      bool valid;
+      const size_t ridx = row_of(t, valid);
+      const float lse2 = valid ? lse_raw * 1.4426950408889634f : INFINITY;
       const int kv_limit = a.causal ? min(a.Sk - 1, qi + (a.Sk - a.Sq)) : a.Sk - 1;
       for (int jj = 0; jj < u.n_kv && ok; ++jj) {
         const int g = g0 + jj;
@@ -883,6 +908,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         __syncwarp();
         if (lane == 0) mbar_arrive(ds_full);
       }
+      if (!ok) break;
+      // the next unit and its statistics first, then this unit's epilogue
+      int tn = n_units;
+      ok = take_unit(k + 1, true, tn);
+      float lse_next = 0.f, dlt_next = 0.f;
+      if (ok) load_stats(tn, lse_next, dlt_next);
       if (ok) ok = warp_wait(dq_done, ul & 1, kSiteBwdDone);
       if (!ok) break;
       tc_fence_after();
@@ -891,6 +922,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
       store_half_row_bf16(tmem + lane_base + 256 + hc * 64, a.scale, a.dq + ridx * kHeadDim + hc * 64, valid);
       g0 += u.n_kv;
       ++ul;
+      t = tn;
+      lse_raw = lse_next;
+      dlt = dlt_next;
     }
   }
 
