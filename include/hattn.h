@@ -23,6 +23,11 @@
  *  - The caller owns every buffer.  Calls allocate nothing, never synchronise
  *    the host, and enqueue their kernels on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream), so they may be captured into a CUDA graph.
+ *    The attention kernels are launched as programmatic dependents of the
+ *    kernel before them on the stream: their setup may overlap its end, but
+ *    they touch no global memory until it has completed, and the last kernel
+ *    of each call completes only after the call's other kernels, so stream
+ *    order holds for everything the caller enqueues around a call.
  *  - Results are bitwise reproducible: every output element is written by one
  *    thread block, reductions run in a fixed order, and tile sizes do not depend
  *    on B, H or the number of SMs, so a row's result does not change with the
