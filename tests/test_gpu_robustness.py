@@ -15,6 +15,7 @@ import ctypes
 import pytest
 import torch
 
+import workloads
 from parity import LSE_MAX_ABS, O_MAX_ABS, fwd_errors, oracle_fwd
 from workloads import Workload, make_bwd_inputs, make_fwd_inputs, make_kvblock_inputs
 
@@ -90,6 +91,37 @@ def test_cuda_graph_capture_matches_eager(h):
     for a, b in ((out_g, out_e), (dq_g, dq_e), (dk_g, dk_e), (dv_g, dv_e)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(lse_g, lse_e)
+
+
+def test_cuda_graph_llm_step_replays_bitwise(h):
+    # the LLM step (B2 Hq32 Hkv8 S2048 causal, forward + backward) in one graph:
+    # the backward's dQ grid starts while dK/dV still runs and takes its units
+    # from a counter in the workspace that the Delta kernel resets, so replays
+    # queued back to back, with no sync between them, must each start from a
+    # reset counter; every replay equals the eager step bit for bit
+    import workloads
+
+    w = workloads.get("llm_gqa")
+    x = {k: v.cuda() for k, v in make_bwd_inputs(w).items()}
+    out_e, lse_e = h.attn_fwd(x["q"], x["k"], x["v"], causal=True)
+    grads_e = h.attn_bwd(x["q"], x["k"], x["v"], out_e, lse_e, x["dout"], causal=True)
+    torch.cuda.synchronize()
+    ws = torch.empty(h.bwd_workspace_size(w.B, w.Hq, w.Sq), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            out_g, lse_g = h.attn_fwd(x["q"], x["k"], x["v"], causal=True, stream=s)
+            grads_g = h.attn_bwd(x["q"], x["k"], x["v"], out_g, lse_g, x["dout"], causal=True, workspace=ws,
+                                 stream=s)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert h.get_device_error() == 0
+    assert torch.equal(out_g.view(torch.int16), out_e.view(torch.int16)) and torch.equal(lse_g, lse_e)
+    for a, b in zip(grads_g, grads_e):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
 def test_fp8_attn_fwd_allocates_nothing_and_captures(h):
