@@ -22,7 +22,7 @@ HattnError with the library's code for a request it refuses)::
     out_s, lse_s = hattn.attn_fwd_kvblocks(q, [k0, k1, k2], [v0, v1, v2])   # blocks folded in order
 """
 _API = ("BF16", "E4M3", "EXPORTED", "NOALLOC_MAX_ROWS", "HattnError", "attn_bwd", "attn_bwd_noalloc",
-        "attn_bwd_onepass", "bwd_onepass_workspace_size", "attn_fwd",
+        "attn_bwd_onepass", "bwd_onepass_workspace_size", "attn_bwd_dsbuf", "bwd_dsbuf_workspace_size", "attn_fwd",
         "attn_fwd_kvblocks", "bwd_workspace_size", "fwd_workspace_size", "get_device_error", "kvblocks_workspace_size",
         "lib", "quantize_e4m3")
 

@@ -63,6 +63,10 @@ struct BwdArgs {
   uint16_t* dk;           // [B,Hkv,Sk,D]
   uint16_t* dv;
   uint32_t* dq_sched;     // dQ kernel: next unit to take (zeroed by the Delta kernel)
+  // attn_bwd_dsbuf: dS^T tiles written by the dK/dV kernel, [B*Hq][n_kt][nq]
+  // tiles of 128 keys x 128 queries (bf16, 32 KB each, in the blocked layout
+  // of ds_tile_offset); null otherwise
+  uint16_t* ds_buf;
   float* dq_acc;          // one-pass backward: fp32 dQ accumulator [B,Hq,Sq,D]
   uint32_t* dq_cnt;       // one-pass backward: contributions added, per (b, q head, query tile)
 };
@@ -203,6 +207,21 @@ __device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, u
   }
 }
 
+// Element offset of dS^T[key][query] within a stored 128 x 128 tile: 8-key x
+// 8-query core blocks of 128 bytes (keys 16 bytes apart), ordered key-group
+// (8 keys) fastest within a 32-key quarter, then 8-query groups, then 32-query
+// groups, then key quarters:
+//     key = 32 kq + 8 kb + kr, query = 32 qg + 8 q8 + qe
+//     offset = 4096 kq + 1024 qg + 256 q8 + 64 kb + 8 kr + qe.
+// A compute warp (one key quarter, 32 queries) then stores 512 contiguous
+// bytes per instruction, and the tile is the no-swizzle MN-major operand
+// layout of the dQ product (core blocks 512 bytes apart along queries, 128
+// along keys).
+__host__ __device__ constexpr int ds_tile_offset(int key, int query) {
+  return 4096 * (key >> 5) + 1024 * (query >> 5) + 256 * ((query >> 3) & 3) + 64 * ((key >> 3) & 3) +
+         8 * (key & 7) + (query & 7);
+}
+
 // The k-th unit of CTA c among G persistent CTAs (the dK/dV kernel and the
 // one-pass backward): the heaviest-first list is dealt out in snake order (c, then
 // 2G-1-c, then 2G+c, ...), which evens out the causal unit sizes.  Increasing
@@ -277,7 +296,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
   }
   uint8_t* smem = smem_raw;
   const int warp = warp_id(), lane = lane_id();
-  const int n_units = ((a.Sk + kTile - 1) / kTile) * a.B * a.Hkv;
+  const int n_kt = (a.Sk + kTile - 1) / kTile, nq_t = (a.Sq + kTile - 1) / kTile;
+  const int n_units = n_kt * a.B * a.Hkv;
   const int cta = blockIdx.x, n_cta = gridDim.x;
   const int G = a.Hq / a.Hkv;
 
@@ -494,10 +514,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
       const int kj = u.j * kTile + r;
       // key kj is visible to query qi iff kj <= qi + (Sk - Sq)
       const int lim = kj - (a.Sk - a.Sq);            // masked iff qi < lim
+      const bool key_in = kj < a.Sk;
       for (int s = 0; s < u.steps && ok; ++s) {
         const int n = n0 + s;
         const int i = u.i0 + s % u.nqi;
         const int ss = n % L::kStatStages;
+        // dS^T tile (query head of this step, key tile j, query tile i), in elements
+        const size_t ds_tile =
+            a.ds_buf ? ((((size_t)(u.bkv / a.Hkv) * a.Hq + (u.bkv % a.Hkv) * G + s / u.nqi) * n_kt + u.j) * nq_t + i) *
+                           (size_t)(kTile * kTile)
+                     : 0;
         ok = warp_wait(&st_full[ss], (n / L::kStatStages) & 1, kSiteBwdStFull);
         if (!ok) break;
         // LSE (log2 domain) then Delta of the tile's 128 queries
@@ -562,6 +588,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                                                         make_float2(-d4.z, -d4.w)));
             pk[ch][e / 2] = pack_bf16x2(a0.x, a0.y);
             pk[ch][e / 2 + 1] = pack_bf16x2(a1.x, a1.y);
+          }
+          if (a.ds_buf) {
+            // this row's 32 queries of the chunk into the step's dS^T tile,
+            // 8 queries (16 bytes) per store, the warp's 32 rows contiguous;
+            // rows past Sk hold zeros (the dQ product multiplies them by the
+            // zero-filled K rows, and their P may not be finite)
+            uint16_t* base = a.ds_buf + ds_tile + ds_tile_offset(r, ch * 64 + hc * 32);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+              *reinterpret_cast<uint4*>(base + 256 * q8) =
+                  key_in ? make_uint4(pk[ch][4 * q8], pk[ch][4 * q8 + 1], pk[ch][4 * q8 + 2], pk[ch][4 * q8 + 3])
+                         : make_uint4(0u, 0u, 0u, 0u);
           }
           __syncwarp();
           tmem_st16(tP + ch * 64, pk[ch]);             // dS^T over the first 16 of these columns

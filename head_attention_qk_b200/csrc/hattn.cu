@@ -19,6 +19,7 @@
 
 #include "../../include/hattn.h"
 #include "bwd_kernel.cuh"
+#include "bwd_dq_gemm_kernel.cuh"
 #include "bwd_onepass_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "per_device.h"
@@ -450,6 +451,32 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* out, const
   uint32_t* sched = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + bwd_sched_offset(B, Hq, Sq));
   return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
                     reinterpret_cast<float*>(workspace), sched, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_bwd_dsbuf_workspace_size(int B, int Hq, int Sq, int Sk) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0 || Sk <= 0) return 0;
+  size_t off_ds = 0;
+  return dsbuf_workspace_parts(B, Hq, Sq, Sk, &off_ds);
+}
+
+int attn_bwd_dsbuf(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                   float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace) return HATTN_EINVAL;
+  int rc = check_common(B, Hq, Hkv, Sq, D, scale);
+  if (rc) return rc;
+  if (Sk <= 0) return HATTN_EINVAL;
+  if (causal && Sq > Sk) return HATTN_EUNSUPPORTED;
+  if (!bwd_sizes_ok(B, Hq, Hkv, Sq, Sk)) return HATTN_EUNSUPPORTED;
+  const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return HATTN_EALIGN;
+  if (workspace_bytes < attn_bwd_dsbuf_workspace_size(B, Hq, Sq, Sk)) return HATTN_EWORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HATTN_ELAUNCH;
+  const int r = launch_bwd_dsbuf(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, scale, causal != 0,
+                                 workspace, sms, reinterpret_cast<cudaStream_t>(stream));
+  return r == -2 ? HATTN_EUNSUPPORTED : (r ? HATTN_ELAUNCH : HATTN_OK);
 }
 
 size_t attn_bwd_onepass_workspace_size(int B, int Hq, int Sq) {

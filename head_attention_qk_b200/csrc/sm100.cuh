@@ -137,6 +137,15 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int c0, in
                : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes (16-byte aligned, a multiple
+// of 16) from global into this CTA's shared memory, counted on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // 3-D tiled TMA load into this CTA's shared memory; completion is signalled on
 // `bar` as transaction bytes.  The innermost coordinate c0 is always a multiple
 // of 64 elements here (16-byte aligned in bytes).
@@ -226,6 +235,10 @@ __device__ __forceinline__ void mma_f16_ts2(uint32_t d, uint32_t a_tmem, uint32_
 // Halves of a 128-byte-swizzle descriptor (see make_sdesc).
 __host__ __device__ constexpr uint32_t sdesc_hi(uint32_t sbo_bytes) {
   return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+// High half of a no-swizzle descriptor (core blocks of 8 rows x 16 bytes).
+__host__ __device__ constexpr uint32_t sdesc_hi_noswizzle(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14);
 }
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);

@@ -40,6 +40,11 @@ lib.attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i
 lib.attn_bwd_noalloc.restype = _i
 lib.attn_bwd_workspace_size.argtypes = [_i, _i, _i]
 lib.attn_bwd_workspace_size.restype = _sz
+lib.attn_bwd_dsbuf.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz,
+                               _vp]
+lib.attn_bwd_dsbuf.restype = _i
+lib.attn_bwd_dsbuf_workspace_size.argtypes = [_i, _i, _i, _i]
+lib.attn_bwd_dsbuf_workspace_size.restype = _sz
 lib.attn_bwd_onepass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp, _sz,
                                  _vp]
 lib.attn_bwd_onepass.restype = _i
@@ -58,7 +63,7 @@ lib.attn_error_string.restype = ctypes.c_char_p
 
 BF16, E4M3 = 0, 1
 EXPORTED = ("attn_fwd", "attn_fwd_ws", "attn_fwd_workspace_size", "attn_quantize_e4m3", "attn_fwd_kvblocks", "attn_fwd_kvblocks_workspace_size", "attn_bwd",
-            "attn_bwd_workspace_size", "attn_bwd_onepass", "attn_bwd_onepass_workspace_size", "attn_bwd_noalloc",
+            "attn_bwd_workspace_size", "attn_bwd_dsbuf", "attn_bwd_dsbuf_workspace_size", "attn_bwd_onepass", "attn_bwd_onepass_workspace_size", "attn_bwd_noalloc",
             "attn_get_device_error", "attn_selftest_bounded_wait", "attn_selftest_counter_wait", "attn_error_string")
 NOALLOC_MAX_ROWS = 1 << 22
 
@@ -339,6 +344,32 @@ def attn_bwd(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, 
                           _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
                           _nbytes(workspace), _sp(st))
     _check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def bwd_dsbuf_workspace_size(B, Hq, Sq, Sk) -> int:
+    return lib.attn_bwd_dsbuf_workspace_size(B, Hq, Sq, Sk)
+
+
+def attn_bwd_dsbuf(q, k, v, out, lse, dout, causal=False, scale=None, workspace=None, dq=None, dk=None, dv=None,
+                   stream=None):
+    """dQ, dK, dV (bf16) with dS stored in the workspace (O(Sq x Sk) bytes,
+    see bwd_dsbuf_workspace_size): dQ is read back as the product dS K."""
+    B, Hq, Hkv, Sq, Sk, D = _bwd_args(q, k, v, out, lse, dout, dq, dk, dv)
+    dev = _device([("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout), ("dq", dq),
+                   ("dk", dk), ("dv", dv), ("workspace", workspace)])
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev), torch.cuda.stream(st):
+        if workspace is None:
+            workspace = torch.empty(bwd_dsbuf_workspace_size(B, Hq, Sq, Sk), dtype=torch.uint8, device=dev)
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        rc = lib.attn_bwd_dsbuf(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), _ptr(workspace),
+                                _nbytes(workspace), _sp(st))
+    _check(rc, "attn_bwd_dsbuf")
     return dq, dk, dv
 
 

@@ -196,6 +196,30 @@ HATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* 
 HATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Sq);
 
 /*
+ * Backward with dS stored (RL-Kernel PR #319, "What the strict contract
+ * costs": a deterministic mha_bwd holding an O(S^2) workspace).  The same
+ * arguments, layouts and checks as attn_bwd, bf16 only.  The dK/dV pass also
+ * writes every bf16 dS tile it forms into the workspace; dQ is then the
+ * product scale * dS K read back from there (one matrix product per pair of
+ * 128-row tiles instead of attn_bwd's recomputation of S, P and dP: 5 in all
+ * instead of 7), summed over key tiles in ascending order by one thread block
+ * per query tile.  Results are bitwise reproducible and independent of batch
+ * composition and head split; they agree with attn_bwd within the gradient
+ * tolerance, not bitwise (dS is formed from the transposed S).
+ *   workspace: at least attn_bwd_dsbuf_workspace_size(B, Hq, Sq, Sk) bytes:
+ *   Delta, then B*Hq*ceil(Sk/128)*ceil(Sq/128) tiles of 32 KB -- memory that
+ *   grows as Sq x Sk (about 537 MB at B2 Hq32 S2048); its contents on entry do
+ *   not matter.
+ */
+HATTN_API int attn_bwd_dsbuf(const void* q, const void* k, const void* v, const void* out, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_bwd_dsbuf needs (for D = 128); 0 for a size <= 0. */
+HATTN_API size_t attn_bwd_dsbuf_workspace_size(int B, int Hq, int Sq, int Sk);
+
+/*
  * One-pass deterministic backward (RL-Kernel PR #319: deterministic mha_bwd,
  * "What the strict contract costs"): the same dQ, dK, dV as attn_bwd (same
  * arguments and layouts, bf16 only), computed by one kernel that forms each

@@ -27,7 +27,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     syms = declared_symbols()
-    for s in ("attn_fwd", "attn_fwd_kvblocks", "attn_bwd", "attn_fwd_kvblocks_workspace_size",
+    for s in ("attn_fwd", "attn_fwd_kvblocks", "attn_bwd", "attn_bwd_dsbuf", "attn_bwd_dsbuf_workspace_size",
+              "attn_fwd_kvblocks_workspace_size",
               "attn_bwd_workspace_size", "attn_get_device_error", "attn_error_string"):
         assert s in syms
 
@@ -200,6 +201,24 @@ def test_bwd_fails_closed(h):
     assert call(dq=MIS) == -3
     assert call(D=96) == -2
     assert call(causal=1, Sq=256, Sk=128) == -2
+
+
+def test_bwd_dsbuf_fails_closed(h):
+    lib = h.lib
+    need = h.bwd_dsbuf_workspace_size(1, 2, 128, 300)
+    # Delta, then 2 heads x 3 key tiles x 1 query tile of 32 KB
+    assert need >= 2 * 3 * 1 * 32768 + 2 * 128 * 4
+    assert h.bwd_dsbuf_workspace_size(0, 2, 128, 300) == 0
+
+    def call(ws=A, wsb=need, causal=0, Sq=128, Sk=300, D=128, dq=A):
+        return lib.attn_bwd_dsbuf(A, A, A, A, A, A, dq, A, A, 1, 2, 2, Sq, Sk, D, 0.088, causal, ws, wsb, None)
+
+    assert call(wsb=need - 1) == -4
+    assert call(ws=None) == -1
+    assert call(dq=None) == -1
+    assert call(dq=MIS) == -3
+    assert call(D=96) == -2
+    assert call(causal=1, Sq=400, Sk=300) == -2
 
 
 def test_bwd_onepass_fails_closed(h):
