@@ -7,7 +7,10 @@ that is already resident in HBM:
   video      (default) O, LSE = attn_fwd(Q, K, V), B=1 H=40 S=32760 D=128 bf16,
              Q/K RMS-normalised per head -- the video-DiT self-attention;
   fp8        attn_fwd on e4m3 inputs with per-head descales, B=1 H=5 S=75600;
-  llm_gqa    attn_fwd + attn_bwd, B=2 Hq=32 Hkv=8 S=2048 causal;
+  llm_gqa    attn_fwd + attn_bwd_dsbuf (the backward that stores dS in an
+             O(Sq x Sk) workspace), B=2 Hq=32 Hkv=8 S=2048 causal; the same
+             step with the O(S)-memory attn_bwd and with attn_bwd_onepass
+             are sub-results;
   streaming  attn_fwd_kvblocks over 21 blocks of 1560 keys + attn_fwd to 512
              text keys, B=1 H=40 Sq=1560;
   cross      attn_fwd, B=1 H=40 Sq=90000 Sk=512 (long-query cross-attention);
@@ -52,7 +55,10 @@ L2_FLUSH_BYTES = 256 << 20
 WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "video": "video-DiT self-attention fwd (B1 H40 S32760 D128 bf16, Q/K RMS-norm)",
                   "fp8": "fp8 e4m3 attention fwd (B1 H5 S75600 D128, per-head descales)",
-                  "llm_gqa": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16)",
+                  "llm_gqa": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16; backward with stored dS, "
+                             "attn_bwd_dsbuf, 537 MB workspace)",
+                  "llm_gqa_attn_bwd": "LLM GQA causal fwd+bwd (B2 Hq32 Hkv8 S2048 D128 bf16; backward attn_bwd, "
+                                      "O(S) workspace)",
                   "streaming": "streaming block-KV fwd (B1 H40 Sq1560, 21x1560 KV blocks + 512 text keys)",
                   "cross": "long-query cross-attention fwd (B1 H40 Sq90000 Sk512 D128 bf16)",
                   "window": "window/sink KV fwd (B1 H12 Sq4680 Sk51480 D128 bf16)",
@@ -65,7 +71,7 @@ WORKLOAD_NAMES = {"tiny": "tiny self-attention fwd (B1 H2 S256 D128 bf16)",
                   "fp8_streaming": "streaming block-KV fwd over an FP8 e4m3 KV cache (B1 H40 Sq1560, 21x1560 blocks "
                                    "with per-block descales, + 512 e4m3 text keys)"}
 FWD_WORKLOADS = ("video", "fp8", "tiny", "cross", "window", "bf16_75600", "fp8_32760")
-SUB_ONLY = ("fp8_prep", "fp8_noscratch", "fp8_streaming", "llm_gqa_onepass")     # measured as sub-results only
+SUB_ONLY = ("fp8_prep", "fp8_noscratch", "fp8_streaming", "llm_gqa_onepass", "llm_gqa_attn_bwd")   # sub-results only
 KERNEL_SOURCES = ["head_attention_qk_b200/csrc/fwd_kernel.cuh", "head_attention_qk_b200/csrc/sm100.cuh"]
 
 
@@ -202,7 +208,7 @@ class Step:
         self.name = name
         self.h = h
         base = {"fp8_prep": "fp8", "fp8_noscratch": "fp8", "fp8_streaming": "streaming",
-                "llm_gqa_onepass": "llm_gqa"}.get(name, name)
+                "llm_gqa_onepass": "llm_gqa", "llm_gqa_attn_bwd": "llm_gqa"}.get(name, name)
         self.w = workloads.get(base)
         if heads:
             self.w = workloads.get(base, Hq=heads, Hkv=max(1, heads * self.w.Hkv // self.w.Hq))
@@ -221,7 +227,7 @@ class Step:
             self.dtype = w.dtype
             if w.dtype == "e4m3":
                 self.launches = 2          # V widened to fp16, then the attention kernel
-        elif name in ("llm_gqa", "llm_gqa_onepass"):
+        elif name in ("llm_gqa", "llm_gqa_onepass", "llm_gqa_attn_bwd"):
             x = make_bwd_inputs(w)
             self.host = x
             self.x = {k: v.cuda() for k, v in x.items()}
@@ -230,10 +236,13 @@ class Step:
             self.dq = torch.empty_like(self.x["q"])
             self.dk = torch.empty_like(self.x["k"])
             self.dv = torch.empty_like(self.x["v"])
-            wsb = h.bwd_onepass_workspace_size if name == "llm_gqa_onepass" else h.bwd_workspace_size
-            self.ws = torch.empty(wsb(w.B, w.Hq, w.Sq), dtype=torch.uint8, device="cuda")
+            wsb = {"llm_gqa": h.bwd_dsbuf_workspace_size(w.B, w.Hq, w.Sq, w.Sk),
+                   "llm_gqa_onepass": h.bwd_onepass_workspace_size(w.B, w.Hq, w.Sq),
+                   "llm_gqa_attn_bwd": h.bwd_workspace_size(w.B, w.Hq, w.Sq)}[name]
+            self.ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
             self.flops = w.fwd_flops() + w.bwd_flops()
-            self.launches = 4 if name == "llm_gqa" else 3      # fwd; Delta + dK/dV + dQ, or Delta + one pass
+            # fwd; then Delta + dK/dV + dQ product, Delta + dK/dV + dQ, or Delta + one pass
+            self.launches = 3 if name == "llm_gqa_onepass" else 4
             self.dtype = "bf16"
         elif name == "fp8_prep":
             # the step before the fp8 forward: bf16 Q, K, V of the fp8 shape -> e4m3 + descales
@@ -316,10 +325,11 @@ class Step:
         elif self.name == "fp8_prep":
             for i, (t, (c, d)) in enumerate(zip(self.src, self.dst)):
                 h.quantize_e4m3(t, rmsnorm=i < 2, codes=c, descale=d)
-        elif self.name in ("llm_gqa", "llm_gqa_onepass"):
+        elif self.name in ("llm_gqa", "llm_gqa_onepass", "llm_gqa_attn_bwd"):
             x = self.x
             h.attn_fwd(x["q"], x["k"], x["v"], causal=True, out=self.out, lse=self.lse)
-            bwd = h.attn_bwd_onepass if self.name == "llm_gqa_onepass" else h.attn_bwd
+            bwd = {"llm_gqa": h.attn_bwd_dsbuf, "llm_gqa_onepass": h.attn_bwd_onepass,
+                   "llm_gqa_attn_bwd": h.attn_bwd}[self.name]
             bwd(x["q"], x["k"], x["v"], self.out, self.lse, x["dout"], causal=True, workspace=self.ws,
                 dq=self.dq, dk=self.dk, dv=self.dv)
         else:
