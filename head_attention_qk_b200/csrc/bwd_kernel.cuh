@@ -40,6 +40,7 @@
 // dQ/dK/dV accumulators are fp32.
 #pragma once
 
+#include "ds_layout.h"
 #include "fwd_kernel.cuh"
 #include "per_device.h"
 #include "sm100.cuh"
@@ -205,21 +206,6 @@ __device__ __forceinline__ void store_half_row_bf16(uint32_t taddr, float mul, u
       }
     }
   }
-}
-
-// Element offset of dS^T[key][query] within a stored 128 x 128 tile: 8-key x
-// 8-query core blocks of 128 bytes (keys 16 bytes apart), ordered key-group
-// (8 keys) fastest within a 32-key quarter, then 8-query groups, then 32-query
-// groups, then key quarters:
-//     key = 32 kq + 8 kb + kr, query = 32 qg + 8 q8 + qe
-//     offset = 4096 kq + 1024 qg + 256 q8 + 64 kb + 8 kr + qe.
-// A compute warp (one key quarter, 32 queries) then stores 512 contiguous
-// bytes per instruction, and the tile is the no-swizzle MN-major operand
-// layout of the dQ product (core blocks 512 bytes apart along queries, 128
-// along keys).
-__host__ __device__ constexpr int ds_tile_offset(int key, int query) {
-  return 4096 * (key >> 5) + 1024 * (query >> 5) + 256 * ((query >> 3) & 3) + 64 * ((key >> 3) & 3) +
-         8 * (key & 7) + (query & 7);
 }
 
 // The k-th unit of CTA c among G persistent CTAs (the dK/dV kernel and the
